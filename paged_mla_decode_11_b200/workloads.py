@@ -1,0 +1,197 @@
+"""Seeded synthetic inputs for paged MLA decode.
+
+This module only draws inputs: sequence lengths, absorbed queries, the shared pool of
+64-token latent pages and the block table that maps each sequence's logical pages onto
+that pool.  It holds none of the attention arithmetic, so both the CUDA path and the
+fp64 oracle can consume what it produces.
+
+Layouts (FlashMLA call shape, "OpenSourceWeek Day 1 - FlashMLA" section V.2 and the
+q-reshape / params-struct listings of section II):
+
+    q            [batch, s_q, h_q, 576]           bf16  (512 latent + 64 rope columns)
+    k_cache      [num_pages + 1, 64, h_kv, 576]   bf16  (last page = poison page)
+    block_table  [batch, max_pages]               int32 (unused entries -> poison page)
+    cache_seqlens[batch]                          int32
+
+Draw order for one workload, all from one CPU ``torch.Generator`` seeded with ``seed``:
+
+    1. cache_seqlens (uniform integers where the workload draws them)
+    2. q ~ N(0, 1), rounded to bf16
+    3. pool ~ N(0, 1) for the real pages, rounded to bf16; the extra last page = POISON
+    4. outlier rows (only workloads with ``outlier_frac`` > 0): that fraction of the real
+       pool's token rows, chosen by ``randperm``, multiplied by 8 (exact in bf16)
+    5. perm = randperm(num_pages); sequence b's logical page p -> perm[offset_b + p]
+    6. tail slots of every sequence's last page (token >= L_b) set to POISON
+
+POISON is large but finite, so any read of a slot that should be masked shows up as a
+parity failure without producing NaN (0 * NaN would poison a correct P.V product).
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Sequence
+
+import torch
+
+PAGE = 64
+D_QK = 576
+D_V = 512
+POISON = 256.0
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic decode batch.
+
+    ``seqlens`` selects how cache_seqlens is produced:
+      ("fixed", (L0, L1, ...))      given lengths, nothing drawn
+      ("const", L)                  every sequence has length L, nothing drawn
+      ("uniform", lo, hi)           torch.randint(lo, hi + 1)
+      ("skewed", L0, lo, hi)        uniform draw for all, then sequence 0 set to L0
+    """
+
+    name: str
+    batch: int
+    s_q: int
+    h_q: int
+    h_kv: int
+    seqlens: tuple
+    causal: bool = True
+    outlier_frac: float = 0.0
+    softmax_scale: Optional[float] = None  # None -> 576 ** -0.5
+
+    @property
+    def rows_per_kv_head(self) -> int:
+        return self.s_q * self.h_q // self.h_kv
+
+    @property
+    def scale(self) -> float:
+        return self.softmax_scale if self.softmax_scale is not None else D_QK ** -0.5
+
+
+# The five decode workloads, named by what they are.
+TINY = Workload("tiny b2 h16 L{37,130}", 2, 1, 16, 1, ("fixed", (37, 130)))
+MEMORY_BOUND = Workload("memory-bound b64 h16 L~U[1,4096]", 64, 1, 16, 1, ("uniform", 1, 4096))
+COMPUTE_BOUND = Workload("compute-bound b128 h128 L=4096", 128, 1, 128, 1, ("const", 4096))
+CAUSAL_MTP = Workload("causal s_q=2 b32 h128 L~U[2,16384] 5% x8 rows", 32, 2, 128, 1,
+                      ("uniform", 2, 16384), causal=True, outlier_frac=0.05)
+SKEWED = Workload("skewed b132 h64 L0=65536 others~U[256,2048]", 132, 1, 64, 1,
+                  ("skewed", 65536, 256, 2048))
+
+WORKLOADS = {
+    "tiny": TINY,
+    "memory_bound": MEMORY_BOUND,
+    "compute_bound": COMPUTE_BOUND,
+    "causal_mtp": CAUSAL_MTP,
+    "skewed": SKEWED,
+}
+
+
+def _draw_seqlens(w: Workload, g: torch.Generator) -> torch.Tensor:
+    kind = w.seqlens[0]
+    if kind == "fixed":
+        vals = list(w.seqlens[1])
+        if len(vals) != w.batch:
+            raise ValueError("fixed seqlens must list one length per sequence")
+        return torch.tensor(vals, dtype=torch.int32)
+    if kind == "const":
+        return torch.full((w.batch,), int(w.seqlens[1]), dtype=torch.int32)
+    if kind == "uniform":
+        lo, hi = w.seqlens[1], w.seqlens[2]
+        return torch.randint(lo, hi + 1, (w.batch,), generator=g, dtype=torch.int64).to(torch.int32)
+    if kind == "skewed":
+        first, lo, hi = w.seqlens[1], w.seqlens[2], w.seqlens[3]
+        s = torch.randint(lo, hi + 1, (w.batch,), generator=g, dtype=torch.int64).to(torch.int32)
+        s[0] = first
+        return s
+    raise ValueError(f"unknown seqlen rule {kind!r}")
+
+
+def make_inputs(w: Workload, seed: int = 0, max_pages: Optional[int] = None) -> dict:
+    """Draw one workload's inputs on the CPU (see the module docstring for the order).
+
+    Returns a dict with q, k_cache, block_table, cache_seqlens (CPU tensors), plus
+    num_pages (real pages, the poison page has index num_pages), max_pages and the
+    workload's scalar parameters.
+    """
+    g = torch.Generator().manual_seed(seed)
+    seqlens = _draw_seqlens(w, g)
+    if w.h_q % w.h_kv != 0:
+        raise ValueError("h_q must be a multiple of h_kv")
+    if int(seqlens.min()) < 0:
+        raise ValueError("negative sequence length")
+    pages = [(int(L) + PAGE - 1) // PAGE for L in seqlens.tolist()]
+    num_pages = sum(pages)
+    width = max(pages) if pages else 0
+    if max_pages is not None:
+        if max_pages < width:
+            raise ValueError("max_pages smaller than the longest sequence")
+        width = max_pages
+    width = max(width, 1)
+
+    q = torch.randn(w.batch, w.s_q, w.h_q, D_QK, generator=g).to(torch.bfloat16)
+
+    pool = torch.empty(num_pages + 1, PAGE, w.h_kv, D_QK, dtype=torch.bfloat16)
+    pool[:num_pages] = torch.randn(num_pages, PAGE, w.h_kv, D_QK, generator=g).to(torch.bfloat16)
+    pool[num_pages] = POISON
+
+    if w.outlier_frac > 0 and num_pages > 0:
+        n_rows = num_pages * PAGE
+        n_out = int(round(w.outlier_frac * n_rows))
+        rows = torch.randperm(n_rows, generator=g)[:n_out]
+        flat = pool[:num_pages].view(n_rows, w.h_kv, D_QK)
+        flat[rows] = flat[rows] * 8
+
+    perm = torch.randperm(num_pages, generator=g).to(torch.int32)
+    block_table = torch.full((w.batch, width), num_pages, dtype=torch.int32)
+    off = 0
+    for b, n in enumerate(pages):
+        block_table[b, :n] = perm[off:off + n]
+        off += n
+
+    for b, L in enumerate(seqlens.tolist()):
+        if L % PAGE and pages[b] > 0:
+            last = int(block_table[b, pages[b] - 1])
+            pool[last, L % PAGE:] = POISON
+
+    return dict(q=q, k_cache=pool, block_table=block_table, cache_seqlens=seqlens,
+                num_pages=num_pages, max_pages=width, s_q=w.s_q, h_q=w.h_q, h_kv=w.h_kv,
+                causal=w.causal, softmax_scale=w.scale, dv=D_V)
+
+
+def custom(batch: int, s_q: int, h_q: int, h_kv: int, seqlens: Sequence[int],
+           causal: bool = True, scale: Optional[float] = None, outlier_frac: float = 0.0,
+           name: str = "custom") -> Workload:
+    """A workload with given lengths (used for small parity cases and edge cases)."""
+    return Workload(name, batch, s_q, h_q, h_kv, ("fixed", tuple(int(x) for x in seqlens)),
+                    causal=causal, outlier_frac=outlier_frac, softmax_scale=scale)
+
+
+def algorithmic_work(seqlens: Sequence[int], s_q: int, h_q: int, h_kv: int, causal: bool,
+                     d: int = D_QK, dv: int = D_V, batch_meta: bool = True) -> tuple[int, int]:
+    """Algorithmic (bytes, flops) of one decode call.
+
+    Bytes: every valid token's latent row (h_kv heads x d bf16) read once, q read once,
+    out (bf16) and lse (fp32) written once, plus cache_seqlens and the block-table rows
+    actually addressed.  Flops: 2 * (d + dv) per (query row, unmasked key).
+    """
+    nbytes = 0
+    flops = 0
+    for L in seqlens:
+        L = int(L)
+        nbytes += L * h_kv * d * 2
+        nbytes += s_q * h_q * d * 2 + s_q * h_q * dv * 2 + s_q * h_q * 4
+        if batch_meta:
+            nbytes += 4 + ((L + PAGE - 1) // PAGE) * 4
+        for s in range(s_q):
+            n = L - (s_q - 1 - s) if causal else L
+            n = max(n, 0)
+            flops += 2 * (d + dv) * n * h_q
+    return nbytes, flops
+
+
+def whole_page_bytes(seqlens: Sequence[int], h_kv: int, d: int = D_QK) -> int:
+    """Bytes of the whole 64-token pages a kernel streams (tail padding included)."""
+    return sum(((int(L) + PAGE - 1) // PAGE) * PAGE * h_kv * d * 2 for L in seqlens)
+
