@@ -1,0 +1,192 @@
+/*
+ * pagedmla.h -- C ABI of libpagedmla.so: FlashMLA-style decode attention for
+ * Multi-head Latent Attention over a paged latent KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (absorbed-query MLA decode):
+ *   Each cached token stores ONE latent row c of d = 576 bf16 values (512 latent + 64
+ *   rope) per latent head; there is no per-head K or V.  With the query absorbed into
+ *   latent space (q' = W^UK^T q, "DeepSeek FlashMLA practitioner notes", dpshk.com,
+ *   section 2.1) a query head's score against token j is scale * (q' . c_j) over all 576
+ *   columns, and its output is the softmax-weighted sum of the first dv = 512 columns of
+ *   the same rows.  Tokens live in fixed 64-token pages addressed through a block table
+ *   ("OpenSourceWeek Day 1 - FlashMLA", section II.1, and its params-struct listing with
+ *   page_block_size = 64).  Query heads are grouped consecutively per latent head: with
+ *   g = h_q / h_kv, head h reads latent head h / g, and the s_q * g query rows of one
+ *   latent head form one tile (same page, q.view(b, s_q, h_kv, g, d) listing).
+ *
+ *   For row (b, s, h): n = causal ? L_b - (s_q - 1 - s) : L_b keys are visible (the s_q
+ *   new tokens are the last s_q cache entries), and
+ *     out[b, s, h, :] = sum_j softmax_j(scale * q'.c_j) * c_j[0:dv]      (bf16)
+ *     lse[b, h, s]    = ln sum_j exp(scale * q'.c_j)                      (fp32)
+ *   A row with no visible key gets out = 0 and lse = -inf.
+ *
+ * Call sequence (same page, section V.2: get_mla_metadata, then flash_mla_with_kvcache):
+ *   mla_device_sm_count -> mla_num_parts -> mla_get_metadata (device, once per step)
+ *   -> mla_workspace_size -> mla_decode_paged (runs the combine unless told not to).
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" must be device memory of the current CUDA device; the
+ *     caller owns all memory.  The library allocates no device memory.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Nothing synchronises the host except mla_query_status.
+ *   - Return MLA_OK (0) or a negative MLA_ERR_* code; on error nothing was enqueued and
+ *     mla_last_error_string() (thread-local) says why.
+ *   - bf16 tensors are passed as void* holding IEEE bfloat16 bit patterns.
+ */
+#ifndef PAGEDMLA_H_
+#define PAGEDMLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#define MLA_OK 0
+#define MLA_ERR_ARG (-1)          /* bad shape, stride, pointer or value */
+#define MLA_ERR_UNSUPPORTED (-2)  /* d != 576, dv != 512, page != 64, device not sm_100 */
+#define MLA_ERR_WORKSPACE (-3)    /* workspace missing, misaligned or too small */
+#define MLA_ERR_TIMEOUT (-4)      /* a device-side wait hit its time limit */
+#define MLA_ERR_CUDA (-5)         /* a CUDA runtime/driver call failed */
+
+#define MLA_PAGE_SIZE 64          /* tokens per cache page */
+#define MLA_D_QK 576              /* latent row width: 512 latent + 64 rope */
+#define MLA_D_V 512               /* value width: first 512 latent columns */
+#define MLA_TILE_FIELDS 8         /* int32 fields per tile_metadata entry */
+#define MLA_SPLIT_OVERHEAD 5      /* scheduler's fixed cost of one split, in pages */
+#define MLA_ROWS_PER_SM 64        /* query rows one SM serves; sets the part count */
+#define MLA_MAX_BATCH 16384       /* largest batch mla_get_metadata accepts */
+
+#define MLA_FLAG_SKIP_COMBINE 1u  /* mla_decode_paged: leave split partials unmerged */
+
+typedef struct CUstream_st *mla_stream_t; /* identical to cudaStream_t */
+
+/*
+ * mla_device_sm_count -- number of SMs of CUDA device `device` (148 on B200).
+ * Host only.  Errors: MLA_ERR_ARG (null out pointer), MLA_ERR_CUDA.
+ */
+MLA_API int mla_device_sm_count(int device, int *num_sms);
+
+/*
+ * mla_num_parts -- how many split-KV parts the scheduler plans for a device with
+ * `num_sms` SMs:  max(1, num_sms / (h_kv * ceil(rows_per_kv_head / MLA_ROWS_PER_SM))).
+ * rows_per_kv_head = s_q * h_q / h_kv (the second argument of the pages'
+ * get_mla_metadata call).  Host only, pure arithmetic.  Errors: MLA_ERR_ARG.
+ */
+MLA_API int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_parts);
+
+/*
+ * mla_get_metadata -- the split-KV tile scheduler ("OpenSourceWeek Day 1 - FlashMLA",
+ * section V.2: get_mla_metadata(cache_seqlens, s_q*h_q//h_kv, h_kv) -> tile_metadata,
+ * num_splits; the pages print its call only, the plan is this library's specification).
+ *
+ * Spreads sum_b ceil(L_b / 64) pages, plus MLA_SPLIT_OVERHEAD per split, over
+ * `num_parts` parts by a greedy walk: payload = ceil(total / num_parts) + OVERHEAD; each
+ * part finishes whole sequences while they fit and otherwise takes the next
+ * (remaining - OVERHEAD) pages of the current sequence.
+ *
+ *   cache_seqlens  device int32 [batch], each >= 0
+ *   tile_metadata  device int32 [num_parts][8], written:
+ *                  {begin_seq, begin_token, end_seq, end_token, begin_split_ordinal, 0,0,0}
+ *                  the part covers tokens from (begin_seq, begin_token) up to but
+ *                  excluding (end_seq, end_token); tokens are multiples of 64
+ *   num_splits     device int32 [batch + 1], written: prefix sums of the number of parts
+ *                  touching each sequence (num_splits[0] = 0)
+ * rows_per_kv_head and h_kv only enter through num_parts (pass mla_num_parts' result).
+ * Launches one small kernel on `stream`.  Errors: MLA_ERR_ARG (null pointer, batch < 1
+ * or > MLA_MAX_BATCH, num_parts < 1), MLA_ERR_CUDA.  Negative lengths are not detected
+ * on the device; mla_decode_paged's callers must pass lengths >= 0.
+ */
+MLA_API int mla_get_metadata(const int32_t *cache_seqlens, int batch, int num_parts,
+                     int32_t *tile_metadata, int32_t *num_splits, mla_stream_t stream);
+
+/*
+ * mla_workspace_size -- bytes of scratch mla_decode_paged needs: a 256-byte status
+ * block, then fp32 LSE and fp32 normalised outputs of up to (batch + num_parts) split
+ * partials per latent head.  Host only.  Errors: MLA_ERR_ARG.
+ * The workspace must be 256-byte aligned and its first 256 bytes zero before first
+ * use (the library sets a status word there only when a device wait times out, and
+ * mla_query_status clears it again).
+ */
+MLA_API int mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int num_parts, size_t *bytes);
+
+/*
+ * mla_decode_paged -- fused paged MLA decode (see the operation above), following the
+ * pages' flash_mla_with_kvcache(q, k_cache, block_table, cache_seqlens, dv,
+ * tile_metadata, num_splits, causal=True) (same page, section V.2), with softmax_scale
+ * made explicit (the pages' scale is 1/sqrt(d) = 576^-0.5).
+ *
+ *   q              device bf16 [batch][s_q][h_q][d]; q_strides = element strides of its
+ *                  first three dims (the last dim must be contiguous, rows 16-byte
+ *                  aligned)
+ *   k_cache        device bf16 [num_pages][page_size][h_kv][d], contiguous, 16-byte
+ *                  aligned.  Tail slots of a sequence's last page must hold finite values
+ *                  (they are loaded and multiplied by zero weights).
+ *   block_table    device int32 [batch][>= ceil(L_b/64)] with row stride
+ *                  block_table_stride elements; entries used must be in [0, num_pages)
+ *                  (not checked on the device)
+ *   cache_seqlens  device int32 [batch]; L_b >= 0
+ *   dv             must be 512; d must be 576; page_size must be 64
+ *   tile_metadata, num_parts, num_splits: from mla_get_metadata on the same lengths
+ *   softmax_scale  score scale (> 0, finite)
+ *   causal         nonzero: row s sees keys j < L_b - (s_q - 1 - s)
+ *   out            device bf16 [batch][s_q][h_q][dv], contiguous (written)
+ *   lse            device fp32 [batch][h_q][s_q], contiguous (written; natural log)
+ *   workspace      device scratch of mla_workspace_size bytes (see there)
+ *   flags          0, or MLA_FLAG_SKIP_COMBINE to leave the split partials in the
+ *                  workspace for a later mla_combine
+ * Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.  A device
+ * wait that times out (never in correct use) sets the workspace status word; read it
+ * with mla_query_status.
+ */
+MLA_API int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s_q, int h_q,
+                     int d, const void *k_cache, int64_t num_pages, int page_size, int h_kv,
+                     const int32_t *block_table, int64_t block_table_stride,
+                     const int32_t *cache_seqlens, int dv, const int32_t *tile_metadata,
+                     int num_parts, const int32_t *num_splits, float softmax_scale,
+                     int causal, void *out, float *lse, void *workspace,
+                     size_t workspace_bytes, unsigned flags, mla_stream_t stream);
+
+/*
+ * mla_combine -- log-sum-exp merge of split-KV partials: for every sequence with more
+ * than one split and every query row, lse = ln sum_k exp(lse_k) and
+ * out = sum_k exp(lse_k - lse) * o_k (partials with lse_k = -inf weigh nothing).
+ * Reads the partials mla_decode_paged(..., MLA_FLAG_SKIP_COMBINE) left in `workspace`;
+ * writes out/lse rows of split sequences only.  Arguments as in mla_decode_paged.
+ * Errors: MLA_ERR_ARG, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.
+ */
+MLA_API int mla_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv, int dv,
+                int num_parts, const void *workspace, size_t workspace_bytes, void *out,
+                float *lse, mla_stream_t stream);
+
+/*
+ * mla_query_status -- synchronise `stream`, read and clear the workspace status block.
+ * Returns MLA_OK, MLA_ERR_TIMEOUT (a device wait gave up; its results are invalid) or
+ * MLA_ERR_CUDA (the stream reported an error).
+ */
+MLA_API int mla_query_status(void *workspace, mla_stream_t stream);
+
+/*
+ * mla_watchdog_selftest -- launches one CTA that waits on a shared-memory barrier that
+ * nothing ever completes, with the same bounded wait the decode kernel uses and a
+ * limit of `timeout_ns`; the wait gives up, sets the workspace status word and the
+ * kernel returns.  Lets a test check the time-out path without hanging a GPU.
+ * Errors: MLA_ERR_ARG, MLA_ERR_CUDA.
+ */
+MLA_API int mla_watchdog_selftest(void *workspace, uint64_t timeout_ns, mla_stream_t stream);
+
+/* Thread-local description of this thread's last error ("" when none). */
+MLA_API const char *mla_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDMLA_H_ */

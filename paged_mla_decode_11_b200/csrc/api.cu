@@ -1,0 +1,280 @@
+// C ABI of libpagedmla.so (declared in include/pagedmla.h): argument checks, the TMA
+// tensor map of the page pool, workspace carving and kernel launches.  Nothing here
+// allocates device memory or synchronises, except mla_query_status.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "launch.h"
+#include "pagedmla.h"
+
+using namespace pagedmla;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+  return fail(MLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr unsigned long long kWatchdogNs = 2000000000ull;  // 2 s per device-side wait
+constexpr size_t kStatusBytes = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace layout: [status 256 B][lse_accum fp32 splits*h_kv*R][o_accum fp32 ...*512].
+struct WorkspaceLayout {
+  size_t lse_off, o_off, total;
+};
+
+WorkspaceLayout workspace_layout(int batch, int R, int h_kv, int num_parts) {
+  const size_t splits = size_t(batch) + size_t(num_parts);
+  WorkspaceLayout w;
+  w.lse_off = kStatusBytes;
+  w.o_off = align256(w.lse_off + splits * h_kv * R * sizeof(float));
+  w.total = w.o_off + splits * h_kv * R * kDV * sizeof(float);
+  return w;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The kernels are built for sm_100a only; refuse other devices up front.
+int check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(MLA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100 (B200) only",
+                dev, major, minor);
+  return MLA_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Page pool [num_pages * 64 tokens][h_kv][576] bf16 as a 3-D map (columns, latent head,
+// token); one box = 64 columns (128 bytes, 128-byte swizzle) x 1 head x 64 tokens.
+int encode_kv_map(CUtensorMap *map, const void *k_cache, int64_t num_pages, int h_kv) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(h_kv), cuuint64_t(num_pages) * kPage};
+  cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(h_kv) * kD * 2};
+  cuuint32_t box[3] = {64, 1, cuuint32_t(kPage)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k_cache), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return MLA_OK;
+}
+
+int check_common(int batch, int s_q, int h_q, int h_kv, int dv) {
+  if (batch < 1 || s_q < 1 || h_q < 1 || h_kv < 1)
+    return fail(MLA_ERR_ARG, "batch, s_q, h_q and h_kv must be >= 1");
+  if (h_q % h_kv != 0) return fail(MLA_ERR_ARG, "h_q (%d) must be a multiple of h_kv (%d)", h_q, h_kv);
+  if (dv != kDV) return fail(MLA_ERR_UNSUPPORTED, "dv must be %d (got %d)", kDV, dv);
+  const long long R = (long long)s_q * (h_q / h_kv);
+  if (R > (1 << 20)) return fail(MLA_ERR_ARG, "s_q * h_q / h_kv too large");
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mla_last_error_string(void) { return g_last_error.c_str(); }
+
+int mla_device_sm_count(int device, int *num_sms) {
+  if (!num_sms) return fail(MLA_ERR_ARG, "num_sms is null");
+  cudaError_t e = cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(MultiProcessorCount)");
+  return MLA_OK;
+}
+
+int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_parts) {
+  if (!num_parts) return fail(MLA_ERR_ARG, "num_parts is null");
+  if (num_sms < 1 || rows_per_kv_head < 1 || h_kv < 1)
+    return fail(MLA_ERR_ARG, "num_sms, rows_per_kv_head and h_kv must be >= 1");
+  const long long m_blocks = (rows_per_kv_head + MLA_ROWS_PER_SM - 1) / MLA_ROWS_PER_SM;
+  const long long parts = num_sms / (h_kv * m_blocks);
+  *num_parts = parts < 1 ? 1 : int(parts);
+  return MLA_OK;
+}
+
+int mla_get_metadata(const int32_t *cache_seqlens, int batch, int num_parts,
+                     int32_t *tile_metadata, int32_t *num_splits, mla_stream_t stream) {
+  if (!cache_seqlens || !tile_metadata || !num_splits)
+    return fail(MLA_ERR_ARG, "null pointer argument");
+  if (batch < 1 || batch > MLA_MAX_BATCH)
+    return fail(MLA_ERR_ARG, "batch must be in [1, %d] (got %d)", MLA_MAX_BATCH, batch);
+  if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
+  cudaError_t e = launch_metadata(cache_seqlens, batch, num_parts, tile_metadata, num_splits,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "metadata kernel launch");
+  return MLA_OK;
+}
+
+int mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int num_parts, size_t *bytes) {
+  if (!bytes) return fail(MLA_ERR_ARG, "bytes is null");
+  int rc = check_common(batch, s_q, h_q, h_kv, kDV);
+  if (rc) return rc;
+  if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
+  *bytes = workspace_layout(batch, s_q * (h_q / h_kv), h_kv, num_parts).total;
+  return MLA_OK;
+}
+
+int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s_q, int h_q,
+                     int d, const void *k_cache, int64_t num_pages, int page_size, int h_kv,
+                     const int32_t *block_table, int64_t block_table_stride,
+                     const int32_t *cache_seqlens, int dv, const int32_t *tile_metadata,
+                     int num_parts, const int32_t *num_splits, float softmax_scale,
+                     int causal, void *out, float *lse, void *workspace,
+                     size_t workspace_bytes, unsigned flags, mla_stream_t stream) {
+  if (!q || !q_strides || !k_cache || !block_table || !cache_seqlens || !tile_metadata ||
+      !num_splits || !out || !lse)
+    return fail(MLA_ERR_ARG, "null pointer argument");
+  int rc = check_common(batch, s_q, h_q, h_kv, dv);
+  if (rc) return rc;
+  if (d != kD) return fail(MLA_ERR_UNSUPPORTED, "d must be %d (got %d)", kD, d);
+  if (page_size != kPage) return fail(MLA_ERR_UNSUPPORTED, "page_size must be %d (got %d)", kPage, page_size);
+  if (num_pages < 1 || num_pages > (int64_t(1) << 25))
+    return fail(MLA_ERR_ARG, "num_pages must be in [1, 2^25]");
+  if (block_table_stride < 1) return fail(MLA_ERR_ARG, "block_table_stride must be >= 1");
+  if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(MLA_ERR_ARG, "softmax_scale must be positive and finite");
+  if (flags & ~MLA_FLAG_SKIP_COMBINE) return fail(MLA_ERR_ARG, "unknown flags 0x%x", flags);
+  for (int i = 0; i < 3; ++i)
+    if (q_strides[i] < 0 || q_strides[i] % 8 != 0)
+      return fail(MLA_ERR_ARG, "q strides must be non-negative multiples of 8 elements");
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return fail(MLA_ERR_ARG, "q, k_cache and out must be 16-byte aligned, lse 4-byte aligned");
+  rc = check_device();
+  if (rc) return rc;
+
+  const int g = h_q / h_kv, R = s_q * g;
+  const WorkspaceLayout wl = workspace_layout(batch, R, h_kv, num_parts);
+  if (!workspace) return fail(MLA_ERR_WORKSPACE, "workspace is null");
+  if (!aligned(workspace, 256)) return fail(MLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (workspace_bytes < wl.total)
+    return fail(MLA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, wl.total);
+
+  CUtensorMap map;
+  rc = encode_kv_map(&map, k_cache, num_pages, h_kv);
+  if (rc) return rc;
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.q_sb = q_strides[0];
+  p.q_ss = q_strides[1];
+  p.q_sh = q_strides[2];
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.g = g;
+  p.R = R;
+  p.block_table = block_table;
+  p.bt_stride = block_table_stride;
+  p.seqlens = cache_seqlens;
+  p.tile_md = tile_metadata;
+  p.num_parts = num_parts;
+  p.num_splits = num_splits;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.lse_accum = reinterpret_cast<float *>(ws + wl.lse_off);
+  p.o_accum = reinterpret_cast<float *>(ws + wl.o_off);
+  p.status = reinterpret_cast<int *>(ws);
+  p.watchdog_ns = kWatchdogNs;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_decode_mma(map, p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  if (!(flags & MLA_FLAG_SKIP_COMBINE)) {
+    e = launch_combine(num_splits, batch, s_q, h_q, h_kv, p.lse_accum, p.o_accum, p.out, lse, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+  }
+  return MLA_OK;
+}
+
+int mla_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv, int dv,
+                int num_parts, const void *workspace, size_t workspace_bytes, void *out,
+                float *lse, mla_stream_t stream) {
+  if (!num_splits || !out || !lse) return fail(MLA_ERR_ARG, "null pointer argument");
+  int rc = check_common(batch, s_q, h_q, h_kv, dv);
+  if (rc) return rc;
+  if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
+  if (!aligned(out, 16) || !aligned(lse, 4)) return fail(MLA_ERR_ARG, "out must be 16-byte aligned");
+  const int R = s_q * (h_q / h_kv);
+  const WorkspaceLayout wl = workspace_layout(batch, R, h_kv, num_parts);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < wl.total)
+    return fail(MLA_ERR_WORKSPACE, "workspace missing, misaligned or smaller than %zu bytes", wl.total);
+  const uint8_t *ws = static_cast<const uint8_t *>(workspace);
+  cudaError_t e = launch_combine(num_splits, batch, s_q, h_q, h_kv,
+                                 reinterpret_cast<const float *>(ws + wl.lse_off),
+                                 reinterpret_cast<const float *>(ws + wl.o_off),
+                                 static_cast<__nv_bfloat16 *>(out), lse,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+  return MLA_OK;
+}
+
+int mla_query_status(void *workspace, mla_stream_t stream) {
+  if (!workspace) return fail(MLA_ERR_ARG, "workspace is null");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int status = 0;
+  e = cudaMemcpy(&status, workspace, sizeof status, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the workspace status");
+  if (status != 0) {
+    e = cudaMemset(workspace, 0, sizeof status);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace status");
+    if (status & kStatusTimeout)
+      return fail(MLA_ERR_TIMEOUT, "a device-side wait timed out; results of that call are invalid");
+  }
+  return MLA_OK;
+}
+
+int mla_watchdog_selftest(void *workspace, uint64_t timeout_ns, mla_stream_t stream) {
+  if (!workspace || !aligned(workspace, 256)) return fail(MLA_ERR_ARG, "workspace null or misaligned");
+  if (timeout_ns == 0 || timeout_ns > 10ull * 1000000000ull)
+    return fail(MLA_ERR_ARG, "timeout_ns must be in (0, 10 s]");
+  cudaError_t e = launch_watchdog_selftest(static_cast<int *>(workspace), timeout_ns,
+                                           reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "watchdog self-test launch");
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+// Log-sum-exp combine of split-KV partials (the method's merge of the partial results
+// of one sequence's splits): lse = ln sum_k exp(lse_k), out = sum_k exp(lse_k - lse) o_k.
+//
+// One warp per (sequence, latent head, query row); sequences with a single split are
+// skipped (the decode kernel wrote them directly).  Each lane owns 16 of the 512 value
+// columns as four float4s strided 128 apart, so every warp-wide access covers 512
+// contiguous bytes.
+#include "launch.h"
+
+namespace pagedmla {
+
+constexpr int kCombineWarps = 8;
+
+__global__ void __launch_bounds__(kCombineWarps * 32)
+    combine_kernel(const int32_t *__restrict__ num_splits, int s_q, int h_q, int h_kv, int R,
+                   const float *__restrict__ lse_accum, const float *__restrict__ o_accum,
+                   __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+  const int b = blockIdx.x, kvh = blockIdx.z;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int row = blockIdx.y * kCombineWarps + warp;
+  const int ns0 = num_splits[b];
+  const int n = num_splits[b + 1] - ns0;
+  if (n <= 1 || row >= R) return;
+  const int g = h_q / h_kv;
+  const int64_t stride = int64_t(h_kv) * R;  // between consecutive splits
+  const int64_t base = (int64_t(ns0) * h_kv + kvh) * R + row;
+
+  float mx = -INFINITY;
+  for (int k = lane; k < n; k += 32) mx = fmaxf(mx, lse_accum[base + k * stride]);
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+  if (mx != -INFINITY)
+    for (int k = lane; k < n; k += 32) sum += expf(lse_accum[base + k * stride] - mx);
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float tot = mx == -INFINITY ? -INFINITY : mx + logf(sum);
+
+  float4 acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tot != -INFINITY) {
+    for (int k = 0; k < n; ++k) {
+      const float w = expf(lse_accum[base + k * stride] - tot);
+      const float4 *src = reinterpret_cast<const float4 *>(o_accum + (base + k * stride) * kDV);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = src[lane + 32 * i];
+        acc[i].x += w * v.x;
+        acc[i].y += w * v.y;
+        acc[i].z += w * v.z;
+        acc[i].w += w * v.w;
+      }
+    }
+  }
+  const int s = row / g, h = kvh * g + row % g;
+  __nv_bfloat16 *dst = out + ((int64_t(b) * s_q + s) * h_q + h) * kDV;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint2 v;
+    v.x = pack_bf16x2(acc[i].x, acc[i].y);
+    v.y = pack_bf16x2(acc[i].z, acc[i].w);
+    *reinterpret_cast<uint2 *>(dst + 4 * (lane + 32 * i)) = v;
+  }
+  if (lane == 0) lse[(int64_t(b) * h_q + h) * s_q + s] = tot;
+}
+
+cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,
+                           const float *lse_accum, const float *o_accum, __nv_bfloat16 *out,
+                           float *lse, cudaStream_t stream) {
+  const int R = s_q * (h_q / h_kv);
+  dim3 grid(batch, (R + kCombineWarps - 1) / kCombineWarps, h_kv);
+  combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(num_splits, s_q, h_q, h_kv, R, lse_accum,
+                                                          o_accum, out, lse);
+  return cudaGetLastError();
+}
+
+// A CTA that waits on a barrier nothing completes, with the decode kernels' bounded
+// wait; the wait gives up after timeout_ns, records the time-out and returns.
+__global__ void watchdog_selftest_kernel(int *status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, status, timeout_ns);
+  __syncthreads();
+}
+
+cudaError_t launch_watchdog_selftest(int *status, unsigned long long timeout_ns, cudaStream_t stream) {
+  watchdog_selftest_kernel<<<1, 32, 0, stream>>>(status, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace pagedmla

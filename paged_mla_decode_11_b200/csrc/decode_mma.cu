@@ -1,0 +1,367 @@
+// Paged MLA decode, warp-MMA variant (mma.sync m16n8k16 bf16, fp32 accumulate).
+//
+// One CTA per (split-KV part, 16- or 64-row block of query rows, latent head).  A
+// producer warp streams whole 64-token latent pages (64 x 576 bf16 = 73,728 B) from the
+// paged cache into a two-stage shared-memory ring with TMA (128-byte swizzle), each
+// page addressed through block_table ("OpenSourceWeek Day 1 - FlashMLA", section II.1:
+// fixed 64-token blocks).  Consumer warps compute per page
+//     S = scale * Q K^T over all 576 columns (absorbed-query score, dpshk.com notes 2.1)
+//     online softmax: running max m, running sum l, O <- O * 2^(m_old - m_new)
+//     O += P V with V = the page's first 512 columns                (same notes, 2.2)
+// and write either the final bf16 output and natural-log LSE or, when the scheduler
+// split the sequence, an fp32 partial (O / l, lse) for the log-sum-exp combine.
+//
+// Warp layout: BM / 16 row groups x DVS value slices.  In a row group the DVS warps
+// split the 64 keys of S (NK = 64 / DVS each) and the 512 value columns of O
+// (NDV = 512 / DVS each); the row maximum and the P tile are exchanged through shared
+// memory, the row sums only once per segment.
+#include "common.cuh"
+#include "launch.h"
+
+namespace pagedmla {
+
+template <int BM, int DVS>
+struct MmaTile {
+  static constexpr int RG = BM / 16;
+  static constexpr int NCW = RG * DVS;      // consumer warps
+  static constexpr int kThreads = (NCW + 1) * 32;
+  static constexpr int NK = kPage / DVS;    // keys of S per warp
+  static constexpr int NT = NK / 8;         // 8-key n-tiles of S per warp
+  static constexpr int NDV = kDV / DVS;     // value columns per warp
+  static constexpr int NO = NDV / 8;        // 8-column n-tiles of O per warp
+  static constexpr int kStages = 2;
+  static constexpr int kQBlock = BM * 128;  // one 64-column block of the Q tile
+  static constexpr int kOffQ = kStages * kPageBytes;
+  static constexpr int kOffP = kOffQ + kColBlocks * kQBlock;
+  static constexpr int kOffRed = kOffP + BM * 128;
+  static constexpr int kRedFloats = RG * DVS * 16;
+  static constexpr int kOffBar = kOffRed + 2 * kRedFloats * 4;
+  static constexpr int kOffAbort = kOffBar + 2 * kStages * 8;
+  static constexpr int kSmemBytes = kOffAbort + 16 + 1024;  // + slack for 1 KB alignment
+  static_assert(NT >= 1 && (NT == 1 || NT % 2 == 0), "S tiling");
+  static_assert(NO % 2 == 0, "O tiling");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+// Last key (exclusive) any row of m-block `mb` may see: causal rows see fewer keys.
+__device__ __forceinline__ int block_visible_end(const DecodeParams &p, int L, int mb, int BM) {
+  if (!p.causal) return L;
+  const int last_row = min(p.R - 1, mb * BM + BM - 1);
+  return L - (p.s_q - 1 - last_row / p.g);
+}
+
+template <int BM, int DVS>
+__global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeParams p) {
+  using T = MmaTile<BM, DVS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int part = blockIdx.x, mb = blockIdx.y, kvh = blockIdx.z;
+  const uint32_t full_bar = smem_u32(smem + T::kOffBar);
+  const uint32_t empty_bar = full_bar + 8 * T::kStages;
+  volatile int *abort = reinterpret_cast<volatile int *>(smem + T::kOffAbort);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < T::kStages; ++s) {
+      mbar_init(full_bar + 8 * s, 1);
+      mbar_init(empty_bar + 8 * s, T::NCW);
+    }
+    *abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const PartCursor pc = load_part(p.tile_md, part);
+
+  if (warp == T::NCW) {
+    // ---------------- producer warp: page gather through block_table ----------------
+    if (lane == 0) prefetch_tensormap(&kv_map);
+    int it = 0;
+    int last_it[T::kStages];
+#pragma unroll
+    for (int s = 0; s < T::kStages; ++s) last_it[s] = -1;
+    bool ok = true;
+    for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
+      const int L = p.seqlens[seq];
+      const int t0 = seq == pc.bi ? pc.bt : 0;
+      const int t1 = min(seq == pc.ei ? pc.et : L, block_visible_end(p, L, mb, BM));
+      const int npages = t1 > t0 ? (t1 - t0 + kPage - 1) / kPage : 0;
+      const int32_t *bt_row = p.block_table + (int64_t)seq * p.bt_stride + t0 / kPage;
+      for (int base = 0; ok && base < npages; base += 32) {
+        const int mine = base + lane < npages ? bt_row[base + lane] : 0;
+        const int cnt = min(32, npages - base);
+        for (int i = 0; i < cnt; ++i) {
+          const int phys = __shfl_sync(0xffffffffu, mine, i);
+          const int s = it % T::kStages;
+          const uint32_t ph = (it / T::kStages) & 1;
+          int good = 1;
+          if (lane == 0) {
+            if (!mbar_wait(empty_bar + 8 * s, ph ^ 1, abort, p.status, p.watchdog_ns)) {
+              good = 0;
+            } else {
+              mbar_arrive_expect_tx(full_bar + 8 * s, kPageBytes);
+              const uint32_t dst = smem_u32(smem) + s * kPageBytes;
+#pragma unroll
+              for (int c = 0; c < kColBlocks; ++c)
+                tma_load_3d(dst + c * kPageBlockBytes, &kv_map, full_bar + 8 * s, c * 64, kvh,
+                            phys * kPage);
+              last_it[s] = it;
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, good, 0) != 0;
+          if (!ok) break;
+          ++it;
+        }
+      }
+    }
+    // Wait (bounded) until every copy this warp issued has landed before the CTA exits.
+    if (lane == 0) {
+      int never = 0;
+      for (int s = 0; s < T::kStages; ++s)
+        if (last_it[s] >= 0)
+          mbar_wait(full_bar + 8 * s, (last_it[s] / T::kStages) & 1, &never, p.status,
+                    p.watchdog_ns);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- consumer warps ----------------
+    const int rg = warp / DVS, wd = warp % DVS;
+    const int g4 = lane / 4, c4 = lane % 4;
+    const uint32_t sPages = smem_u32(smem);
+    const uint32_t sQ = smem_u32(smem + T::kOffQ);
+    const uint32_t sP = smem_u32(smem + T::kOffP);
+    float *red_max = reinterpret_cast<float *>(smem + T::kOffRed);
+    float *red_sum = red_max + T::kRedFloats;
+    const int rows[2] = {mb * BM + rg * 16 + g4, mb * BM + rg * 16 + g4 + 8};
+    const int group_bar = 1 + rg, all_bar = 1 + T::RG;
+    const int tid = threadIdx.x;
+    int it = 0;
+    bool ok = true;
+
+    for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
+      const int L = p.seqlens[seq];
+      const int t0 = seq == pc.bi ? pc.bt : 0;
+      const int t1 = min(seq == pc.ei ? pc.et : L, block_visible_end(p, L, mb, BM));
+      const int npages = t1 > t0 ? (t1 - t0 + kPage - 1) / kPage : 0;
+      int lim[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = rows[r];
+        lim[r] = row < p.R ? min(t1, p.causal ? L - (p.s_q - 1 - row / p.g) : L) : -1;
+      }
+
+      // Q tile of this sequence: rows mb*BM.., all 576 columns, 128-byte swizzled.
+      named_bar_sync(all_bar, T::NCW * 32);
+      for (int idx = tid; idx < BM * 72; idx += T::NCW * 32) {
+        const int row = idx / 72, ch = idx % 72;
+        const int r = mb * BM + row;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < p.R) {
+          const int s = r / p.g, h = kvh * p.g + r % p.g;
+          v = __ldg(reinterpret_cast<const uint4 *>(p.q + (int64_t)seq * p.q_sb +
+                                                    (int64_t)s * p.q_ss + (int64_t)h * p.q_sh) +
+                    ch);
+        }
+        *reinterpret_cast<uint4 *>(smem + T::kOffQ + (ch / 8) * T::kQBlock + sw128(row, ch % 8)) = v;
+      }
+      named_bar_sync(all_bar, T::NCW * 32);
+
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      float o[T::NO][4];
+#pragma unroll
+      for (int j = 0; j < T::NO; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+
+      for (int pg = 0; pg < npages; ++pg, ++it) {
+        const int s = it % T::kStages;
+        const uint32_t ph = (it / T::kStages) & 1;
+        if (!mbar_wait(full_bar + 8 * s, ph, abort, p.status, p.watchdog_ns)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sK = sPages + s * kPageBytes;
+
+        // ---- S = Q K^T over the warp's NK keys ----
+        float sc[T::NT][4];
+#pragma unroll
+        for (int t = 0; t < T::NT; ++t) sc[t][0] = sc[t][1] = sc[t][2] = sc[t][3] = 0.f;
+        if constexpr (T::NT == 1) {
+#pragma unroll 2
+          for (int kk = 0; kk < kD / 16; kk += 2) {
+            uint32_t a0[4], a1[4], b[4];
+            const int cb = kk / 4;
+            const int qr = rg * 16 + (lane % 16);
+            ldsm_x4(sQ + cb * T::kQBlock + sw128(qr, (kk % 4) * 2 + lane / 16), a0[0], a0[1], a0[2], a0[3]);
+            ldsm_x4(sQ + cb * T::kQBlock + sw128(qr, ((kk + 1) % 4) * 2 + lane / 16), a1[0], a1[1], a1[2], a1[3]);
+            ldsm_x4(sK + cb * kPageBlockBytes + sw128(wd * 8 + (lane % 8), (kk % 4) * 2 + lane / 8),
+                    b[0], b[1], b[2], b[3]);
+            mma_bf16_16816(sc[0], a0, b[0], b[1]);
+            mma_bf16_16816(sc[0], a1, b[2], b[3]);
+          }
+        } else {
+#pragma unroll 2
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            uint32_t a[4];
+            const int cb = kk / 4;
+            ldsm_x4(sQ + cb * T::kQBlock + sw128(rg * 16 + (lane % 16), (kk % 4) * 2 + lane / 16),
+                    a[0], a[1], a[2], a[3]);
+#pragma unroll
+            for (int np = 0; np < T::NT / 2; ++np) {
+              uint32_t b[4];
+              const int key = wd * T::NK + np * 16 + (lane % 8) + (lane / 16) * 8;
+              ldsm_x4(sK + cb * kPageBlockBytes + sw128(key, (kk % 4) * 2 + (lane / 8) % 2), b[0],
+                      b[1], b[2], b[3]);
+              mma_bf16_16816(sc[2 * np], a, b[0], b[1]);
+              mma_bf16_16816(sc[2 * np + 1], a, b[2], b[3]);
+            }
+          }
+        }
+
+        // ---- mask, scale to the log2 domain, row maximum across the row group ----
+        const int key_base = (t0 / kPage + pg) * kPage + wd * T::NK;
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int t = 0; t < T::NT; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = e / 2;
+            const int key = key_base + t * 8 + c4 * 2 + (e & 1);
+            const float v = key < lim[r] ? sc[t][e] * p.scale_log2 : -INFINITY;
+            sc[t][e] = v;
+            mx[r] = fmaxf(mx[r], v);
+          }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+        }
+        if (c4 == 0) {
+          red_max[(rg * DVS + wd) * 16 + g4] = mx[0];
+          red_max[(rg * DVS + wd) * 16 + g4 + 8] = mx[1];
+        }
+        named_bar_sync(group_bar, DVS * 32);
+        float alpha[2], base[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          float mn = m[r];
+#pragma unroll
+          for (int w = 0; w < DVS; ++w) mn = fmaxf(mn, red_max[(rg * DVS + w) * 16 + g4 + 8 * r]);
+          base[r] = mn == -INFINITY ? 0.f : mn;
+          alpha[r] = fast_exp2(m[r] - base[r]);   // m = -inf -> 0
+          m[r] = mn;
+        }
+
+        // ---- P = 2^(S - m) -> bf16 tile in shared memory; partial row sums ----
+        float ps[2] = {0.f, 0.f};
+#pragma unroll
+        for (int t = 0; t < T::NT; ++t) {
+          const float p0 = fast_exp2(sc[t][0] - base[0]), p1 = fast_exp2(sc[t][1] - base[0]);
+          const float p2 = fast_exp2(sc[t][2] - base[1]), p3 = fast_exp2(sc[t][3] - base[1]);
+          ps[0] += p0 + p1;
+          ps[1] += p2 + p3;
+          const int kl = wd * T::NK + t * 8 + c4 * 2;
+          const uint32_t off = (kl % 8) * 2;
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + sw128(rg * 16 + g4, kl / 8) + off),
+                       "r"(pack_bf16x2(p0, p1)));
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(sP + sw128(rg * 16 + g4 + 8, kl / 8) + off),
+                       "r"(pack_bf16x2(p2, p3)));
+        }
+        l[0] = l[0] * alpha[0] + ps[0];
+        l[1] = l[1] * alpha[1] + ps[1];
+        named_bar_sync(group_bar, DVS * 32);
+
+        // ---- O = O * alpha + P V over the warp's NDV value columns ----
+#pragma unroll
+        for (int j = 0; j < T::NO; ++j) {
+          o[j][0] *= alpha[0];
+          o[j][1] *= alpha[0];
+          o[j][2] *= alpha[1];
+          o[j][3] *= alpha[1];
+        }
+#pragma unroll
+        for (int ks = 0; ks < kPage / 16; ++ks) {
+          uint32_t a[4];
+          ldsm_x4(sP + sw128(rg * 16 + (lane % 16), ks * 2 + lane / 16), a[0], a[1], a[2], a[3]);
+          const int key = ks * 16 + (lane % 8) + ((lane / 8) % 2) * 8;
+#pragma unroll
+          for (int jp = 0; jp < T::NO / 2; ++jp) {
+            const int dv0 = wd * T::NDV + jp * 16;
+            uint32_t b[4];
+            ldsm_x4_t(sK + (dv0 / 64) * kPageBlockBytes + sw128(key, (dv0 % 64) / 8 + lane / 16),
+                      b[0], b[1], b[2], b[3]);
+            mma_bf16_16816(o[2 * jp], a, b[0], b[1]);
+            mma_bf16_16816(o[2 * jp + 1], a, b[2], b[3]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar + 8 * s);
+      }
+      if (!ok) break;
+
+      // ---- epilogue: total row sums, then final output or split partial ----
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+        l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+      }
+      if (c4 == 0) {
+        red_sum[(rg * DVS + wd) * 16 + g4] = l[0];
+        red_sum[(rg * DVS + wd) * 16 + g4 + 8] = l[1];
+      }
+      named_bar_sync(group_bar, DVS * 32);
+      const int ns0 = p.num_splits[seq];
+      const int nsplit = p.num_splits[seq + 1] - ns0;
+      const int ord = seq == pc.bi ? pc.bord : 0;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = rows[r];
+        if (row >= p.R) continue;
+        float lt = 0.f;
+#pragma unroll
+        for (int w = 0; w < DVS; ++w) lt += red_sum[(rg * DVS + w) * 16 + g4 + 8 * r];
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float lse_v = lt > 0.f ? (m[r] + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+        if (nsplit == 1) {
+          const int s = row / p.g, h = kvh * p.g + row % p.g;
+          __nv_bfloat16 *orow = p.out + (((int64_t)seq * p.s_q + s) * p.h_q + h) * kDV;
+#pragma unroll
+          for (int j = 0; j < T::NO; ++j) {
+            const int dv = wd * T::NDV + j * 8 + c4 * 2;
+            *reinterpret_cast<uint32_t *>(orow + dv) =
+                pack_bf16x2(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
+          }
+          if (wd == 0 && c4 == 0) p.lse[((int64_t)seq * p.h_q + h) * p.s_q + s] = lse_v;
+        } else {
+          const int64_t sidx = ((int64_t)(ns0 + ord) * p.h_kv + kvh) * p.R + row;
+          float *orow = p.o_accum + sidx * kDV;
+#pragma unroll
+          for (int j = 0; j < T::NO; ++j) {
+            const int dv = wd * T::NDV + j * 8 + c4 * 2;
+            *reinterpret_cast<float2 *>(orow + dv) = make_float2(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
+          }
+          if (wd == 0 && c4 == 0) p.lse_accum[sidx] = lse_v;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+template <int BM, int DVS>
+static cudaError_t launch_mma(const CUtensorMap &map, const DecodeParams &p, int m_blocks,
+                              cudaStream_t stream) {
+  using T = MmaTile<BM, DVS>;
+  auto kern = decode_mma_kernel<BM, DVS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.num_parts, m_blocks, p.h_kv);
+  kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(map, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_mma(const CUtensorMap &map, const DecodeParams &p, cudaStream_t stream) {
+  if (p.R <= 16) return launch_mma<16, 8>(map, p, 1, stream);
+  return launch_mma<64, 2>(map, p, (p.R + 63) / 64, stream);
+}
+
+}  // namespace pagedmla

@@ -1,0 +1,21 @@
+// Internal launch entry points of the kernels behind the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace pagedmla {
+
+cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, int32_t *tile_md,
+                            int32_t *num_splits, cudaStream_t stream);
+cudaError_t launch_decode_mma(const CUtensorMap &map, const DecodeParams &p, cudaStream_t stream);
+cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,
+                           const float *lse_accum, const float *o_accum, __nv_bfloat16 *out,
+                           float *lse, cudaStream_t stream);
+cudaError_t launch_watchdog_selftest(int *status, unsigned long long timeout_ns,
+                                     cudaStream_t stream);
+
+}  // namespace pagedmla

@@ -1,0 +1,246 @@
+"""Python binding of libpagedmla.so: argument marshalling only.
+
+Every step of the decode path runs in the library's CUDA kernels; this module checks
+tensor dtypes, devices and shapes, allocates outputs with torch and passes raw pointers
+and the current CUDA stream.  There is no CPU fallback: without the built library every
+call raises.
+
+The call sequence mirrors the pages' FlashMLA usage ("OpenSourceWeek Day 1 - FlashMLA",
+section V.2):
+
+    tile_metadata, num_splits = get_mla_metadata(cache_seqlens, s_q * h_q // h_kv, h_kv)
+    out, lse = flash_mla_with_kvcache(q, k_cache, block_table, cache_seqlens, dv,
+                                      tile_metadata, num_splits, causal=True)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedmla.so")
+
+MLA_OK = 0
+MLA_ERR_TIMEOUT = -4
+MLA_FLAG_SKIP_COMBINE = 1
+PAGE = 64
+D_QK = 576
+D_V = 512
+TILE_FIELDS = 8
+
+EXPORTED = (
+    "mla_device_sm_count", "mla_num_parts", "mla_get_metadata", "mla_workspace_size",
+    "mla_decode_paged", "mla_combine", "mla_query_status", "mla_watchdog_selftest",
+    "mla_last_error_string",
+)
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+class MlaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"pagedmla error {code}: {msg}")
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libpagedmla.so and declare its C signatures (raises if it is not built)."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with `python -m paged_mla_decode_11_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, I, I64, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64
+        sig = {
+            "mla_device_sm_count": [I, P],
+            "mla_num_parts": [I, I, I, P],
+            "mla_get_metadata": [P, I, I, P, P, P],
+            "mla_workspace_size": [I, I, I, I, I, P],
+            "mla_decode_paged": [P, P, I, I, I, I, P, I64, I, I, P, I64, P, I, P, I, P,
+                                 ctypes.c_float, I, P, P, P, ctypes.c_size_t, ctypes.c_uint, P],
+            "mla_combine": [P, I, I, I, I, I, I, P, ctypes.c_size_t, P, P, P],
+            "mla_query_status": [P, P],
+            "mla_watchdog_selftest": [P, U64, P],
+        }
+        for name, args in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = I
+        lib.mla_last_error_string.argtypes = []
+        lib.mla_last_error_string.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def _check(rc: int) -> None:
+    if rc != MLA_OK:
+        msg = load_library().mla_last_error_string().decode(errors="replace")
+        raise MlaError(rc, msg)
+
+
+def _stream_ptr(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _require_cuda(t: torch.Tensor, name: str, dtype: torch.dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+
+
+_sm_count: dict = {}
+
+
+def device_sm_count(device: Optional[torch.device] = None) -> int:
+    dev = torch.cuda.current_device() if device is None else torch.device(device).index
+    if dev not in _sm_count:
+        lib = load_library()
+        n = ctypes.c_int(0)
+        _check(lib.mla_device_sm_count(dev, ctypes.byref(n)))
+        _sm_count[dev] = n.value
+    return _sm_count[dev]
+
+
+def num_parts_for(num_sms: int, rows_per_kv_head: int, h_kv: int) -> int:
+    lib = load_library()
+    n = ctypes.c_int(0)
+    _check(lib.mla_num_parts(num_sms, rows_per_kv_head, h_kv, ctypes.byref(n)))
+    return n.value
+
+
+def get_mla_metadata(cache_seqlens: torch.Tensor, rows_per_kv_head: int, h_kv: int,
+                     num_parts: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split-KV plan for one decode step: (tile_metadata [num_parts, 8], num_splits [b+1])."""
+    _require_cuda(cache_seqlens, "cache_seqlens", torch.int32)
+    if cache_seqlens.dim() != 1 or not cache_seqlens.is_contiguous():
+        raise ValueError("cache_seqlens must be a contiguous 1-D int32 tensor")
+    dev = cache_seqlens.device
+    if num_parts is None:
+        num_parts = num_parts_for(device_sm_count(dev), rows_per_kv_head, h_kv)
+    batch = cache_seqlens.shape[0]
+    tile = torch.empty(num_parts, TILE_FIELDS, dtype=torch.int32, device=dev)
+    splits = torch.empty(batch + 1, dtype=torch.int32, device=dev)
+    _check(load_library().mla_get_metadata(cache_seqlens.data_ptr(), batch, num_parts,
+                                           tile.data_ptr(), splits.data_ptr(), _stream_ptr(dev)))
+    return tile, splits
+
+
+def workspace_size(batch: int, s_q: int, h_q: int, h_kv: int, num_parts: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().mla_workspace_size(batch, s_q, h_q, h_kv, num_parts, ctypes.byref(n)))
+    return n.value
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """A zeroed scratch buffer for mla_decode_paged (its status block must start at 0)."""
+    return torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+_ws_cache: dict = {}
+
+
+def _default_workspace(nbytes: int, device: torch.device) -> torch.Tensor:
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = new_workspace(nbytes, device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor,
+                     cache_seqlens: torch.Tensor, dv: int, tile_metadata: torch.Tensor,
+                     num_splits: torch.Tensor, softmax_scale: Optional[float] = None,
+                     causal: bool = False, workspace: Optional[torch.Tensor] = None,
+                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                     skip_combine: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Paged MLA decode.  q [b, s_q, h_q, 576] bf16, k_cache [pages, 64, h_kv, 576] bf16,
+    block_table [b, w] int32, cache_seqlens [b] int32.  Returns (out [b, s_q, h_q, dv]
+    bf16, lse [b, h_q, s_q] fp32).  The default softmax_scale is 576 ** -0.5.
+
+    Without ``workspace`` a per-(device, stream) scratch buffer is reused; calls that may
+    run concurrently on one stream's buffer must pass their own."""
+    _require_cuda(q, "q", torch.bfloat16)
+    _require_cuda(k_cache, "k_cache", torch.bfloat16)
+    _require_cuda(block_table, "block_table", torch.int32)
+    _require_cuda(cache_seqlens, "cache_seqlens", torch.int32)
+    _require_cuda(tile_metadata, "tile_metadata", torch.int32)
+    _require_cuda(num_splits, "num_splits", torch.int32)
+    if q.dim() != 4 or k_cache.dim() != 4 or block_table.dim() != 2:
+        raise ValueError("q and k_cache must be 4-D, block_table 2-D")
+    b, s_q, h_q, d = q.shape
+    num_pages, page, h_kv, d2 = k_cache.shape
+    if d2 != d:
+        raise ValueError("q and k_cache disagree on the latent width")
+    if q.stride(3) != 1:
+        raise ValueError("q's last dimension must be contiguous")
+    if not k_cache.is_contiguous():
+        raise ValueError("k_cache must be contiguous")
+    if block_table.stride(1) != 1 or block_table.shape[0] != b:
+        raise ValueError("block_table must be [batch, max_pages] with contiguous rows")
+    if cache_seqlens.shape != (b,) or not cache_seqlens.is_contiguous():
+        raise ValueError("cache_seqlens must be a contiguous [batch] tensor")
+    if tile_metadata.dim() != 2 or tile_metadata.shape[1] != TILE_FIELDS or not tile_metadata.is_contiguous():
+        raise ValueError("tile_metadata must be a contiguous [num_parts, 8] tensor")
+    if num_splits.shape != (b + 1,):
+        raise ValueError("num_splits must be [batch + 1]")
+    dev = q.device
+    num_parts = tile_metadata.shape[0]
+    scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty(b, s_q, h_q, dv, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(b, h_q, s_q, dtype=torch.float32, device=dev)
+    if out.shape != (b, s_q, h_q, dv) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [b, s_q, h_q, dv] tensor")
+    if lse.shape != (b, h_q, s_q) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [b, h_q, s_q] tensor")
+    need = workspace_size(b, s_q, h_q, h_kv, num_parts)
+    if workspace is None:
+        workspace = _default_workspace(need, dev)
+    strides = (ctypes.c_int64 * 3)(q.stride(0), q.stride(1), q.stride(2))
+    flags = MLA_FLAG_SKIP_COMBINE if skip_combine else 0
+    _check(load_library().mla_decode_paged(
+        q.data_ptr(), strides, b, s_q, h_q, d, k_cache.data_ptr(), num_pages, page, h_kv,
+        block_table.data_ptr(), block_table.stride(0), cache_seqlens.data_ptr(), dv,
+        tile_metadata.data_ptr(), num_parts, num_splits.data_ptr(), scale, int(bool(causal)),
+        out.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel(), flags,
+        _stream_ptr(dev)))
+    return out, lse
+
+
+# The pages' name for the decode call.
+flash_mla_with_kvcache = mla_decode_paged
+
+
+def mla_combine(num_splits: torch.Tensor, s_q: int, h_q: int, h_kv: int, num_parts: int,
+                workspace: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, dv: int = D_V) -> None:
+    """Merge split partials left by mla_decode_paged(..., skip_combine=True) into out/lse."""
+    _require_cuda(num_splits, "num_splits", torch.int32)
+    b = num_splits.shape[0] - 1
+    _check(load_library().mla_combine(num_splits.data_ptr(), b, s_q, h_q, h_kv, dv, num_parts,
+                                      workspace.data_ptr(), workspace.numel(), out.data_ptr(),
+                                      lse.data_ptr(), _stream_ptr(out.device)))
+
+
+def query_status(workspace: torch.Tensor) -> int:
+    """Synchronise the current stream; return 0 or MLA_ERR_TIMEOUT (and clear it)."""
+    rc = load_library().mla_query_status(workspace.data_ptr(), _stream_ptr(workspace.device))
+    if rc not in (MLA_OK, MLA_ERR_TIMEOUT):
+        _check(rc)
+    return rc
+
+
+def watchdog_selftest(workspace: torch.Tensor, timeout_ns: int) -> None:
+    """Run a bounded wait that can only time out (see mla_watchdog_selftest)."""
+    _check(load_library().mla_watchdog_selftest(workspace.data_ptr(), int(timeout_ns),
+                                                _stream_ptr(workspace.device)))

@@ -1,0 +1,74 @@
+"""Host-side checks of the C ABI: the library loads on a machine without a GPU, exports
+every entry point include/pagedmla.h declares, and its host-only logic (part count,
+workspace size, argument rejection) behaves as documented."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_mla_decode_11_b200 import build as B
+from paged_mla_decode_11_b200 import ops
+from oracle import metadata as spec
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "pagedmla.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return ops.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*MLA_API\s+(?:const\s+)?\w+\s*\*?\s*(mla_\w+)\s*\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 9, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in pagedmla.h but not exported"
+    assert set(names) == set(ops.EXPORTED)
+
+
+def test_num_parts_matches_scheduler_granularity(lib):
+    for sms in (1, 4, 132, 148):
+        for R in (1, 16, 63, 64, 65, 128, 256, 1000):
+            for h_kv in (1, 2, 3):
+                assert ops.num_parts_for(sms, R, h_kv) == spec.num_parts_for(sms, R, h_kv)
+
+
+def test_workspace_size(lib):
+    n = ops.workspace_size(64, 1, 16, 1, 148)
+    splits = 64 + 148
+    R = 16
+    lse_bytes = splits * R * 4
+    o_off = (256 + lse_bytes + 255) // 256 * 256
+    assert n == o_off + splits * R * 512 * 4
+
+
+def test_host_side_rejections(lib):
+    out = ctypes.c_size_t(0)
+    assert lib.mla_workspace_size(4, 1, 16, 3, 10, ctypes.byref(out)) == -1   # h_q % h_kv
+    assert b"multiple" in lib.mla_last_error_string()
+    assert lib.mla_workspace_size(0, 1, 16, 1, 10, ctypes.byref(out)) == -1
+    n = ctypes.c_int(0)
+    assert lib.mla_num_parts(0, 16, 1, ctypes.byref(n)) == -1
+    assert lib.mla_get_metadata(None, 4, 10, None, None, None) == -1
+    strides = (ctypes.c_int64 * 3)(576, 576, 576)
+    # d != 576 and dv != 512 are refused before anything touches a device
+    rc = lib.mla_decode_paged(16, strides, 1, 1, 16, 512, 16, 1, 64, 1, 16, 1, 16, 512, 16, 1, 16,
+                              ctypes.c_float(0.04), 1, 16, 16, 256, 1 << 20, 0, None)
+    assert rc == -2 and b"d must be 576" in lib.mla_last_error_string()
+    rc = lib.mla_decode_paged(16, strides, 1, 1, 16, 576, 16, 1, 64, 1, 16, 1, 16, 256, 16, 1, 16,
+                              ctypes.c_float(0.04), 1, 16, 16, 256, 1 << 20, 0, None)
+    assert rc == -2 and b"dv must be 512" in lib.mla_last_error_string()
+    rc = lib.mla_decode_paged(16, strides, 1, 1, 16, 576, 16, 1, 32, 1, 16, 1, 16, 512, 16, 1, 16,
+                              ctypes.c_float(0.04), 1, 16, 16, 256, 1 << 20, 0, None)
+    assert rc == -2 and b"page_size" in lib.mla_last_error_string()
+    rc = lib.mla_decode_paged(16, strides, 1, 1, 16, 576, 16, 1, 64, 1, 16, 1, 16, 512, 16, 1, 16,
+                              ctypes.c_float(-1.0), 1, 16, 16, 256, 1 << 20, 0, None)
+    assert rc == -1 and b"softmax_scale" in lib.mla_last_error_string()

@@ -1,0 +1,181 @@
+"""GPU parity of the CUDA decode path against the fp64 oracle, through the C ABI.
+
+Tolerances (fixed by the specification of this path): bf16 outputs within
+max |out - ref| <= 1e-2 * max |ref|, fp32 LSE within relative 1e-4, rows without any
+visible key exactly out = 0 and lse = -inf; the split-KV plan bit-exact against the
+oracle's scheduler specification.  The LSE's relative error is taken against
+max(|ref|, 1): lse = ln Z is the log of the softmax normaliser, so an absolute LSE error
+of 1e-4 is a relative error of 1e-4 in Z, and a plain relative test is ill-conditioned
+where a single visible key puts the LSE near zero.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import metadata as spec
+from paged_mla_decode_11_b200 import ops
+from paged_mla_decode_11_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 1e-2
+LSE_RTOL = 1e-4
+
+
+def to_dev(x):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+def run_gpu(x, num_parts=None, q=None, skip_combine=False):
+    d = to_dev(x)
+    R = x["s_q"] * x["h_q"] // x["h_kv"]
+    tile, splits = ops.get_mla_metadata(d["cache_seqlens"], R, x["h_kv"], num_parts=num_parts)
+    qq = d["q"] if q is None else q
+    out, lse = ops.mla_decode_paged(qq, d["k_cache"], d["block_table"], d["cache_seqlens"], x["dv"],
+                                    tile, splits, softmax_scale=x["softmax_scale"],
+                                    causal=x["causal"], skip_combine=skip_combine)
+    torch.cuda.synchronize()
+    return out, lse, tile, splits
+
+
+def check_metadata(x, tile, splits):
+    want_tiles, want_splits = spec.schedule(x["cache_seqlens"].tolist(), tile.shape[0])
+    assert tile.cpu().tolist() == want_tiles
+    assert splits.cpu().tolist() == want_splits
+
+
+def assert_parity(out, lse, ref_out, ref_lse):
+    out = out.double().cpu().numpy()
+    lse = lse.double().cpu().numpy()
+    ref_inf = np.isneginf(ref_lse)
+    np.testing.assert_array_equal(np.isneginf(lse), ref_inf)
+    scale = max(np.abs(ref_out).max(), 1e-30)
+    err = np.abs(out - ref_out).max()
+    assert err <= OUT_TOL * scale, f"max abs err {err:.3e} > {OUT_TOL} * {scale:.3e}"
+    fin = ~ref_inf
+    if fin.any():
+        rel = np.abs(lse[fin] - ref_lse[fin]) / np.maximum(np.abs(ref_lse[fin]), 1.0)
+        assert rel.max() <= LSE_RTOL, f"lse rel err {rel.max():.3e}"
+
+
+def full_parity(x, **kw):
+    out, lse, tile, splits = run_gpu(x, **kw)
+    check_metadata(x, tile, splits)
+    ref_out, ref_lse = oracle.mla_decode(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"],
+                                         dv=x["dv"], softmax_scale=x["softmax_scale"], causal=x["causal"])
+    assert_parity(out, lse, ref_out, ref_lse)
+    # rows that see no key are exactly zero
+    empty = np.isneginf(ref_lse).transpose(0, 2, 1)
+    if empty.any():
+        assert (out.float().cpu().numpy()[empty] == 0).all()
+    return out, lse, splits
+
+
+SMALL_CASES = [
+    # (batch, s_q, h_q, h_kv, seqlens, causal)
+    (2, 1, 16, 1, [37, 130], True),                      # the tiny decode workload
+    (5, 1, 16, 1, [1, 63, 64, 65, 300], False),          # ragged tails around page edges
+    (3, 1, 64, 1, [130, 1000, 7], True),                 # 64 rows per latent head
+    (2, 1, 128, 1, [500, 77], True),                     # two 64-row blocks
+    (3, 2, 128, 1, [2, 129, 700], True),                 # causal multi-token, 256 rows
+    (2, 1, 32, 2, [100, 200], False),                    # two latent heads
+    (3, 1, 16, 1, [0, 5, 0], True),                      # empty sequences
+    (2, 2, 16, 1, [1, 66], True),                        # causal row with no visible key
+    (4, 2, 8, 1, [64, 1, 2, 3000], True),                # short causal rows and a long split one
+    (1, 1, 16, 1, [6000], False),                        # one long sequence over many splits
+]
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: f"b{c[0]}sq{c[1]}h{c[2]}kv{c[3]}")
+def test_parity_small(case):
+    b, s_q, h_q, h_kv, lens, causal = case
+    x = W.make_inputs(W.custom(b, s_q, h_q, h_kv, lens, causal=causal), seed=sum(lens) % 97)
+    full_parity(x)
+
+
+def test_parity_outlier_rows_and_scale():
+    x = W.make_inputs(W.custom(3, 2, 64, 1, [900, 45, 2000], causal=True, outlier_frac=0.05, scale=0.11),
+                      seed=21)
+    full_parity(x)
+
+
+@pytest.mark.parametrize("num_parts", [1, 2, 7, 148, 400])
+def test_parity_any_part_count(num_parts):
+    x = W.make_inputs(W.custom(6, 1, 16, 1, [3000, 1, 0, 640, 64, 999], causal=True), seed=5)
+    full_parity(x, num_parts=num_parts)
+
+
+def test_strided_query_view():
+    x = W.make_inputs(W.custom(3, 1, 16, 1, [70, 300, 5], causal=True), seed=8)
+    big = torch.zeros(3, 1, 24, 640, dtype=torch.bfloat16, device="cuda")
+    big[:, :, 4:20, :576] = x["q"].cuda()
+    qv = big[:, :, 4:20, :576]
+    assert not qv.is_contiguous()
+    out, lse, _, _ = run_gpu(x, q=qv)
+    ref_out, ref_lse = oracle.mla_decode(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"],
+                                         dv=512, softmax_scale=x["softmax_scale"], causal=True)
+    assert_parity(out, lse, ref_out, ref_lse)
+
+
+def test_separate_combine_matches_fused():
+    x = W.make_inputs(W.custom(2, 1, 64, 1, [5000, 300], causal=True), seed=9)
+    out_a, lse_a, tile, splits = run_gpu(x)
+    d = to_dev(x)
+    ws = ops.new_workspace(ops.workspace_size(2, 1, 64, 1, tile.shape[0]), "cuda")
+    out_b, lse_b = ops.mla_decode_paged(d["q"], d["k_cache"], d["block_table"], d["cache_seqlens"], 512,
+                                        tile, splits, softmax_scale=x["softmax_scale"], causal=True,
+                                        workspace=ws, skip_combine=True)
+    ops.mla_combine(splits, 1, 64, 1, tile.shape[0], ws, out_b, lse_b)
+    torch.cuda.synchronize()
+    assert int(splits[1] - splits[0]) > 1
+    assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
+
+
+def test_deterministic():
+    x = W.make_inputs(W.custom(4, 1, 128, 1, [4000, 100, 2500, 64], causal=True), seed=10)
+    a = run_gpu(x)
+    b = run_gpu(x)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_watchdog_times_out_and_context_survives():
+    ws = ops.new_workspace(256, "cuda")
+    ops.watchdog_selftest(ws, 50_000_000)           # 50 ms limit on a wait nothing completes
+    assert ops.query_status(ws) == ops.MLA_ERR_TIMEOUT
+    assert ops.query_status(ws) == ops.MLA_OK          # cleared
+    x = W.make_inputs(W.TINY)
+    full_parity(x)                                     # the context is still usable
+
+
+# ---------------------------------------------------------------------------------------
+# Full-size workloads, in the launch configuration the benchmark times: bit-exact plan,
+# finite outputs everywhere, and sampled rows against the oracle computed one by one.
+# ---------------------------------------------------------------------------------------
+def sample_rows(x, per_seq=2, seed=0):
+    rng = np.random.default_rng(seed)
+    b, s_q, h_q = x["q"].shape[:3]
+    rows = []
+    for i in range(b):
+        for _ in range(per_seq):
+            rows.append((i, rng.integers(s_q), rng.integers(h_q)))
+        rows.append((i, s_q - 1, h_q - 1))
+    return np.array(rows, dtype=np.int32)
+
+
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_full_size_workloads(name):
+    x = W.make_inputs(W.WORKLOADS[name], seed=0)
+    out, lse, tile, splits = run_gpu(x)
+    check_metadata(x, tile, splits)
+    assert torch.isfinite(out).all()
+    assert torch.isfinite(lse).all()
+    rows = sample_rows(x)
+    ro, rl = oracle.mla_decode_rows(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], rows,
+                                    dv=512, softmax_scale=x["softmax_scale"], causal=x["causal"])
+    o = out.double().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    l = lse.double().cpu().numpy()[rows[:, 0], rows[:, 2], rows[:, 1]]
+    err = np.abs(o - ro).max()
+    assert err <= OUT_TOL * np.abs(ro).max(), err
+    assert (np.abs(l - rl) / np.maximum(np.abs(rl), 1.0)).max() <= LSE_RTOL
