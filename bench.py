@@ -1,0 +1,459 @@
+"""Benchmark of the paged MLA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole path over one decode batch: the split-KV scheduler
+(mla_get_metadata), the fused decode kernel (mla_decode_paged) and the log-sum-exp
+combine (mla_combine).  The default workload is the memory-bound decode batch
+(batch 64, s_q 1, 16 query heads on one latent head, d = 576, dv = 512, 64-token pages,
+cache lengths uniform in [1, 4096] from seed 0); its metric is HBM GB/s over the
+algorithmic bytes (every valid token's latent row read once, plus q, out, lse and the
+addressed block-table entries and lengths).  Compute-bound workloads report TFLOP/s over
+2 * (576 + 512) flops per (query row, visible key).
+
+Timing: W warm-up steps, then exactly K steps replayed from one CUDA graph, bracketed by
+a barrier and a device synchronisation on both sides and timed with CUDA events on the
+launching stream; the maximum over ranks is reported.  Steps rotate over enough copies
+of the inputs that everything a step reads was last touched more than one L2 (126 MB)
+ago.  Timing events inside the graph bracket every decode-kernel launch; their average
+is the roofline duration.
+
+N > 1 (torchrun, one process per GPU): sequences are independent, so every rank decodes
+its own batch with no data-path collective (weak scaling); only the timing is reduced.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on the host cores,
+each step a bounded sample of whole sequences of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_mla_decode_11_b200 import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["common.cuh", "decode_mma.cu"]
+
+
+# ----------------------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------------------
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), \
+        int(os.environ.get("WORLD_SIZE", "1"))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "paged_mla_decode_11_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
+    the current kernel sources; None otherwise."""
+    path = os.path.join(ROOT, "profiles", f"decode_{workload}_ncu.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    if not m_t or not m_h or m_h.group(1) != kernel_source_hash():
+        return None
+    return float(m_t.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU is loaded."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", ident, "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def workload_work(x, w):
+    lens = x["cache_seqlens"].tolist()
+    nbytes, flops = W.algorithmic_work(lens, w.s_q, w.h_q, w.h_kv, w.causal)
+    return nbytes, flops
+
+
+def metric_of(w_name):
+    if w_name in ("compute_bound", "causal_mtp"):
+        return "TFLOP/s", "tensor"
+    return "GB/s", "hbm"
+
+
+METRIC = "paged MLA decode on 1 B200: HBM GB/s (mem-bound), TFLOPS (compute-bound)"
+
+
+def workload_config(w):
+    lens = w.seqlens
+    return {"workload": f"{w.name}: batch={w.batch}, s_q={w.s_q}, h_q={w.h_q}, h_kv={w.h_kv}, "
+                        f"d=576, dv=512, page 64, seqlens {lens}, causal={w.causal}, "
+                        f"scale={w.scale:.6g}, bf16 q/cache ~N(0,1), random block_table over one pool, "
+                        "seed 0"}
+
+
+# ----------------------------------------------------------------------------------------
+# CPU oracle timing (our arm's cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------------------
+def oracle_sample(x, w, seqs):
+    import numpy as np
+    import oracle
+    rows = [(b, s, h) for b in seqs for s in range(w.s_q) for h in range(w.h_q)]
+    rows = np.array(rows, dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle.mla_decode_rows(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], rows, dv=512,
+                           softmax_scale=w.scale, causal=w.causal)
+    dt = time.perf_counter() - t0
+    lens = [int(x["cache_seqlens"][b]) for b in seqs]
+    nb, fl = W.algorithmic_work(lens, w.s_q, w.h_q, w.h_kv, w.causal)
+    return dt, nb, fl
+
+
+def pick_sample(x, w, seconds):
+    """Whole sequences, cycling from a start index, totalling about `seconds` of oracle work."""
+    dt, nb, fl = oracle_sample(x, w, [0])
+    per_flop = dt / max(fl, 1)
+    lens = x["cache_seqlens"].tolist()
+    order = list(range(w.batch))
+    chosen, acc = [], 0.0
+    for b in order:
+        _, f = W.algorithmic_work([lens[b]], w.s_q, w.h_q, w.h_kv, w.causal)
+        chosen.append(b)
+        acc += f * per_flop
+        if acc >= seconds:
+            break
+    return chosen
+
+
+def cpu_baseline(x, w, unit, seconds=10.0):
+    import oracle
+    seqs = pick_sample(x, w, seconds)
+    dt, nb, fl = oracle_sample(x, w, seqs)
+    val = nb / dt / 1e9 if unit == "GB/s" else fl / dt / 1e12
+    return {"value": val, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(seqs)} of {w.batch} sequences (all query rows), {dt:.1f} s of fp64 oracle work"}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    w = W.WORKLOADS[args.workload]
+    x = W.make_inputs(w, seed=0)
+    unit, _ = metric_of(args.workload)
+    budget = 90.0 / max(args.steps + args.warmup, 1)
+    per_step = min(2.0, max(0.05, budget))
+    # samples are consecutive runs of whole sequences, cycling over the batch
+    dt1, _, fl1 = oracle_sample(x, w, [0])
+    lens = x["cache_seqlens"].tolist()
+    per_flop = dt1 / max(fl1, 1)
+    cursor = 0
+
+    def next_sample():
+        nonlocal cursor
+        seqs, acc = [], 0.0
+        while acc < per_step and len(seqs) < w.batch:
+            b = cursor % w.batch
+            _, f = W.algorithmic_work([lens[b]], w.s_q, w.h_q, w.h_kv, w.causal)
+            seqs.append(b)
+            acc += f * per_flop
+            cursor += 1
+        return seqs
+
+    for _ in range(args.warmup):
+        oracle_sample(x, w, next_sample())
+    tot_t = tot_b = tot_f = 0.0
+    nseq = 0
+    for _ in range(args.steps):
+        s = next_sample()
+        dt, nb, fl = oracle_sample(x, w, s)
+        tot_t += dt
+        tot_b += nb
+        tot_f += fl
+        nseq += len(s)
+    val = tot_b / tot_t / 1e9 if unit == "GB/s" else tot_f / tot_t / 1e12
+    sample = (f"each step: consecutive whole sequences (about {per_step:.2f} s of fp64 oracle work), "
+              f"{nseq} sequences over {args.steps} steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": val, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------------------
+def run_ours(args):
+    from paged_mla_decode_11_b200 import ops
+    rank, local_rank, world = dist_env()
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} processes (launch with torchrun)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            t = torch.zeros(1, device=dev)
+            pg.all_reduce(t)
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(v: float) -> float:
+        if pg is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        return float(t.item())
+
+    w = W.WORKLOADS[args.workload]
+    R = w.rows_per_kv_head
+    x = W.make_inputs(w, seed=args.seed + rank)
+    nbytes, flops = workload_work(x, w)
+    unit, bound = metric_of(args.workload)
+    per_rep = x["k_cache"].numel() * 2
+    n_rep = max(2, math.ceil(1.5 * L2_BYTES / per_rep) + 1)
+
+    reps = []
+    for r in range(n_rep):
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+        if r > 0:
+            d = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+        nparts = ops.num_parts_for(ops.device_sm_count(dev), R, w.h_kv)
+        d["ws"] = ops.new_workspace(ops.workspace_size(w.batch, w.s_q, w.h_q, w.h_kv, nparts), dev)
+        d["out"] = torch.empty(w.batch, w.s_q, w.h_q, 512, dtype=torch.bfloat16, device=dev)
+        d["lse"] = torch.empty(w.batch, w.h_q, w.s_q, dtype=torch.float32, device=dev)
+        reps.append(d)
+
+    def step(d, ev=None):
+        tile, splits = ops.get_mla_metadata(d["cache_seqlens"], R, w.h_kv)
+        if ev is not None:
+            ev[0].record()
+        ops.mla_decode_paged(d["q"], d["k_cache"], d["block_table"], d["cache_seqlens"], 512, tile,
+                             splits, softmax_scale=w.scale, causal=w.causal, workspace=d["ws"],
+                             out=d["out"], lse=d["lse"], skip_combine=True)
+        if ev is not None:
+            ev[1].record()
+        ops.mla_combine(splits, w.s_q, w.h_q, w.h_kv, tile.shape[0], d["ws"], d["out"], d["lse"])
+
+    # eager warm-up (first launches, allocator, tensor maps), then graph capture
+    for i in range(max(args.warmup, 3)):
+        step(reps[i % n_rep])
+    torch.cuda.synchronize(dev)
+
+    stream = torch.cuda.Stream(device=dev)
+    warm_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(warm_graph, stream=stream):
+        for i in range(max(args.warmup, 3)):
+            step(reps[i % n_rep])
+    events = [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(args.steps):
+            step(reps[i % n_rep], events[i])
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(local_rank)
+    # keep the GPU loaded for ~1 s before timing so the sampled clocks describe the load
+    t_end = time.perf_counter() + 1.0
+    while time.perf_counter() < t_end:
+        warm_graph.replay()
+        torch.cuda.synchronize(dev)
+    barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        graph.replay()
+        end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    elapsed = max_over_ranks(start.elapsed_time(end) * 1e-3)
+    kernel_s = sum(a.elapsed_time(b) for a, b in events) * 1e-3 / args.steps
+    kernel_s = max_over_ranks(kernel_s)
+    per_step = elapsed / args.steps
+    total_bytes = nbytes * world
+    total_flops = flops * world
+    value = (total_bytes / per_step / 1e9) if unit == "GB/s" else (total_flops / per_step / 1e12)
+
+    peaks, peak_kind = load_peaks()
+    if bound == "hbm":
+        achieved = nbytes / kernel_s / 1e9
+        peak = peaks["hbm_gbs"]
+        r_unit = "GB/s"
+    else:
+        achieved = flops / kernel_s / 1e12
+        peak = peaks["bf16_tflops"]
+        r_unit = "TFLOP/s"
+    traffic = recorded_traffic(args.workload)
+
+    # end to end through the public API from pinned host buffers (the latent page pool is
+    # resident device state; each step sends q, block_table and cache_seqlens and reads
+    # back out and lse)
+    e2e_steps = min(args.steps, 50)
+    hq = x["q"].pin_memory()
+    hbt = x["block_table"].pin_memory()
+    hsl = x["cache_seqlens"].pin_memory()
+    hout = torch.empty(w.batch, w.s_q, w.h_q, 512, dtype=torch.bfloat16).pin_memory()
+    hlse = torch.empty(w.batch, w.h_q, w.s_q, dtype=torch.float32).pin_memory()
+    d0 = reps[0]
+    ws_e2e = d0["ws"]
+
+    def e2e_step():
+        q = hq.to(dev, non_blocking=True)
+        bt = hbt.to(dev, non_blocking=True)
+        sl = hsl.to(dev, non_blocking=True)
+        tile, splits = ops.get_mla_metadata(sl, R, w.h_kv)
+        out, lse = ops.flash_mla_with_kvcache(q, d0["k_cache"], bt, sl, 512, tile, splits,
+                                              softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e)
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) * 1e-3 / e2e_steps)
+    e2e_val = (total_bytes / e2e_s / 1e9) if unit == "GB/s" else (total_flops / e2e_s / 1e12)
+    h2d = hq.numel() * 2 + hbt.numel() * 4 + hsl.numel() * 4
+    d2h = hout.numel() * 2 + hlse.numel() * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(x, w, unit)
+
+    if pg is not None:
+        pg.destroy_process_group()
+    if rank != 0:
+        return
+    cfg = workload_config(w)
+    cfg["l2"] = (f"inputs larger than L2: steps rotate over {n_rep} copies of the inputs "
+                 f"({per_rep / 1e6:.0f} MB latent pool each)")
+    cfg["parallelism"] = f"dp{world} (independent batches per GPU)"
+    cfg["timing"] = f"{args.steps} steps replayed from one CUDA graph"
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": cfg,
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+                     "kernel": "decode", "kernel_ms": kernel_s * 1e3,
+                     "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="memory_bound", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

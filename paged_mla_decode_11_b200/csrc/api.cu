@@ -8,6 +8,8 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <utility>
+#include <vector>
 
 #include "launch.h"
 #include "pagedmla.h"
@@ -107,6 +109,24 @@ int check_common(int batch, int s_q, int h_q, int h_kv, int dv) {
 }
 
 }  // namespace
+
+namespace pagedmla {
+
+cudaError_t set_smem_once(const void *kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void *, int>> done;  // (kernel, device)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto &d : done)
+    if (d.first == kernel && d.second == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.emplace_back(kernel, dev);
+  return e;
+}
+
+}  // namespace pagedmla
 
 extern "C" {
 

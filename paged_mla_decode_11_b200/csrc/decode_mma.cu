@@ -352,7 +352,7 @@ static cudaError_t launch_mma(const CUtensorMap &map, const DecodeParams &p, int
                               cudaStream_t stream) {
   using T = MmaTile<BM, DVS>;
   auto kern = decode_mma_kernel<BM, DVS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::kSmemBytes);
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), T::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_parts, m_blocks, p.h_kv);
   kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(map, p);

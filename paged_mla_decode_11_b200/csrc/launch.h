@@ -9,6 +9,10 @@
 
 namespace pagedmla {
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device), so that
+// launches inside CUDA-graph capture make no attribute calls.
+cudaError_t set_smem_once(const void *kernel, int bytes);
+
 cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, int32_t *tile_md,
                             int32_t *num_splits, cudaStream_t stream);
 cudaError_t launch_decode_mma(const CUtensorMap &map, const DecodeParams &p, cudaStream_t stream);

@@ -9,6 +9,7 @@
 // plan there (integer arithmetic only, so the result is exact), then the split counts
 // are turned into prefix sums.
 #include "launch.h"
+#include "pagedmla.h"
 
 namespace pagedmla {
 
@@ -83,8 +84,8 @@ cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, in
                             int32_t *num_splits, cudaStream_t stream) {
   const size_t smem = size_t(batch) * 2 * sizeof(int32_t);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(metadata_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(metadata_kernel),
+                                  2 * MLA_MAX_BATCH * int(sizeof(int32_t)));
     if (e != cudaSuccess) return e;
   }
   metadata_kernel<<<1, kMetaThreads, smem, stream>>>(seqlens, batch, num_parts, tile_md, num_splits);
