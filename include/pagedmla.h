@@ -87,10 +87,12 @@ MLA_API int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_
  * section V.2: get_mla_metadata(cache_seqlens, s_q*h_q//h_kv, h_kv) -> tile_metadata,
  * num_splits; the pages print its call only, the plan is this library's specification).
  *
- * Spreads sum_b ceil(L_b / 64) pages, plus MLA_SPLIT_OVERHEAD per split, over
- * `num_parts` parts by a greedy walk: payload = ceil(total / num_parts) + OVERHEAD; each
- * part finishes whole sequences while they fit and otherwise takes the next
- * (remaining - OVERHEAD) pages of the current sequence.
+ * Plan ("balanced cuts"): sequence b occupies OVH + ceil(L_b / 64) units of a cost axis
+ * (OVH = MLA_SPLIT_OVERHEAD units first, then one unit per page).  With T the axis length
+ * and payload = ceil(T / num_parts), part p covers [p*payload, (p+1)*payload) clipped to
+ * T.  A cut at position x inside sequence i becomes the cursor (i, max(0, x - start_i -
+ * OVH)) in pages, so a cut inside a sequence's overhead units moves the whole sequence to
+ * the next part.  Each part does at most payload + OVH units of work.
  *
  *   cache_seqlens  device int32 [batch], each >= 0
  *   tile_metadata  device int32 [num_parts][8], written:

@@ -7,25 +7,24 @@ passes the returned ``tile_metadata`` and ``num_splits`` to the kernel; the Baid
 variable-length sequences over a paged cache, without padding work.  The pages print no
 algorithm, so the plan below is this library's own specification, written out here in
 plain Python.  Parity unpinned against the pages: it is pinned by its coverage invariants
-(every page of every sequence covered exactly once, in order) and by hand-worked cases.
+(every page of every sequence covered exactly once, in order), its load bound and
+hand-worked cases.
 
-Specification
+Specification ("balanced cuts")
   PAGE = 64 tokens, OVH = 5 (fixed cost of one split, in pages)
-  pages_b  = ceil(L_b / PAGE);  total = sum_b (pages_b + OVH)
-  payload  = ceil(total / num_parts) + OVH
-  Walk the sequences with a cursor (i, k) = (sequence, page within it), starting at (0, 0).
-  For each part in order: begin = cursor, rem = payload, then repeat while i < B:
-      left = pages_i - k
-      if left + OVH <= rem:  the part finishes sequence i (rem -= left + OVH; i += 1; k = 0)
-      else: if rem - OVH > 0 the part takes the next rem - OVH pages of sequence i
-            (k += rem - OVH); stop.
-  end = cursor.  A part touches sequence i when it finishes it or takes pages of it;
-  num_splits[b] counts the parts touching b.
+  Lay the sequences end to end on a cost axis: sequence b occupies OVH + ceil(L_b / 64)
+  units, its OVH units first, then one unit per page.  T = total length of the axis.
+  payload = ceil(T / num_parts).  Part p covers the axis interval
+  [min(p * payload, T), min((p + 1) * payload, T)).
+  An axis position x maps to the cursor (sequence i, page k): x >= T -> (B, 0); otherwise
+  i is the sequence whose interval holds x and k = max(0, x - start_i - OVH), so a cut
+  inside a sequence's OVH units moves the whole sequence to the next part.
+  Part p runs from the cursor of its first position up to (excluding) the cursor of its
+  end, so each part does at most payload + OVH units of work.
 
 Outputs
   tile_metadata[p] = (begin_i, begin_k * PAGE, end_i, end_k * PAGE, begin_split_ord, 0, 0, 0)
-      The part covers tokens from (begin_i, begin_k*PAGE) up to, excluding,
-      (end_i, end_k*PAGE).  begin_split_ord = how many earlier parts touched begin_i.
+      begin_split_ord = how many earlier parts touched begin_i.
   num_splits[0] = 0; num_splits[b + 1] = num_splits[b] + (parts touching b).
 """
 
@@ -47,32 +46,42 @@ def schedule(cache_seqlens, num_parts: int):
     """Return (tile_metadata: list of num_parts 8-int lists, num_splits: list of B+1)."""
     lens = [int(x) for x in cache_seqlens]
     B = len(lens)
-    pages = [-(-L // PAGE) for L in lens]
-    total = sum(p + OVH for p in pages)
-    payload = -(-total // num_parts) + OVH
+    cost = [OVH + -(-L // PAGE) for L in lens]
+    start = []
+    acc = 0
+    for c in cost:
+        start.append(acc)
+        acc += c
+    T = acc
+    payload = -(-T // num_parts)
+
+    def cursor(x):
+        if x >= T:
+            return B, 0
+        i = 0
+        while i + 1 < B and start[i + 1] <= x:
+            i += 1
+        return i, max(0, x - start[i] - OVH)
+
+    cuts = [cursor(min(p * payload, T)) for p in range(num_parts + 1)]
     touched = [0] * B
-    i, k = 0, 0
     tiles = []
-    for _ in range(num_parts):
-        begin_i, begin_k = i, k
-        begin_ord = touched[i] if i < B else 0
-        rem = payload
-        while i < B:
-            left = pages[i] - k
-            if left + OVH <= rem:
-                rem -= left + OVH
-                touched[i] += 1
-                i, k = i + 1, 0
-            else:
-                if rem - OVH > 0:
-                    k += rem - OVH
-                    touched[i] += 1
-                break
-        tiles.append([begin_i, begin_k * PAGE, i, k * PAGE, begin_ord, 0, 0, 0])
+    for p in range(num_parts):
+        (bi, bk), (ei, ek) = cuts[p], cuts[p + 1]
+        ordinal = touched[bi] if bi < B else 0
+        last = ei if ek > 0 else ei - 1          # last sequence this part touches
+        for s in range(bi, min(last, B - 1) + 1):
+            touched[s] += 1
+        tiles.append([bi, bk * PAGE, ei, ek * PAGE, ordinal, 0, 0, 0])
     num_splits = [0]
     for b in range(B):
         num_splits.append(num_splits[-1] + touched[b])
     return tiles, num_splits
+
+
+def payload_of(cache_seqlens, num_parts: int) -> int:
+    T = sum(OVH + -(-int(L) // PAGE) for L in cache_seqlens)
+    return -(-T // num_parts)
 
 
 def segments(tiles, cache_seqlens):

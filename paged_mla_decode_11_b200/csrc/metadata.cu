@@ -1,91 +1,124 @@
 // Split-KV tile scheduler (the pages' get_mla_metadata: "OpenSourceWeek Day 1 -
-// FlashMLA", section V.2, which shows only its call).  Plan, as specified in pagedmla.h:
-// pages_b = ceil(L_b / 64); total = sum_b (pages_b + OVH); payload = ceil(total / parts)
-// + OVH; each part, in order, finishes whole sequences while (pages left + OVH) fits in
-// what remains of its payload and otherwise takes the next (remaining - OVH) pages of
-// the current sequence, if that is positive.
+// FlashMLA", section V.2, which shows only its call).  Plan ("balanced cuts", specified
+// in pagedmla.h): sequence b occupies OVH + ceil(L_b / 64) units of a cost axis (its OVH
+// units first, then one unit per page); with T the axis length and
+// payload = ceil(T / num_parts), part p covers [p * payload, (p + 1) * payload) clipped
+// to T.  Position x maps to the cursor (i, max(0, x - start_i - OVH)) of the sequence i
+// holding it, or (B, 0) at the end.
 //
-// One CTA: the lengths are read in parallel into shared memory, one thread walks the
-// plan there (integer arithmetic only, so the result is exact), then the split counts
-// are turned into prefix sums.
+// Everything is a closed form of the prefix sums start_b, so one CTA computes the plan
+// in parallel: a block scan of the costs, then one binary search per part cut and one
+// closed-form split count per sequence, then a block scan of the split counts.
 #include "launch.h"
 #include "pagedmla.h"
 
 namespace pagedmla {
 
-constexpr int kOvh = 5;
-constexpr int kMetaThreads = 256;
+constexpr int kOvh = MLA_SPLIT_OVERHEAD;
+constexpr int kMetaThreads = 512;
+
+// Exclusive block-wide prefix sum of one value per thread; *total receives the sum.
+__device__ long long block_exclusive_scan(long long v, long long *scratch, long long *total) {
+  const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+  constexpr int kWarps = kMetaThreads / 32;
+  long long incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    long long w = lane < kWarps ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long t = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += t;
+    }
+    if (lane < kWarps) scratch[lane] = w;
+  }
+  __syncthreads();
+  const long long before = warp > 0 ? scratch[warp - 1] : 0;
+  *total = scratch[kWarps - 1];
+  __syncthreads();
+  return before + incl - v;
+}
 
 __global__ void __launch_bounds__(kMetaThreads)
     metadata_kernel(const int32_t *__restrict__ seqlens, int batch, int num_parts,
                     int32_t *__restrict__ tile_md, int32_t *__restrict__ num_splits) {
-  extern __shared__ int32_t sh[];
-  int32_t *pages = sh;
-  int32_t *touched = sh + batch;
-  __shared__ long long warp_tot[kMetaThreads / 32];
+  extern __shared__ long long start[];  // [batch + 1]
+  __shared__ long long scratch[32];
+  const int per = (batch + kMetaThreads - 1) / kMetaThreads;
+  const int lo = threadIdx.x * per, hi = min(batch, lo + per);
 
-  long long local = 0;
-  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
-    const int L = max(seqlens[b], 0);
-    pages[b] = (L + kPage - 1) / kPage;
-    touched[b] = 0;
-    local += pages[b] + kOvh;
+  // 1. start_b = exclusive prefix sum of (OVH + pages_b)
+  long long mine = 0;
+  for (int b = lo; b < hi; ++b) mine += kOvh + (max(seqlens[b], 0) + kPage - 1) / kPage;
+  long long total;
+  long long run = block_exclusive_scan(mine, scratch, &total);
+  for (int b = lo; b < hi; ++b) {
+    start[b] = run;
+    run += kOvh + (max(seqlens[b], 0) + kPage - 1) / kPage;
   }
-  for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-  if (threadIdx.x % 32 == 0) warp_tot[threadIdx.x / 32] = local;
+  if (threadIdx.x == 0) start[batch] = total;
   __syncthreads();
+  const long long T = total;
+  const long long payload = (T + num_parts - 1) / num_parts;
 
-  if (threadIdx.x == 0) {
-    long long total = 0;
-    for (int w = 0; w < kMetaThreads / 32; ++w) total += warp_tot[w];
-    const long long payload = (total + num_parts - 1) / num_parts + kOvh;
-    int i = 0;
-    long long k = 0;
-    for (int part = 0; part < num_parts; ++part) {
-      const int begin_i = i;
-      const long long begin_k = k;
-      const int ord = i < batch ? touched[i] : 0;
-      long long rem = payload;
-      while (i < batch) {
-        const long long left = pages[i] - k;
-        if (left + kOvh <= rem) {
-          rem -= left + kOvh;
-          touched[i] += 1;
-          ++i;
-          k = 0;
-        } else {
-          if (rem - kOvh > 0) {
-            k += rem - kOvh;
-            touched[i] += 1;
-          }
-          break;
+  // 2. one thread per part: both cuts -> cursors by binary search over start[]
+  for (int p = threadIdx.x; p < num_parts; p += kMetaThreads) {
+    int ci[2];
+    long long ck[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const long long x = min((long long)(p + e) * payload, T);
+      if (x >= T) {
+        ci[e] = batch;
+        ck[e] = 0;
+      } else {
+        int a = 0, z = batch - 1;  // largest i with start[i] <= x
+        while (a < z) {
+          const int mid = (a + z + 1) / 2;
+          if (start[mid] <= x) a = mid;
+          else z = mid - 1;
         }
+        ci[e] = a;
+        ck[e] = max(0ll, x - start[a] - kOvh);
       }
-      int32_t *t = tile_md + part * 8;
-      t[0] = begin_i;
-      t[1] = static_cast<int32_t>(begin_k * kPage);
-      t[2] = i;
-      t[3] = static_cast<int32_t>(k * kPage);
-      t[4] = ord;
-      t[5] = 0;
-      t[6] = 0;
-      t[7] = 0;
     }
-    int acc = 0;
-    num_splits[0] = 0;
-    for (int b = 0; b < batch; ++b) {
-      acc += touched[b];
-      num_splits[b + 1] = acc;
-    }
+    const int ord = ck[0] > 0 ? int(p - (start[ci[0]] + kOvh) / payload) : 0;
+    int32_t *t = tile_md + p * 8;
+    t[0] = ci[0];
+    t[1] = int32_t(ck[0] * kPage);
+    t[2] = ci[1];
+    t[3] = int32_t(ck[1] * kPage);
+    t[4] = ord;
+    t[5] = 0;
+    t[6] = 0;
+    t[7] = 0;
+  }
+
+  // 3. parts touching sequence b: 1 + cuts strictly inside its page units
+  long long cnt = 0;
+  for (int b = lo; b < hi; ++b)
+    cnt += 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + kOvh) / payload);
+  long long all;
+  run = block_exclusive_scan(cnt, scratch, &all);
+  if (threadIdx.x == 0) num_splits[0] = 0;
+  for (int b = lo; b < hi; ++b) {
+    run += 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + kOvh) / payload);
+    num_splits[b + 1] = int32_t(run);
   }
 }
 
 cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, int32_t *tile_md,
                             int32_t *num_splits, cudaStream_t stream) {
-  const size_t smem = size_t(batch) * 2 * sizeof(int32_t);
+  const size_t smem = size_t(batch + 1) * sizeof(long long);
   if (smem > 48 * 1024) {
     cudaError_t e = set_smem_once(reinterpret_cast<const void *>(metadata_kernel),
-                                  2 * MLA_MAX_BATCH * int(sizeof(int32_t)));
+                                  int((MLA_MAX_BATCH + 1) * sizeof(long long)));
     if (e != cudaSuccess) return e;
   }
   metadata_kernel<<<1, kMetaThreads, smem, stream>>>(seqlens, batch, num_parts, tile_md, num_splits);

@@ -26,10 +26,9 @@ def test_hand_worked_cases():
 
 def check_plan(lens, num_parts, tiles, splits):
     """Coverage: every page of every sequence exactly once, in order; split counts agree;
-    no part exceeds the payload; ordinals count earlier parts touching a sequence."""
-    pages = [-(-L // M.PAGE) for L in lens]
-    total = sum(p + M.OVH for p in pages)
-    payload = -(-total // num_parts) + M.OVH
+    no part does more than payload + OVH units of work; ordinals count earlier parts
+    touching a sequence."""
+    payload = M.payload_of(lens, num_parts) + M.OVH
     assert len(tiles) == num_parts and len(splits) == len(lens) + 1 and splits[0] == 0
     segs = M.segments(tiles, lens)
     cursor = {}
