@@ -65,6 +65,8 @@ extern "C" {
 #define MLA_MAX_BATCH 16384       /* largest batch mla_get_metadata accepts */
 
 #define MLA_FLAG_SKIP_COMBINE 1u  /* mla_decode_paged: leave split partials unmerged */
+#define MLA_FLAG_WARP_MMA 2u      /* mla_decode_paged: run the warp-MMA (mma.sync) kernel
+                                     instead of the tcgen05 one (a baseline for comparison) */
 
 typedef struct CUstream_st *mla_stream_t; /* identical to cudaStream_t */
 
@@ -142,8 +144,10 @@ MLA_API int mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int num_pa
  *   out            device bf16 [batch][s_q][h_q][dv], contiguous (written)
  *   lse            device fp32 [batch][h_q][s_q], contiguous (written; natural log)
  *   workspace      device scratch of mla_workspace_size bytes (see there)
- *   flags          0, or MLA_FLAG_SKIP_COMBINE to leave the split partials in the
- *                  workspace for a later mla_combine
+ *   flags          0, or an OR of MLA_FLAG_SKIP_COMBINE (leave the split partials in
+ *                  the workspace for a later mla_combine) and MLA_FLAG_WARP_MMA (use the
+ *                  warp-MMA kernel; the default is the tcgen05 kernel where one exists for
+ *                  the shape: up to 64 query rows per latent head)
  * Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.  A device
  * wait that times out (never in correct use) sets the workspace status word; read it
  * with mla_query_status.

@@ -98,6 +98,26 @@ int encode_kv_map(CUtensorMap *map, const void *k_cache, int64_t num_pages, int 
   return MLA_OK;
 }
 
+// Query [batch][s_q][h_q][576] bf16 with element strides (sb, ss, sh) as a 4-D map
+// (columns, head, s_q, batch); one box = 64 columns (128-byte swizzle) x the g heads of one
+// latent head x all s_q positions, i.e. the R query rows of one tile in row order s*g + h.
+int encode_q_map(CUtensorMap *map, const void *q, int batch, int s_q, int h_q, int g,
+                 const int64_t strides[3]) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[4] = {cuuint64_t(kD), cuuint64_t(h_q), cuuint64_t(s_q), cuuint64_t(batch)};
+  cuuint64_t gstr[3] = {cuuint64_t(strides[2]) * 2, cuuint64_t(strides[1]) * 2, cuuint64_t(strides[0]) * 2};
+  for (int i = 0; i < 3; ++i)
+    if (gstr[i] == 0) gstr[i] = 16;  // a dimension of extent 1 may carry stride 0
+  cuuint32_t box[4] = {64, cuuint32_t(g), cuuint32_t(s_q), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), dims, gstr, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled (query) failed (%d)", int(r));
+  return MLA_OK;
+}
+
 int check_common(int batch, int s_q, int h_q, int h_kv, int dv) {
   if (batch < 1 || s_q < 1 || h_q < 1 || h_kv < 1)
     return fail(MLA_ERR_ARG, "batch, s_q, h_q and h_kv must be >= 1");
@@ -191,7 +211,7 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     return fail(MLA_ERR_ARG, "softmax_scale must be positive and finite");
-  if (flags & ~MLA_FLAG_SKIP_COMBINE) return fail(MLA_ERR_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~(MLA_FLAG_SKIP_COMBINE | MLA_FLAG_WARP_MMA)) return fail(MLA_ERR_ARG, "unknown flags 0x%x", flags);
   for (int i = 0; i < 3; ++i)
     if (q_strides[i] < 0 || q_strides[i] % 8 != 0)
       return fail(MLA_ERR_ARG, "q strides must be non-negative multiples of 8 elements");
@@ -239,7 +259,15 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   p.watchdog_ns = kWatchdogNs;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_decode_mma(map, p, st);
+  cudaError_t e;
+  if (R <= 64 && !(flags & MLA_FLAG_WARP_MMA)) {
+    CUtensorMap qmap;
+    rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, q_strides);
+    if (rc) return rc;
+    e = launch_decode_tc_narrow(map, qmap, p, st);
+  } else {
+    e = launch_decode_mma(map, p, st);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   if (!(flags & MLA_FLAG_SKIP_COMBINE)) {
     e = launch_combine(num_splits, batch, s_q, h_q, h_kv, p.lse_accum, p.o_accum, p.out, lse, st);

@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
     int it = 0;
     bool ok = true;
 
-    for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
+    for (int seq = pc.bi; part_has(pc, seq); ++seq) {
       const int L = p.seqlens[seq];
       const int t0 = seq == pc.bi ? pc.bt : 0;
       const int t1 = min(seq == pc.ei ? pc.et : L, block_visible_end(p, L, mb, BM));
@@ -175,10 +175,9 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
       for (int pg = 0; pg < npages; ++pg, ++it) {
         const int s = it % T::kStages;
         const uint32_t ph = (it / T::kStages) & 1;
-        if (!mbar_wait(full_bar + 8 * s, ph, abort, p.status, p.watchdog_ns)) {
-          ok = false;
-          break;
-        }
+        // After a failed wait the warp keeps walking the same named-barrier sequence
+        // without touching the page, so no other warp is left waiting at a bar.sync.
+        ok = ok && mbar_wait(full_bar + 8 * s, ph, abort, p.status, p.watchdog_ns);
         const uint32_t sK = sPages + s * kPageBytes;
 
         // ---- S = Q K^T over the warp's NK keys ----
@@ -296,8 +295,6 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar + 8 * s);
       }
-      if (!ok) break;
-
       // ---- epilogue: total row sums, then final output or split partial ----
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
@@ -315,7 +312,7 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int row = rows[r];
-        if (row >= p.R) continue;
+        if (row >= p.R || !ok) continue;
         float lt = 0.f;
 #pragma unroll
         for (int w = 0; w < DVS; ++w) lt += red_sum[(rg * DVS + w) * 16 + g4 + 8 * r];

@@ -28,6 +28,7 @@ LIB_PATH = os.path.join(_HERE, "libpagedmla.so")
 MLA_OK = 0
 MLA_ERR_TIMEOUT = -4
 MLA_FLAG_SKIP_COMBINE = 1
+MLA_FLAG_WARP_MMA = 2
 PAGE = 64
 D_QK = 576
 D_V = 512
@@ -162,13 +163,14 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
                      num_splits: torch.Tensor, softmax_scale: Optional[float] = None,
                      causal: bool = False, workspace: Optional[torch.Tensor] = None,
                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                     skip_combine: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+                     skip_combine: bool = False, warp_mma: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
     """Paged MLA decode.  q [b, s_q, h_q, 576] bf16, k_cache [pages, 64, h_kv, 576] bf16,
     block_table [b, w] int32, cache_seqlens [b] int32.  Returns (out [b, s_q, h_q, dv]
     bf16, lse [b, h_q, s_q] fp32).  The default softmax_scale is 576 ** -0.5.
 
     Without ``workspace`` a per-(device, stream) scratch buffer is reused; calls that may
-    run concurrently on one stream's buffer must pass their own."""
+    run concurrently on one stream's buffer must pass their own.  ``warp_mma`` selects the
+    warp-MMA (mma.sync) kernel instead of the tcgen05 one, as a baseline."""
     _require_cuda(q, "q", torch.bfloat16)
     _require_cuda(k_cache, "k_cache", torch.bfloat16)
     _require_cuda(block_table, "block_table", torch.int32)
@@ -208,7 +210,7 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
     if workspace is None:
         workspace = _default_workspace(need, dev)
     strides = (ctypes.c_int64 * 3)(q.stride(0), q.stride(1), q.stride(2))
-    flags = MLA_FLAG_SKIP_COMBINE if skip_combine else 0
+    flags = (MLA_FLAG_SKIP_COMBINE if skip_combine else 0) | (MLA_FLAG_WARP_MMA if warp_mma else 0)
     _check(load_library().mla_decode_paged(
         q.data_ptr(), strides, b, s_q, h_q, d, k_cache.data_ptr(), num_pages, page, h_kv,
         block_table.data_ptr(), block_table.stride(0), cache_seqlens.data_ptr(), dv,
