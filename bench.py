@@ -47,7 +47,7 @@ from paged_mla_decode_11_b200 import workloads as W  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["common.cuh", "decode_mma.cu"]
+KERNEL_SOURCES = ["common.cuh", "decode_tc.cu", "decode_mma.cu"]
 
 
 # ----------------------------------------------------------------------------------------
@@ -309,7 +309,8 @@ def run_ours(args):
             ev[0].record()
         ops.mla_decode_paged(d["q"], d["k_cache"], d["block_table"], d["cache_seqlens"], 512, tile,
                              splits, softmax_scale=w.scale, causal=w.causal, workspace=d["ws"],
-                             out=d["out"], lse=d["lse"], skip_combine=True)
+                             out=d["out"], lse=d["lse"], skip_combine=True,
+                             warp_mma=args.kernel == "warp_mma")
         if ev is not None:
             ev[1].record()
         ops.mla_combine(splits, w.s_q, w.h_q, w.h_kv, tile.shape[0], d["ws"], d["out"], d["lse"])
@@ -385,7 +386,8 @@ def run_ours(args):
         sl = hsl.to(dev, non_blocking=True)
         tile, splits = ops.get_mla_metadata(sl, R, w.h_kv)
         out, lse = ops.flash_mla_with_kvcache(q, d0["k_cache"], bt, sl, 512, tile, splits,
-                                              softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e)
+                                              softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
+                                              warp_mma=args.kernel == "warp_mma")
         hout.copy_(out, non_blocking=True)
         hlse.copy_(lse, non_blocking=True)
         torch.cuda.current_stream(dev).synchronize()
@@ -419,6 +421,7 @@ def run_ours(args):
                  f"({per_rep / 1e6:.0f} MB latent pool each)")
     cfg["parallelism"] = f"dp{world} (independent batches per GPU)"
     cfg["timing"] = f"{args.steps} steps replayed from one CUDA graph"
+    cfg["kernel"] = args.kernel
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
@@ -446,6 +449,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", default="tcgen05", choices=["tcgen05", "warp_mma"],
+                    help="decode kernel variant (warp_mma = the mma.sync baseline)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

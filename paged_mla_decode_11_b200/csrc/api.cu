@@ -83,13 +83,14 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Page pool [num_pages * 64 tokens][h_kv][576] bf16 as a 3-D map (columns, latent head,
-// token); one box = 64 columns (128 bytes, 128-byte swizzle) x 1 head x 64 tokens.
-int encode_kv_map(CUtensorMap *map, const void *k_cache, int64_t num_pages, int h_kv) {
+// token); one box = 64 columns (128 bytes, 128-byte swizzle) x 1 head x box_tokens tokens
+// (64 = a page for the warp-MMA kernel, 32 = half a page for the tcgen05 kernel).
+int encode_kv_map(CUtensorMap *map, const void *k_cache, int64_t num_pages, int h_kv, int box_tokens) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(h_kv), cuuint64_t(num_pages) * kPage};
   cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(h_kv) * kD * 2};
-  cuuint32_t box[3] = {64, 1, cuuint32_t(kPage)};
+  cuuint32_t box[3] = {64, 1, cuuint32_t(box_tokens)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k_cache), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -227,8 +228,9 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   if (workspace_bytes < wl.total)
     return fail(MLA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, wl.total);
 
+  const bool use_tc = R <= 64 && !(flags & MLA_FLAG_WARP_MMA);
   CUtensorMap map;
-  rc = encode_kv_map(&map, k_cache, num_pages, h_kv);
+  rc = encode_kv_map(&map, k_cache, num_pages, h_kv, use_tc ? 32 : kPage);
   if (rc) return rc;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -260,7 +262,7 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (R <= 64 && !(flags & MLA_FLAG_WARP_MMA)) {
+  if (use_tc) {
     CUtensorMap qmap;
     rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, q_strides);
     if (rc) return rc;

@@ -3,22 +3,29 @@
 //
 // Per CTA: one split-KV part of the scheduler's plan, all R = s_q * h_q / h_kv query rows
 // of one latent head.  Warp roles:
-//   warp 0      TMA producer: the query tile (4-D tensor map, once per sequence) and whole
-//               64-token latent pages (64 x 576 bf16) gathered through block_table into a
-//               two-stage ring ("OpenSourceWeek Day 1 - FlashMLA", section II.1: fixed
-//               64-token blocks).
-//   warp 1      MMA issuer (one thread) and TMEM owner:
-//                 S   = Q K^T              M = 128 query rows, N = 64 keys, K = 576
+//   warp 0      TMA producer: the query tile (4-D tensor map, once per sequence) and the
+//               latent pages gathered through block_table ("OpenSourceWeek Day 1 -
+//               FlashMLA", section II.1: fixed 64-token blocks), staged as 32-token
+//               half pages (32 x 576 bf16 = 36,864 B) in a 3- to 5-deep ring so that two
+//               to two and a half pages per SM are in flight from HBM.
+//   warp 1      MMA issuer (one thread) and TMEM owner, per 32-key chunk:
+//                 S   = Q K^T              M = 128 query rows, N = 32 keys, K = 576;
+//                                          up to 32 rows Q is the A operand in TMEM
+//                                          (tcgen05.cp once per sequence), so the
+//                                          tensor core reads only the key slab from
+//                                          shared memory
 //                 O^T += V^T P^T           M = 128 value columns (x 4 blocks), N = R_pad,
-//                                          K = 64 keys; V = the page's first 512 columns
+//                                          K = 32 keys; V = the chunk's first 512 columns
 //               (absorbed-query score over the whole latent row, dpshk.com notes 2.1).
 //   warps 2-5   softmax / correction / epilogue warpgroup: thread = query row for S,
 //               thread = value column for O^T.  Online softmax (same notes, 2.2) with the
 //               running maximum refreshed only when it grows by more than 8 in log2 units;
 //               O^T and the row sum always share the maximum they were scaled with, so the
 //               result is exact.
-// Accumulating O transposed keeps TMEM at 128 (S, double-buffered) + 4 * R_pad (O^T)
-// columns, and lets V be read straight from the TMA page tile as an MN-major operand.
+// Accumulating O transposed keeps TMEM at 64 (S, double-buffered) + 4 * R_pad (O^T)
+// columns, and lets V be read straight from the TMA chunk tile as an MN-major operand.
+// QK of chunk n+1 is issued before PV of chunk n, so the softmax of one chunk overlaps
+// tensor-core work on the next.
 // Rows R .. 127 of the S tile read whatever follows the query tile in shared memory; they
 // are never used.
 //
@@ -32,18 +39,24 @@ namespace pagedmla {
 template <int RP>
 struct TcNarrow {
   static constexpr int kThreads = 192;
-  static constexpr int NQ = RP <= 32 ? 2 : 1;  // query tile buffers
-  static constexpr int NP = RP <= 32 ? 2 : 1;  // P tile buffers
-  static constexpr int kStages = 2;            // page ring (also the S double buffer)
-  static constexpr int kQBlock = RP * 128;     // one 64-column block of the query tile
+  static constexpr int KC = 32;                          // keys per chunk (half a page)
+  static constexpr int kChunkBlock = KC * 128;           // one 64-column block of a chunk
+  static constexpr int kChunkBytes = kColBlocks * kChunkBlock;  // 36,864 B
+  // Up to 32 rows the query tile lives in TMEM (the A operand of S = Q K^T), copied there
+  // once per sequence, so each QK MMA reads only its 1 KB key slab from shared memory.
+  static constexpr bool kQinTmem = RP <= 32;
+  static constexpr int NS = RP == 64 ? 3 : (RP == 48 ? 4 : 5);  // chunk ring depth
+  static constexpr int NQ = 1;                           // shared-memory query tile buffers
+  static constexpr int NP = 2;                           // P tile buffers
+  static constexpr int kQBlock = RP * 128;               // one 64-column block of the query tile
   static constexpr int kQBytes = kColBlocks * kQBlock;
-  static constexpr int kPBytes = RP * 128;
+  static constexpr int kPBytes = RP * 128;               // 32 keys per 128-byte row (first half)
   static constexpr int kOffQ = 0;
   static constexpr int kOffP = NQ * kQBytes;
-  static constexpr int kOffPages = ((kOffP + NP * kPBytes + 1023) / 1024) * 1024;
-  static constexpr int kOffRows = kOffPages + kStages * kPageBytes;  // l, m, alpha [64] each
+  static constexpr int kOffRing = ((kOffP + NP * kPBytes + 1023) / 1024) * 1024;
+  static constexpr int kOffRows = kOffRing + NS * kChunkBytes;  // l, m, alpha [64] each
   enum {
-    FULL = 0, EMPTY = FULL + kStages, QFULL = EMPTY + kStages, QFREE = QFULL + NQ,
+    FULL = 0, EMPTY = FULL + NS, QFULL = EMPTY + NS, QFREE = QFULL + NQ,
     SFULL = QFREE + NQ, SFREE = SFULL + 2, PFULL = SFREE + 2, PFREE = PFULL + NP,
     OFULL = PFREE + NP, OFREE = OFULL + 1, FINAL = OFREE + 1, NBARS = FINAL + 1
   };
@@ -52,7 +65,9 @@ struct TcNarrow {
   static constexpr int kOffAbort = kOffTmem + 8;
   static constexpr int kSmemBytes = kOffAbort + 8 + 1024;  // + slack for 1 KB alignment
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTmemO = 128;  // O^T blocks start after the two S buffers
+  static constexpr uint32_t kTmemO = 2 * KC;  // O^T blocks start after the two S buffers
+  static constexpr uint32_t kTmemQ = kTmemCols - kD / 2;  // Q: 288 columns (2 bf16 each)
+  static_assert(!kQinTmem || kTmemO + 4 * RP <= kTmemQ, "tensor memory budget with Q");
   static_assert(RP % 16 == 0 && RP >= 16 && RP <= 64, "rows per tile");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
   static_assert(kTmemO + 4 * RP <= kTmemCols, "tensor memory budget");
@@ -61,18 +76,18 @@ struct TcNarrow {
 };
 
 struct Segment {
-  int seq, L, t0, t1, npages;
+  int seq, L, t0, t1, nch;  // nch = 32-key chunks in [t0, t1); t0 is page aligned
 };
 
 // One sequence piece of a part; the narrow kernel holds all query rows, so causal
-// visibility never trims whole pages (the last row sees every key).
+// visibility never trims whole chunks (the last row sees every key).
 __device__ __forceinline__ Segment make_segment(const DecodeParams &p, const PartCursor &pc, int seq) {
   Segment s;
   s.seq = seq;
   s.L = p.seqlens[seq];
   s.t0 = seq == pc.bi ? pc.bt : 0;
   s.t1 = seq == pc.ei ? pc.et : s.L;
-  s.npages = s.t1 > s.t0 ? (s.t1 - s.t0 + kPage - 1) / kPage : 0;
+  s.nch = s.t1 > s.t0 ? (s.t1 - s.t0 + 31) / 32 : 0;
   return s;
 }
 
@@ -90,10 +105,10 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
   const uint32_t bar0 = sbase + T::kOffBar;
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
   volatile int *abort = reinterpret_cast<volatile int *>(smem + T::kOffAbort);
-  const uint32_t sQ = sbase + T::kOffQ, sP = sbase + T::kOffP, sPages = sbase + T::kOffPages;
+  const uint32_t sQ = sbase + T::kOffQ, sP = sbase + T::kOffP, sRing = sbase + T::kOffRing;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < T::kStages; ++s) {
+    for (int s = 0; s < T::NS; ++s) {
       mbar_init(bar(T::FULL + s), 1);
       mbar_init(bar(T::EMPTY + s), 1);
     }
@@ -124,21 +139,21 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
   const unsigned long long lim_ns = p.watchdog_ns;
 
   if (warp == 0) {
-    // ------------------------- producer: query tiles and pages -------------------------
+    // ------------------------- producer: query tiles and key chunks -------------------------
     if (lane == 0) {
       prefetch_tensormap(&kv_map);
       prefetch_tensormap(&q_map);
     }
     int it = 0, qs = 0;
-    int last_page[T::kStages], last_q[T::NQ];
+    int last_chunk[T::NS], last_q[T::NQ];
 #pragma unroll
-    for (int s = 0; s < T::kStages; ++s) last_page[s] = -1;
+    for (int s = 0; s < T::NS; ++s) last_chunk[s] = -1;
 #pragma unroll
     for (int s = 0; s < T::NQ; ++s) last_q[s] = -1;
     bool ok = true;
     for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
       const Segment sg = make_segment(p, pc, seq);
-      if (sg.npages == 0) continue;
+      if (sg.nch == 0) continue;
       const int qb = qs % T::NQ;
       int good = 1;
       if (lane == 0) {
@@ -155,25 +170,26 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
       }
       ok = __shfl_sync(0xffffffffu, good, 0) != 0;
       ++qs;
+      // chunk i of the segment = half (i & 1) of logical page t0/64 + i/2
       const int32_t *bt_row = p.block_table + (int64_t)seq * p.bt_stride + sg.t0 / kPage;
-      for (int base = 0; ok && base < sg.npages; base += 32) {
-        const int mine = base + lane < sg.npages ? bt_row[base + lane] : 0;
-        const int cnt = min(32, sg.npages - base);
+      for (int base = 0; ok && base < sg.nch; base += 32) {
+        const int mine = base + lane < sg.nch ? bt_row[(base + lane) >> 1] : 0;
+        const int cnt = min(32, sg.nch - base);
         for (int i = 0; ok && i < cnt; ++i, ++it) {
           const int phys = __shfl_sync(0xffffffffu, mine, i);
-          const int s = it & 1;
+          const int s = it % T::NS;
           int g2 = 1;
           if (lane == 0) {
-            if (!mbar_wait(bar(T::EMPTY + s), ((it >> 1) & 1) ^ 1, abort, p.status, lim_ns)) {
+            if (!mbar_wait(bar(T::EMPTY + s), ((it / T::NS) & 1) ^ 1, abort, p.status, lim_ns)) {
               g2 = 0;
             } else {
-              mbar_arrive_expect_tx(bar(T::FULL + s), kPageBytes);
-              const uint32_t dst = sPages + s * kPageBytes;
+              mbar_arrive_expect_tx(bar(T::FULL + s), T::kChunkBytes);
+              const uint32_t dst = sRing + s * T::kChunkBytes;
+              const int row = phys * kPage + ((base + i) & 1) * T::KC;
 #pragma unroll
               for (int c = 0; c < kColBlocks; ++c)
-                tma_load_3d(dst + c * kPageBlockBytes, &kv_map, bar(T::FULL + s), c * 64, kvh,
-                            phys * kPage);
-              last_page[s] = it;
+                tma_load_3d(dst + c * T::kChunkBlock, &kv_map, bar(T::FULL + s), c * 64, kvh, row);
+              last_chunk[s] = it;
             }
           }
           ok = __shfl_sync(0xffffffffu, g2, 0) != 0;
@@ -183,9 +199,9 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
     // every copy issued must land before the CTA exits
     if (lane == 0) {
       int never = 0;
-      for (int s = 0; s < T::kStages; ++s)
-        if (last_page[s] >= 0)
-          mbar_wait(bar(T::FULL + s), (last_page[s] >> 1) & 1, &never, p.status, lim_ns);
+      for (int s = 0; s < T::NS; ++s)
+        if (last_chunk[s] >= 0)
+          mbar_wait(bar(T::FULL + s), (last_chunk[s] / T::NS) & 1, &never, p.status, lim_ns);
       for (int s = 0; s < T::NQ; ++s)
         if (last_q[s] >= 0)
           mbar_wait(bar(T::QFULL + s), (last_q[s] / T::NQ) & 1, &never, p.status, lim_ns);
@@ -194,52 +210,66 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
   } else if (warp == 1) {
     // ------------------------- MMA issuer (one thread) -------------------------
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(128, 64, false, false);
+      const uint32_t idesc_qk = idesc_bf16_f32(128, T::KC, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, RP, true, false);
       int it = 0, qs = 0;
       bool ok = true;
       for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
         const Segment sg = make_segment(p, pc, seq);
-        if (sg.npages == 0) continue;
+        if (sg.nch == 0) continue;
         const int qb = qs % T::NQ;
         if (!mbar_wait(bar(T::QFULL + qb), (qs / T::NQ) & 1, abort, p.status, lim_ns)) {
           ok = false;
           break;
         }
         const uint32_t qtile = sQ + qb * T::kQBytes;
-        auto issue_qk = [&](int cur) -> bool {
-          const int s = cur & 1;
-          const uint32_t ph = (cur >> 1) & 1;
-          if (!mbar_wait(bar(T::FULL + s), ph, abort, p.status, lim_ns)) return false;
-          if (!mbar_wait(bar(T::SFREE + s), ph ^ 1, abort, p.status, lim_ns)) return false;
+        if constexpr (T::kQinTmem) {
+          // Q (rows on lanes, 576 columns as 288 packed pairs) into TMEM; the shared-memory
+          // tile is free again once the copies complete.
           tc_fence_after();
-          const uint32_t page = sPages + s * kPageBytes;
+#pragma unroll 4
+          for (int kk = 0; kk < kD / 16; ++kk)
+            tmem_cp_128x256b(tmem + T::kTmemQ + kk * 8,
+                             smem_desc_sw128(qtile + (kk >> 2) * T::kQBlock + (kk & 3) * 32, 16, 1024));
+          umma_commit(bar(T::QFREE + qb));
+        }
+        auto issue_qk = [&](int cur) -> bool {
+          const int s = cur % T::NS, sb = cur & 1;
+          if (!mbar_wait(bar(T::FULL + s), (cur / T::NS) & 1, abort, p.status, lim_ns)) return false;
+          if (!mbar_wait(bar(T::SFREE + sb), ((cur >> 1) & 1) ^ 1, abort, p.status, lim_ns)) return false;
+          tc_fence_after();
+          const uint32_t chunk = sRing + s * T::kChunkBytes;
+          const uint64_t b0 = smem_desc_sw128(chunk, 16, 1024);
 #pragma unroll 4
           for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (kk & 3) * 32;
-            const uint64_t a = smem_desc_sw128(qtile + (kk >> 2) * T::kQBlock + off, 16, 1024);
-            const uint64_t b = smem_desc_sw128(page + (kk >> 2) * kPageBlockBytes + off, 16, 1024);
-            umma_bf16(tmem + s * 64, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+            const uint32_t off = (kk >> 2) * T::kChunkBlock + (kk & 3) * 32;
+            const uint64_t b = b0 + (off >> 4);
+            if constexpr (T::kQinTmem) {
+              umma_bf16_ts(tmem + sb * T::KC, tmem + T::kTmemQ + kk * 8, b, idesc_qk, kk > 0 ? 1u : 0u);
+            } else {
+              const uint64_t a = smem_desc_sw128(qtile + (kk >> 2) * T::kQBlock + (kk & 3) * 32, 16, 1024);
+              umma_bf16(tmem + sb * T::KC, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+            }
           }
-          umma_commit(bar(T::SFULL + s));
+          umma_commit(bar(T::SFULL + sb));
           return true;
         };
         if (!issue_qk(it)) {
           ok = false;
           break;
         }
-        if (sg.npages == 1) umma_commit(bar(T::QFREE + qb));
-        for (int n = 0; n < sg.npages; ++n) {
+        if (!T::kQinTmem && sg.nch == 1) umma_commit(bar(T::QFREE + qb));
+        for (int n = 0; n < sg.nch; ++n) {
           const int cur = it + n;
-          if (n + 1 < sg.npages) {
+          if (n + 1 < sg.nch) {
             if (!issue_qk(cur + 1)) {
               ok = false;
               break;
             }
-            if (n + 2 == sg.npages) umma_commit(bar(T::QFREE + qb));
+            if (!T::kQinTmem && n + 2 == sg.nch) umma_commit(bar(T::QFREE + qb));
           }
-          const int pb = cur % T::NP;
-          if (!mbar_wait(bar(T::PFULL + pb), (cur / T::NP) & 1, abort, p.status, lim_ns)) {
+          const int pb = cur & 1;
+          if (!mbar_wait(bar(T::PFULL + pb), (cur >> 1) & 1, abort, p.status, lim_ns)) {
             ok = false;
             break;
           }
@@ -248,24 +278,24 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t page = sPages + (cur & 1) * kPageBytes;
+          const uint32_t chunk = sRing + (cur % T::NS) * T::kChunkBytes;
           const uint32_t ptile = sP + pb * T::kPBytes;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              // V^T block j: MN-major over the page's column blocks 2j, 2j+1 (8 KB apart),
+            for (int ks = 0; ks < T::KC / 16; ++ks) {
+              // V^T block j: MN-major over the chunk's column blocks 2j, 2j+1 (4 KB apart),
               // keys 16ks.. (two 8-row groups, 1 KB apart)
-              const uint64_t a = smem_desc_sw128(page + (2 * j) * kPageBlockBytes + ks * 2048,
-                                                 kPageBlockBytes, 1024);
+              const uint64_t a = smem_desc_sw128(chunk + (2 * j) * T::kChunkBlock + ks * 2048,
+                                                 T::kChunkBlock, 1024);
               const uint64_t b = smem_desc_sw128(ptile + ks * 32, 16, 1024);
               umma_bf16(tmem + T::kTmemO + j * RP, a, b, idesc_pv, (n > 0 || ks > 0) ? 1u : 0u);
             }
           umma_commit(bar(T::PFREE + pb));
-          umma_commit(bar(T::EMPTY + (cur & 1)));
-          if (n == sg.npages - 1) umma_commit(bar(T::OFULL));
+          umma_commit(bar(T::EMPTY + cur % T::NS));
+          if (n == sg.nch - 1) umma_commit(bar(T::OFULL));
         }
-        it += sg.npages;
+        it += sg.nch;
         ++qs;
       }
       // all issued tensor-core work completes before TMEM is released
@@ -293,7 +323,7 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
       const int nsplit = p.num_splits[seq + 1] - ns0;
       const int ord = seq == pc.bi ? pc.bord : 0;
       const int64_t acc_row0 = ((int64_t)(ns0 + ord) * p.h_kv + kvh) * p.R;
-      if (sg.npages == 0) {
+      if (sg.nch == 0) {
         for (int idx = tid; idx < p.R * kDV; idx += 128) {
           const int c = idx / kDV, dv = idx % kDV;
           if (nsplit == 1) {
@@ -315,21 +345,13 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
       if (active) lim = min(sg.t1, p.causal ? sg.L - (p.s_q - 1 - row / p.g) : sg.L);
       float m_used = -INFINITY, l = 0.f;
 
-      for (int n = 0; n < sg.npages; ++n) {
+      for (int n = 0; n < sg.nch; ++n) {
         const int cur = it + n;
         const int sb = cur & 1;
         ok = ok && mbar_wait(bar(T::SFULL + sb), (cur >> 1) & 1, abort, p.status, lim_ns);
         tc_fence_after();
-        float s[64];
-        if (ok && warp_rows) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float v[32];
-            tmem_ld32(lanes + sb * 64 + c * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
-          }
-        }
+        float s[T::KC];
+        if (ok && warp_rows) tmem_ld32(lanes + sb * T::KC, s);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(T::SFREE + sb));
@@ -337,10 +359,10 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
         bool need = false;
         float alpha = 1.f;
         if (ok && warp_rows) {
-          const int key0 = sg.t0 + n * kPage;
+          const int key0 = sg.t0 + n * T::KC;
           float mx = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
+          for (int i = 0; i < T::KC; ++i) {
             const float v = key0 + i < lim ? s[i] * p.scale_log2 : -INFINITY;
             s[i] = v;
             mx = fmaxf(mx, v);
@@ -354,18 +376,18 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
           const float base = m_used == -INFINITY ? 0.f : m_used;
           float sum = 0.f;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
+          for (int i = 0; i < T::KC; ++i) {
             s[i] = fast_exp2(s[i] - base);
             sum += s[i];
           }
           l = l * alpha + sum;
         }
-        const int pb = cur % T::NP;
-        ok = ok && mbar_wait(bar(T::PFREE + pb), ((cur / T::NP) & 1) ^ 1, abort, p.status, lim_ns);
+        const int pb = cur & 1;
+        ok = ok && mbar_wait(bar(T::PFREE + pb), ((cur >> 1) & 1) ^ 1, abort, p.status, lim_ns);
         if (ok && warp_rows && row < RP) {
           const uint32_t prow = sP + pb * T::kPBytes;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < T::KC / 8; ++c) {
             const uint32_t w0 = pack_bf16x2(s[8 * c + 0], s[8 * c + 1]);
             const uint32_t w1 = pack_bf16x2(s[8 * c + 2], s[8 * c + 3]);
             const uint32_t w2 = pack_bf16x2(s[8 * c + 4], s[8 * c + 5]);
@@ -378,7 +400,7 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
         // Rescale O^T when some row refreshed its maximum (after the previous PV is done).
         if (named_bar_or(1, 128, need && n > 0 && active)) {
           const int prv = cur - 1;
-          ok = ok && mbar_wait(bar(T::PFREE + prv % T::NP), (prv / T::NP) & 1, abort, p.status, lim_ns);
+          ok = ok && mbar_wait(bar(T::PFREE + (prv & 1)), (prv >> 1) & 1, abort, p.status, lim_ns);
           if (row < RP) a_sm[row] = active ? alpha : 1.f;
           named_bar_sync(1, 128);
           tc_fence_after();
@@ -445,7 +467,7 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
       named_bar_sync(1, 128);
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(T::OFREE));
-      it += sg.npages;
+      it += sg.nch;
       ++qs;
     }
   }
