@@ -309,8 +309,7 @@ def run_ours(args):
             ev[0].record()
         ops.mla_decode_paged(d["q"], d["k_cache"], d["block_table"], d["cache_seqlens"], 512, tile,
                              splits, softmax_scale=w.scale, causal=w.causal, workspace=d["ws"],
-                             out=d["out"], lse=d["lse"], skip_combine=True,
-                             warp_mma=args.kernel == "warp_mma")
+                             out=d["out"], lse=d["lse"], skip_combine=True, kernel=args.kernel)
         if ev is not None:
             ev[1].record()
         ops.mla_combine(splits, w.s_q, w.h_q, w.h_kv, tile.shape[0], d["ws"], d["out"], d["lse"])
@@ -387,7 +386,7 @@ def run_ours(args):
         tile, splits = ops.get_mla_metadata(sl, R, w.h_kv)
         out, lse = ops.flash_mla_with_kvcache(q, d0["k_cache"], bt, sl, 512, tile, splits,
                                               softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
-                                              warp_mma=args.kernel == "warp_mma")
+                                              kernel=args.kernel)
         hout.copy_(out, non_blocking=True)
         hlse.copy_(lse, non_blocking=True)
         torch.cuda.current_stream(dev).synchronize()
@@ -449,8 +448,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", default="tcgen05", choices=["tcgen05", "warp_mma"],
-                    help="decode kernel variant (warp_mma = the mma.sync baseline)")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "warp_mma"],
+                    help="decode kernel choice (auto = the library's choice by shape)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -60,13 +60,14 @@ extern "C" {
 #define MLA_D_QK 576              /* latent row width: 512 latent + 64 rope */
 #define MLA_D_V 512               /* value width: first 512 latent columns */
 #define MLA_TILE_FIELDS 8         /* int32 fields per tile_metadata entry */
-#define MLA_SPLIT_OVERHEAD 5      /* scheduler's fixed cost of one split, in pages */
+#define MLA_SPLIT_OVERHEAD_ROWS 32 /* a split costs max(1, ceil(R / 32)) pages in the plan */
 #define MLA_ROWS_PER_SM 64        /* query rows one SM serves; sets the part count */
 #define MLA_MAX_BATCH 16384       /* largest batch mla_get_metadata accepts */
 
 #define MLA_FLAG_SKIP_COMBINE 1u  /* mla_decode_paged: leave split partials unmerged */
-#define MLA_FLAG_WARP_MMA 2u      /* mla_decode_paged: run the warp-MMA (mma.sync) kernel
-                                     instead of the tcgen05 one (a baseline for comparison) */
+#define MLA_FLAG_WARP_MMA 2u      /* mla_decode_paged: force the warp-MMA (mma.sync) kernels */
+#define MLA_FLAG_TCGEN05 4u       /* mla_decode_paged: force the tcgen05 kernel (rows per
+                                     latent head <= 64 only) */
 
 typedef struct CUstream_st *mla_stream_t; /* identical to cudaStream_t */
 
@@ -89,12 +90,14 @@ MLA_API int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_
  * section V.2: get_mla_metadata(cache_seqlens, s_q*h_q//h_kv, h_kv) -> tile_metadata,
  * num_splits; the pages print its call only, the plan is this library's specification).
  *
- * Plan ("balanced cuts"): sequence b occupies OVH + ceil(L_b / 64) units of a cost axis
- * (OVH = MLA_SPLIT_OVERHEAD units first, then one unit per page).  With T the axis length
- * and payload = ceil(T / num_parts), part p covers [p*payload, (p+1)*payload) clipped to
- * T.  A cut at position x inside sequence i becomes the cursor (i, max(0, x - start_i -
- * OVH)) in pages, so a cut inside a sequence's overhead units moves the whole sequence to
- * the next part.  Each part does at most payload + OVH units of work.
+ * Plan ("balanced cuts"): with R = rows_per_kv_head and OVH = max(1, ceil(R / 32)) pages
+ * (the cost of one split: its fp32 partial of R rows, the query tile, the epilogue),
+ * sequence b occupies OVH + ceil(L_b / 64) units of a cost axis (its OVH units first, then
+ * one unit per page).  With T the axis length and payload = ceil(T / num_parts), part p
+ * covers [p*payload, (p+1)*payload) clipped to T.  A cut at position x inside sequence i
+ * becomes the cursor (i, max(0, x - start_i - OVH)) in pages, so a cut inside a
+ * sequence's overhead units moves the whole sequence to the next part.  Each part does at
+ * most payload + OVH units of work.
  *
  *   cache_seqlens  device int32 [batch], each >= 0
  *   tile_metadata  device int32 [num_parts][8], written:
@@ -103,13 +106,14 @@ MLA_API int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_
  *                  excluding (end_seq, end_token); tokens are multiples of 64
  *   num_splits     device int32 [batch + 1], written: prefix sums of the number of parts
  *                  touching each sequence (num_splits[0] = 0)
- * rows_per_kv_head and h_kv only enter through num_parts (pass mla_num_parts' result).
+ *   rows_per_kv_head  s_q * h_q / h_kv (sets OVH); num_parts from mla_num_parts.
  * Launches one small kernel on `stream`.  Errors: MLA_ERR_ARG (null pointer, batch < 1
- * or > MLA_MAX_BATCH, num_parts < 1), MLA_ERR_CUDA.  Negative lengths are not detected
+ * or > MLA_MAX_BATCH, rows_per_kv_head < 1, num_parts < 1), MLA_ERR_CUDA.  Negative lengths are not detected
  * on the device; mla_decode_paged's callers must pass lengths >= 0.
  */
-MLA_API int mla_get_metadata(const int32_t *cache_seqlens, int batch, int num_parts,
-                     int32_t *tile_metadata, int32_t *num_splits, mla_stream_t stream);
+MLA_API int mla_get_metadata(const int32_t *cache_seqlens, int batch, int rows_per_kv_head,
+                             int num_parts, int32_t *tile_metadata, int32_t *num_splits,
+                             mla_stream_t stream);
 
 /*
  * mla_workspace_size -- bytes of scratch mla_decode_paged needs: a 256-byte status
@@ -145,9 +149,10 @@ MLA_API int mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int num_pa
  *   lse            device fp32 [batch][h_q][s_q], contiguous (written; natural log)
  *   workspace      device scratch of mla_workspace_size bytes (see there)
  *   flags          0, or an OR of MLA_FLAG_SKIP_COMBINE (leave the split partials in
- *                  the workspace for a later mla_combine) and MLA_FLAG_WARP_MMA (use the
- *                  warp-MMA kernel; the default is the tcgen05 kernel where one exists for
- *                  the shape: up to 64 query rows per latent head)
+ *                  the workspace for a later mla_combine) and at most one kernel choice:
+ *                  MLA_FLAG_WARP_MMA or MLA_FLAG_TCGEN05.  By default the kernel follows
+ *                  the measured costs on B200: up to 16 rows per latent head the 16-row
+ *                  warp-MMA kernel, above that the 64-row-tile warp-MMA kernel.
  * Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.  A device
  * wait that times out (never in correct use) sets the workspace status word; read it
  * with mla_query_status.

@@ -11,7 +11,9 @@ plain Python.  Parity unpinned against the pages: it is pinned by its coverage i
 hand-worked cases.
 
 Specification ("balanced cuts")
-  PAGE = 64 tokens, OVH = 5 (fixed cost of one split, in pages)
+  PAGE = 64 tokens; OVH = max(1, ceil(R / 32)) with R = rows per latent head: the cost of
+  one split in pages (its fp32 partial of R rows grows with R; at least one page for the
+  query tile and the epilogue)
   Lay the sequences end to end on a cost axis: sequence b occupies OVH + ceil(L_b / 64)
   units, its OVH units first, then one unit per page.  T = total length of the axis.
   payload = ceil(T / num_parts).  Part p covers the axis interval
@@ -31,8 +33,12 @@ Outputs
 from __future__ import annotations
 
 PAGE = 64
-OVH = 5
 FIELDS = 8
+
+
+def overhead_pages(rows_per_kv_head: int) -> int:
+    """Fixed cost of one split, in pages: max(1, ceil(R / 32))."""
+    return max(1, -(-int(rows_per_kv_head) // 32))
 
 
 def num_parts_for(num_sms: int, rows_per_kv_head: int, h_kv: int, rows_per_sm: int = 64) -> int:
@@ -42,8 +48,9 @@ def num_parts_for(num_sms: int, rows_per_kv_head: int, h_kv: int, rows_per_sm: i
     return max(1, num_sms // (h_kv * m_blocks))
 
 
-def schedule(cache_seqlens, num_parts: int):
+def schedule(cache_seqlens, num_parts: int, rows_per_kv_head: int = 16):
     """Return (tile_metadata: list of num_parts 8-int lists, num_splits: list of B+1)."""
+    OVH = overhead_pages(rows_per_kv_head)
     lens = [int(x) for x in cache_seqlens]
     B = len(lens)
     cost = [OVH + -(-L // PAGE) for L in lens]
@@ -79,7 +86,8 @@ def schedule(cache_seqlens, num_parts: int):
     return tiles, num_splits
 
 
-def payload_of(cache_seqlens, num_parts: int) -> int:
+def payload_of(cache_seqlens, num_parts: int, rows_per_kv_head: int = 16) -> int:
+    OVH = overhead_pages(rows_per_kv_head)
     T = sum(OVH + -(-int(L) // PAGE) for L in cache_seqlens)
     return -(-T // num_parts)
 

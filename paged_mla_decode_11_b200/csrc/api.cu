@@ -3,6 +3,7 @@
 // allocates device memory or synchronises, except mla_query_status.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -170,14 +171,17 @@ int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_parts) {
   return MLA_OK;
 }
 
-int mla_get_metadata(const int32_t *cache_seqlens, int batch, int num_parts,
+int mla_get_metadata(const int32_t *cache_seqlens, int batch, int rows_per_kv_head, int num_parts,
                      int32_t *tile_metadata, int32_t *num_splits, mla_stream_t stream) {
   if (!cache_seqlens || !tile_metadata || !num_splits)
     return fail(MLA_ERR_ARG, "null pointer argument");
   if (batch < 1 || batch > MLA_MAX_BATCH)
     return fail(MLA_ERR_ARG, "batch must be in [1, %d] (got %d)", MLA_MAX_BATCH, batch);
+  if (rows_per_kv_head < 1 || rows_per_kv_head > (1 << 20))
+    return fail(MLA_ERR_ARG, "rows_per_kv_head must be in [1, 2^20]");
   if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
-  cudaError_t e = launch_metadata(cache_seqlens, batch, num_parts, tile_metadata, num_splits,
+  const int ovh = std::max(1, (rows_per_kv_head + MLA_SPLIT_OVERHEAD_ROWS - 1) / MLA_SPLIT_OVERHEAD_ROWS);
+  cudaError_t e = launch_metadata(cache_seqlens, batch, ovh, num_parts, tile_metadata, num_splits,
                                   reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "metadata kernel launch");
   return MLA_OK;
@@ -212,7 +216,10 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     return fail(MLA_ERR_ARG, "softmax_scale must be positive and finite");
-  if (flags & ~(MLA_FLAG_SKIP_COMBINE | MLA_FLAG_WARP_MMA)) return fail(MLA_ERR_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~(MLA_FLAG_SKIP_COMBINE | MLA_FLAG_WARP_MMA | MLA_FLAG_TCGEN05))
+    return fail(MLA_ERR_ARG, "unknown flags 0x%x", flags);
+  if ((flags & MLA_FLAG_WARP_MMA) && (flags & MLA_FLAG_TCGEN05))
+    return fail(MLA_ERR_ARG, "MLA_FLAG_WARP_MMA and MLA_FLAG_TCGEN05 are exclusive");
   for (int i = 0; i < 3; ++i)
     if (q_strides[i] < 0 || q_strides[i] % 8 != 0)
       return fail(MLA_ERR_ARG, "q strides must be non-negative multiples of 8 elements");
@@ -228,9 +235,15 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   if (workspace_bytes < wl.total)
     return fail(MLA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, wl.total);
 
-  const bool use_tc = R <= 64 && !(flags & MLA_FLAG_WARP_MMA);
+  // Kernel choice.  Measured on B200: a tcgen05 MMA costs at least a 128x128x16 tile, so for
+  // few query rows the 16-row warp-MMA tiles do the same work in fewer tensor cycles.
+  enum { kMma16, kMma64, kTc } kind = R <= 16 ? kMma16 : kMma64;
+  if (flags & MLA_FLAG_TCGEN05) {
+    if (R > 64) return fail(MLA_ERR_UNSUPPORTED, "the tcgen05 kernel handles up to 64 rows per latent head");
+    kind = kTc;
+  }
   CUtensorMap map;
-  rc = encode_kv_map(&map, k_cache, num_pages, h_kv, use_tc ? 32 : kPage);
+  rc = encode_kv_map(&map, k_cache, num_pages, h_kv, kind == kMma64 ? kPage : 32);
   if (rc) return rc;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -247,6 +260,8 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   p.R = R;
   p.block_table = block_table;
   p.bt_stride = block_table_stride;
+  p.kv_base = static_cast<const uint8_t *>(k_cache);
+  p.kv_token_bytes = int64_t(h_kv) * kD * 2;
   p.seqlens = cache_seqlens;
   p.tile_md = tile_metadata;
   p.num_parts = num_parts;
@@ -262,13 +277,13 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (use_tc) {
+  if (kind == kMma64) {
+    e = launch_decode_mma(map, p, st);
+  } else {
     CUtensorMap qmap;
     rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, q_strides);
     if (rc) return rc;
-    e = launch_decode_tc_narrow(map, qmap, p, st);
-  } else {
-    e = launch_decode_mma(map, p, st);
+    e = kind == kTc ? launch_decode_tc_narrow(map, qmap, p, st) : launch_decode_mma16(map, qmap, p, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   if (!(flags & MLA_FLAG_SKIP_COMBINE)) {

@@ -27,6 +27,8 @@ struct DecodeParams {
   int batch, s_q, h_q, h_kv, g, R; // g = h_q / h_kv, R = s_q * g rows per latent head
   const int32_t *block_table;
   int64_t bt_stride;
+  const uint8_t *kv_base;          // page pool base (for L2 prefetches)
+  int64_t kv_token_bytes;          // bytes of one token row: h_kv * 576 * 2
   const int32_t *seqlens;
   const int32_t *tile_md;
   int num_parts;
@@ -90,15 +92,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits until the phase with the given parity has completed.  Gives up after
 // `limit_ns` (checked every 256 polls) or as soon as *abort is set by another thread;
 // on giving up it records the time-out and raises *abort.  Returns true on success.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           int *status, unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     if ((i & 255u) == 0) {
       if (*abort) return false;
       if (global_ns() - t0 > limit_ns) {
@@ -120,6 +134,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       "[%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+// Bulk prefetch of a contiguous global range into L2 (16-byte aligned, size multiple of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {

@@ -344,6 +344,420 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
   __syncthreads();
 }
 
+// ---------------------------------------------------------------------------------------
+// Up to 16 query rows: the memory-bound decode shape.  mma.sync's 16-row tile fits these
+// rows exactly (a tcgen05 MMA pads them to 128 and costs at least a 128x128x16 tile).
+//   - Keys stream as 32-token half pages through a 5-deep TMA ring (two and a half pages
+//     per SM in flight from HBM).
+//   - QK warps 0-3: warp (kh, kn) keeps the A fragments of half the 576 columns of Q in
+//     registers for a whole sequence and computes the partial scores of 16 keys; the two
+//     column halves are summed through shared memory, then the online softmax runs and
+//     the kh = 0 warps write the bf16 P tile and the per-row rescale factors.
+//   - PV warps 4-7: O (16 rows x 128 value columns each) += P V from the same chunk.
+//   P tiles are double-buffered between the two groups with producer/consumer named
+//   barriers, so QK of chunk n+1 overlaps PV of chunk n.
+// ---------------------------------------------------------------------------------------
+struct Mma16 {
+  static constexpr int KC = 32;                           // keys per chunk
+  static constexpr int NS = 5;                            // ring depth
+  static constexpr int kQKWarps = 4;
+  static constexpr int kPVWarps = 4;
+  static constexpr int kThreads = (kQKWarps + kPVWarps + 1) * 32;  // + producer warp
+  static constexpr int kChunkBlock = KC * 128;            // one 64-column block: 4 KB
+  static constexpr int kChunkBytes = kColBlocks * kChunkBlock;
+  static constexpr int kOffRing = 0;
+  static constexpr int kOffQ = NS * kChunkBytes;          // 16 rows x 576, 9 blocks of 2 KB
+  static constexpr int kOffP = kOffQ + kColBlocks * 16 * 128;   // 2 x [16 rows x 32 keys]
+  static constexpr int kOffXS = kOffP + 2 * 16 * 128;           // score exchange [4][8][32] f32
+  static constexpr int kOffRed = kOffXS + 4 * 8 * 32 * 4;       // red_max[2][16]
+  static constexpr int kOffAlpha = kOffRed + 2 * 16 * 4;        // alpha[2][16]
+  static constexpr int kOffL = kOffAlpha + 2 * 16 * 4;          // l[2 segs][2 halves][16]
+  static constexpr int kOffM = kOffL + 2 * 2 * 16 * 4;          // m[2 segs][16]
+  static constexpr int kOffBar = kOffM + 2 * 16 * 4;
+  enum { FULL = 0, EMPTY = FULL + NS, QFULL = EMPTY + NS, QFREE = QFULL + 1, NBARS = QFREE + 1 };
+  static constexpr int kOffAbort = kOffBar + NBARS * 8;
+  static constexpr int kSmemBytes = kOffAbort + 16 + 1024;
+  // named barriers: 1 = QK warps; 2, 3 = P tile full; 4, 5 = P tile empty
+  static constexpr int kBarQK = 1, kBarPFull = 2, kBarPEmpty = 4;
+  static constexpr int kPairThreads = (kQKWarps + kPVWarps) * 32;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__global__ void __launch_bounds__(Mma16::kThreads, 1)
+    decode_mma16_kernel(const __grid_constant__ CUtensorMap kv_map,
+                        const __grid_constant__ CUtensorMap q_map, const DecodeParams p) {
+  using T = Mma16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int part = blockIdx.x, kvh = blockIdx.z;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + T::kOffBar;
+  auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+  volatile int *abort = reinterpret_cast<volatile int *>(smem + T::kOffAbort);
+  const uint32_t sRing = sbase + T::kOffRing, sQ = sbase + T::kOffQ, sP = sbase + T::kOffP;
+  float *xs = reinterpret_cast<float *>(smem + T::kOffXS);
+  float *red_max = reinterpret_cast<float *>(smem + T::kOffRed);
+  float *alpha_sm = reinterpret_cast<float *>(smem + T::kOffAlpha);
+  float *l_sm = reinterpret_cast<float *>(smem + T::kOffL);
+  float *m_sm = reinterpret_cast<float *>(smem + T::kOffM);
+  const unsigned long long lim_ns = p.watchdog_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < T::NS; ++s) {
+      mbar_init(bar(T::FULL + s), 1);
+      mbar_init(bar(T::EMPTY + s), T::kPVWarps);
+    }
+    mbar_init(bar(T::QFULL), 1);
+    mbar_init(bar(T::QFREE), T::kQKWarps);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const PartCursor pc = load_part(p.tile_md, part);
+  const int g4 = lane >> 2, c4 = lane & 3;
+
+  if (warp == T::kQKWarps + T::kPVWarps) {
+    // ------------------------- producer: query tiles and key chunks -------------------------
+    if (lane == 0) {
+      prefetch_tensormap(&kv_map);
+      prefetch_tensormap(&q_map);
+    }
+    int it = 0, qs = 0, last_q = -1;
+    int last_chunk[T::NS];
+#pragma unroll
+    for (int s = 0; s < T::NS; ++s) last_chunk[s] = -1;
+    bool ok = true;
+    for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
+      const int L = p.seqlens[seq];
+      const int t0 = seq == pc.bi ? pc.bt : 0;
+      const int t1 = seq == pc.ei ? pc.et : L;
+      const int nch = t1 > t0 ? (t1 - t0 + T::KC - 1) / T::KC : 0;
+      if (nch == 0) continue;
+      int good = 1;
+      if (lane == 0) {
+        if (!mbar_wait(bar(T::QFREE), (qs & 1) ^ 1, abort, p.status, lim_ns)) {
+          good = 0;
+        } else {
+          mbar_arrive_expect_tx(bar(T::QFULL), uint32_t(kColBlocks * p.R * 128));
+#pragma unroll
+          for (int c = 0; c < kColBlocks; ++c)
+            tma_load_4d(sQ + c * 16 * 128, &q_map, bar(T::QFULL), c * 64, kvh * p.g, 0, seq);
+          last_q = qs;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, good, 0) != 0;
+      ++qs;
+      const int32_t *bt_row = p.block_table + (int64_t)seq * p.bt_stride + t0 / kPage;
+      for (int base = 0; ok && base < nch; base += 32) {
+        const int mine = base + lane < nch ? bt_row[(base + lane) >> 1] : 0;
+        const int cnt = min(32, nch - base);
+        for (int i = 0; ok && i < cnt; ++i, ++it) {
+          const int phys = __shfl_sync(0xffffffffu, mine, i);
+          const int s = it % T::NS;
+          int g2 = 1;
+          if (lane == 0) {
+            if (!mbar_wait(bar(T::EMPTY + s), ((it / T::NS) & 1) ^ 1, abort, p.status, lim_ns)) {
+              g2 = 0;
+            } else {
+              mbar_arrive_expect_tx(bar(T::FULL + s), T::kChunkBytes);
+              const uint32_t dst = sRing + s * T::kChunkBytes;
+              const int row = phys * kPage + ((base + i) & 1) * T::KC;
+#pragma unroll
+              for (int c = 0; c < kColBlocks; ++c)
+                tma_load_3d(dst + c * T::kChunkBlock, &kv_map, bar(T::FULL + s), c * 64, kvh, row);
+              last_chunk[s] = it;
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, g2, 0) != 0;
+        }
+      }
+    }
+    if (lane == 0) {
+      int never = 0;
+      for (int s = 0; s < T::NS; ++s)
+        if (last_chunk[s] >= 0)
+          mbar_wait(bar(T::FULL + s), (last_chunk[s] / T::NS) & 1, &never, p.status, lim_ns);
+      if (last_q >= 0) mbar_wait(bar(T::QFULL), last_q & 1, &never, p.status, lim_ns);
+    }
+    __syncwarp();
+  } else if (warp < T::kQKWarps) {
+    // ------------------------- QK + softmax warps -------------------------
+    const int kh = warp >> 1, kn = warp & 1;
+    uint32_t qf[kD / 32][4];  // A fragments of this warp's 288 columns of Q
+    int it = 0, qs = 0;
+    bool ok = true;
+    for (int seq = pc.bi; part_has(pc, seq); ++seq) {
+      const int L = p.seqlens[seq];
+      const int t0 = seq == pc.bi ? pc.bt : 0;
+      const int t1 = seq == pc.ei ? pc.et : L;
+      const int nch = t1 > t0 ? (t1 - t0 + T::KC - 1) / T::KC : 0;
+      if (nch == 0) continue;
+      int lim[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = g4 + 8 * r;
+        lim[r] = row < p.R ? min(t1, p.causal ? L - (p.s_q - 1 - row / p.g) : L) : -1;
+      }
+      ok = ok && mbar_wait(bar(T::QFULL), qs & 1, abort, p.status, lim_ns);
+      if (ok) {
+#pragma unroll
+        for (int kk = 0; kk < kD / 32; ++kk) {
+          const int k = kh * (kD / 32) + kk;
+          ldsm_x4(sQ + (k >> 2) * (16 * 128) + sw128(lane & 15, (k & 3) * 2 + (lane >> 4)), qf[kk][0],
+                  qf[kk][1], qf[kk][2], qf[kk][3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(T::QFREE));
+
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      // S partial of one chunk: 16 rows x this warp's 16 keys over its 288 columns; key
+      // fragments loaded one k-step ahead, four independent accumulator chains
+      auto qk_chunk = [&](int cidx, float(&out)[2][4]) {
+        const uint32_t chunk = sRing + (cidx % T::NS) * T::kChunkBytes;
+        float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) out[0][e] = out[1][e] = 0.f;
+        auto kaddr = [&](int k) {
+          return chunk + (k >> 2) * T::kChunkBlock +
+                 sw128(kn * 16 + (lane & 7) + (lane >> 4) * 8, (k & 3) * 2 + ((lane >> 3) & 1));
+        };
+        uint32_t b[2][4];
+        ldsm_x4(kaddr(kh * (kD / 32)), b[0][0], b[0][1], b[0][2], b[0][3]);
+#pragma unroll
+        for (int kk = 0; kk < kD / 32; ++kk) {
+          if (kk + 1 < kD / 32)
+            ldsm_x4(kaddr(kh * (kD / 32) + kk + 1), b[(kk + 1) & 1][0], b[(kk + 1) & 1][1],
+                    b[(kk + 1) & 1][2], b[(kk + 1) & 1][3]);
+          float(&a0)[4] = (kk & 1) ? sd[0] : out[0];
+          float(&a1)[4] = (kk & 1) ? sd[1] : out[1];
+          mma_bf16_16816(a0, qf[kk], b[kk & 1][0], b[kk & 1][1]);
+          mma_bf16_16816(a1, qf[kk], b[kk & 1][2], b[kk & 1][3]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          out[0][e] += sd[0][e];
+          out[1][e] += sd[1][e];
+        }
+      };
+      float sc[2][4];
+      ok = ok && mbar_wait(bar(T::FULL + it % T::NS), (it / T::NS) & 1, abort, p.status, lim_ns);
+      if (ok) qk_chunk(it, sc);
+      for (int n = 0; n < nch; ++n, ++it) {
+        const int pb = it & 1;
+        // issue the next chunk's QK before this chunk's softmax, so the tensor work of
+        // chunk n+1 overlaps the exchange, softmax and hand-off of chunk n
+        float sn[2][4];
+        if (n + 1 < nch) {
+          ok = ok && mbar_wait(bar(T::FULL + (it + 1) % T::NS), ((it + 1) / T::NS) & 1, abort, p.status, lim_ns);
+          if (ok) qk_chunk(it + 1, sn);
+        }
+        // sum the two column halves
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xs[(warp * 8 + e) * 32 + lane] = sc[e >> 2][e & 3];
+        named_bar_sync(T::kBarQK, T::kQKWarps * 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sc[e >> 2][e & 3] += xs[((warp ^ 2) * 8 + e) * 32 + lane];
+        // mask, log2-domain scale, row maximum over the chunk's 32 keys
+        const int key0 = t0 + n * T::KC + kn * 16 + c4 * 2;
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = e >> 1;
+            const float v = key0 + t * 8 + (e & 1) < lim[r] ? sc[t][e] * p.scale_log2 : -INFINITY;
+            sc[t][e] = v;
+            mx[r] = fmaxf(mx[r], v);
+          }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+          mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+        }
+        if (kh == 0 && c4 == 0) {
+          red_max[kn * 16 + g4] = mx[0];
+          red_max[kn * 16 + g4 + 8] = mx[1];
+        }
+        named_bar_sync(T::kBarQK, T::kQKWarps * 32);
+        float alpha[2], base[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float mn = fmaxf(m[r], fmaxf(red_max[g4 + 8 * r], red_max[16 + g4 + 8 * r]));
+          base[r] = mn == -INFINITY ? 0.f : mn;
+          alpha[r] = fast_exp2(m[r] - base[r]);
+          m[r] = mn;
+        }
+        // P tile (and the rescale factors) into buffer pb once the PV warps are done with it
+        if (it >= 2) named_bar_sync(T::kBarPEmpty + pb, T::kPairThreads);
+        if (kh == 0) {
+          const uint32_t ptile = sP + pb * (16 * 128);
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const float p0 = fast_exp2(sc[t][0] - base[0]), p1 = fast_exp2(sc[t][1] - base[0]);
+            const float p2 = fast_exp2(sc[t][2] - base[1]), p3 = fast_exp2(sc[t][3] - base[1]);
+            l[0] = (t == 0 ? l[0] * alpha[0] : l[0]) + p0 + p1;
+            l[1] = (t == 0 ? l[1] * alpha[1] : l[1]) + p2 + p3;
+            const int kl = kn * 16 + t * 8 + c4 * 2;
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(ptile + sw128(g4, kl / 8) + (kl % 8) * 2),
+                         "r"(pack_bf16x2(p0, p1)));
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(ptile + sw128(g4 + 8, kl / 8) + (kl % 8) * 2),
+                         "r"(pack_bf16x2(p2, p3)));
+          }
+          if (kn == 0 && c4 == 0) {
+            alpha_sm[pb * 16 + g4] = alpha[0];
+            alpha_sm[pb * 16 + g4 + 8] = alpha[1];
+          }
+          if (n == nch - 1) {
+            // per-half row sums and the row maximum for the epilogue of this sequence
+            float lr[2] = {l[0], l[1]};
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              lr[r] += __shfl_xor_sync(0xffffffffu, lr[r], 1);
+              lr[r] += __shfl_xor_sync(0xffffffffu, lr[r], 2);
+            }
+            if (c4 == 0) {
+              l_sm[((qs & 1) * 2 + kn) * 16 + g4] = lr[0];
+              l_sm[((qs & 1) * 2 + kn) * 16 + g4 + 8] = lr[1];
+              if (kn == 0) {
+                m_sm[(qs & 1) * 16 + g4] = m[0];
+                m_sm[(qs & 1) * 16 + g4 + 8] = m[1];
+              }
+            }
+          }
+        }
+        named_bar_arrive(T::kBarPFull + pb, T::kPairThreads);
+        if (n + 1 < nch) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            sc[0][e] = sn[0][e];
+            sc[1][e] = sn[1][e];
+          }
+        }
+      }
+      ++qs;
+    }
+    // consume the last two P-empty signals so every named-barrier arrival is matched
+    for (int c = max(it - 2, 0); c < it; ++c) named_bar_sync(T::kBarPEmpty + (c & 1), T::kPairThreads);
+  } else {
+    // ------------------------- PV warps -------------------------
+    const int v = warp - T::kQKWarps;  // value columns 128 v .. 128 v + 127
+    int it = 0, qs = 0;
+    bool ok = true;
+    for (int seq = pc.bi; part_has(pc, seq); ++seq) {
+      const int L = p.seqlens[seq];
+      const int t0 = seq == pc.bi ? pc.bt : 0;
+      const int t1 = seq == pc.ei ? pc.et : L;
+      const int nch = t1 > t0 ? (t1 - t0 + T::KC - 1) / T::KC : 0;
+      const int ns0 = p.num_splits[seq];
+      const int nsplit = p.num_splits[seq + 1] - ns0;
+      const int ord = seq == pc.bi ? pc.bord : 0;
+      const int64_t acc_row0 = ((int64_t)(ns0 + ord) * p.h_kv + kvh) * p.R;
+      if (nch == 0) {
+        const int tid = threadIdx.x - T::kQKWarps * 32;
+        for (int idx = tid; idx < p.R * kDV; idx += T::kPVWarps * 32) {
+          const int c = idx / kDV, dv = idx % kDV;
+          if (nsplit == 1)
+            p.out[(((int64_t)seq * p.s_q + c / p.g) * p.h_q + kvh * p.g + c % p.g) * kDV + dv] =
+                __float2bfloat16(0.f);
+          else
+            p.o_accum[(acc_row0 + c) * kDV + dv] = 0.f;
+        }
+        if (tid < p.R) {
+          if (nsplit == 1)
+            p.lse[((int64_t)seq * p.h_q + kvh * p.g + tid % p.g) * p.s_q + tid / p.g] = -INFINITY;
+          else
+            p.lse_accum[acc_row0 + tid] = -INFINITY;
+        }
+        continue;
+      }
+      float o[16][4];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+      for (int n = 0; n < nch; ++n, ++it) {
+        const int s = it % T::NS, pb = it & 1;
+        named_bar_sync(T::kBarPFull + pb, T::kPairThreads);
+        const float a0 = alpha_sm[pb * 16 + g4], a1 = alpha_sm[pb * 16 + g4 + 8];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          o[j][0] *= a0;
+          o[j][1] *= a0;
+          o[j][2] *= a1;
+          o[j][3] *= a1;
+        }
+        const uint32_t chunk = sRing + s * T::kChunkBytes;
+        const uint32_t ptile = sP + pb * (16 * 128);
+        ok = ok && !*abort;
+        if (ok) {
+#pragma unroll
+          for (int ks = 0; ks < T::KC / 16; ++ks) {
+            // all fragments of this 16-key step first, then the 16 independent MMAs
+            uint32_t a[4], b[8][4];
+            ldsm_x4(ptile + sw128(lane & 15, ks * 2 + (lane >> 4)), a[0], a[1], a[2], a[3]);
+            const int key = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int jp = 0; jp < 8; ++jp) {
+              const int dv0 = v * 128 + jp * 16;
+              ldsm_x4_t(chunk + (dv0 / 64) * T::kChunkBlock + sw128(key, (dv0 % 64) / 8 + (lane >> 4)), b[jp][0],
+                        b[jp][1], b[jp][2], b[jp][3]);
+            }
+#pragma unroll
+            for (int jp = 0; jp < 8; ++jp) {
+              mma_bf16_16816(o[2 * jp], a, b[jp][0], b[jp][1]);
+              mma_bf16_16816(o[2 * jp + 1], a, b[jp][2], b[jp][3]);
+            }
+          }
+        }
+        named_bar_arrive(T::kBarPEmpty + pb, T::kPairThreads);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(T::EMPTY + s));
+      }
+      // ---- epilogue: O / l -> output (or fp32 split partial), natural-log LSE ----
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = g4 + 8 * r;
+        if (row >= p.R || !ok) continue;
+        const float lt = l_sm[((qs & 1) * 2) * 16 + row] + l_sm[((qs & 1) * 2 + 1) * 16 + row];
+        const float mr = m_sm[(qs & 1) * 16 + row];
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const int sq = row / p.g, h = kvh * p.g + row % p.g;
+        const float lse_v = lt > 0.f ? (mr + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+        if (nsplit == 1) {
+          __nv_bfloat16 *orow = p.out + (((int64_t)seq * p.s_q + sq) * p.h_q + h) * kDV + v * 128 + c4 * 2;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            *reinterpret_cast<uint32_t *>(orow + j * 8) = pack_bf16x2(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
+          if (v == 0 && c4 == 0) p.lse[((int64_t)seq * p.h_q + h) * p.s_q + sq] = lse_v;
+        } else {
+          float *orow = p.o_accum + (acc_row0 + row) * kDV + v * 128 + c4 * 2;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            *reinterpret_cast<float2 *>(orow + j * 8) = make_float2(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
+          if (v == 0 && c4 == 0) p.lse_accum[acc_row0 + row] = lse_v;
+        }
+      }
+      ++qs;
+    }
+  }
+  __syncthreads();
+}
+
+cudaError_t launch_decode_mma16(const CUtensorMap &kv_map, const CUtensorMap &q_map, const DecodeParams &p,
+                                cudaStream_t stream) {
+  using T = Mma16;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(decode_mma16_kernel), T::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.num_parts, 1, p.h_kv);
+  decode_mma16_kernel<<<grid, T::kThreads, T::kSmemBytes, stream>>>(kv_map, q_map, p);
+  return cudaGetLastError();
+}
+
 template <int BM, int DVS>
 static cudaError_t launch_mma(const CUtensorMap &map, const DecodeParams &p, int m_blocks,
                               cudaStream_t stream) {
@@ -357,7 +771,6 @@ static cudaError_t launch_mma(const CUtensorMap &map, const DecodeParams &p, int
 }
 
 cudaError_t launch_decode_mma(const CUtensorMap &map, const DecodeParams &p, cudaStream_t stream) {
-  if (p.R <= 16) return launch_mma<16, 8>(map, p, 1, stream);
   return launch_mma<64, 2>(map, p, (p.R + 63) / 64, stream);
 }
 

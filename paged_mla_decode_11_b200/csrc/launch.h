@@ -13,9 +13,11 @@ namespace pagedmla {
 // launches inside CUDA-graph capture make no attribute calls.
 cudaError_t set_smem_once(const void *kernel, int bytes);
 
-cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, int32_t *tile_md,
+cudaError_t launch_metadata(const int32_t *seqlens, int batch, int ovh, int num_parts, int32_t *tile_md,
                             int32_t *num_splits, cudaStream_t stream);
 cudaError_t launch_decode_mma(const CUtensorMap &map, const DecodeParams &p, cudaStream_t stream);
+cudaError_t launch_decode_mma16(const CUtensorMap &kv_map, const CUtensorMap &q_map, const DecodeParams &p,
+                                cudaStream_t stream);
 cudaError_t launch_decode_tc_narrow(const CUtensorMap &kv_map, const CUtensorMap &q_map,
                                     const DecodeParams &p, cudaStream_t stream);
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,

@@ -1,7 +1,7 @@
 // Split-KV tile scheduler (the pages' get_mla_metadata: "OpenSourceWeek Day 1 -
 // FlashMLA", section V.2, which shows only its call).  Plan ("balanced cuts", specified
-// in pagedmla.h): sequence b occupies OVH + ceil(L_b / 64) units of a cost axis (its OVH
-// units first, then one unit per page); with T the axis length and
+// in pagedmla.h): with OVH = max(1, ceil(R / 32)) pages per split, sequence b occupies
+// OVH + ceil(L_b / 64) units of a cost axis (its OVH units first, then one unit per page); with T the axis length and
 // payload = ceil(T / num_parts), part p covers [p * payload, (p + 1) * payload) clipped
 // to T.  Position x maps to the cursor (i, max(0, x - start_i - OVH)) of the sequence i
 // holding it, or (B, 0) at the end.
@@ -14,7 +14,6 @@
 
 namespace pagedmla {
 
-constexpr int kOvh = MLA_SPLIT_OVERHEAD;
 constexpr int kMetaThreads = 512;
 
 // Exclusive block-wide prefix sum of one value per thread; *total receives the sum.
@@ -46,7 +45,7 @@ __device__ long long block_exclusive_scan(long long v, long long *scratch, long 
 }
 
 __global__ void __launch_bounds__(kMetaThreads)
-    metadata_kernel(const int32_t *__restrict__ seqlens, int batch, int num_parts,
+    metadata_kernel(const int32_t *__restrict__ seqlens, int batch, int ovh, int num_parts,
                     int32_t *__restrict__ tile_md, int32_t *__restrict__ num_splits) {
   extern __shared__ long long start[];  // [batch + 1]
   __shared__ long long scratch[32];
@@ -55,12 +54,12 @@ __global__ void __launch_bounds__(kMetaThreads)
 
   // 1. start_b = exclusive prefix sum of (OVH + pages_b)
   long long mine = 0;
-  for (int b = lo; b < hi; ++b) mine += kOvh + (max(seqlens[b], 0) + kPage - 1) / kPage;
+  for (int b = lo; b < hi; ++b) mine += ovh + (max(seqlens[b], 0) + kPage - 1) / kPage;
   long long total;
   long long run = block_exclusive_scan(mine, scratch, &total);
   for (int b = lo; b < hi; ++b) {
     start[b] = run;
-    run += kOvh + (max(seqlens[b], 0) + kPage - 1) / kPage;
+    run += ovh + (max(seqlens[b], 0) + kPage - 1) / kPage;
   }
   if (threadIdx.x == 0) start[batch] = total;
   __syncthreads();
@@ -85,10 +84,10 @@ __global__ void __launch_bounds__(kMetaThreads)
           else z = mid - 1;
         }
         ci[e] = a;
-        ck[e] = max(0ll, x - start[a] - kOvh);
+        ck[e] = max(0ll, x - start[a] - ovh);
       }
     }
-    const int ord = ck[0] > 0 ? int(p - (start[ci[0]] + kOvh) / payload) : 0;
+    const int ord = ck[0] > 0 ? int(p - (start[ci[0]] + ovh) / payload) : 0;
     int32_t *t = tile_md + p * 8;
     t[0] = ci[0];
     t[1] = int32_t(ck[0] * kPage);
@@ -103,17 +102,17 @@ __global__ void __launch_bounds__(kMetaThreads)
   // 3. parts touching sequence b: 1 + cuts strictly inside its page units
   long long cnt = 0;
   for (int b = lo; b < hi; ++b)
-    cnt += 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + kOvh) / payload);
+    cnt += 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + ovh) / payload);
   long long all;
   run = block_exclusive_scan(cnt, scratch, &all);
   if (threadIdx.x == 0) num_splits[0] = 0;
   for (int b = lo; b < hi; ++b) {
-    run += 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + kOvh) / payload);
+    run += 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + ovh) / payload);
     num_splits[b + 1] = int32_t(run);
   }
 }
 
-cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, int32_t *tile_md,
+cudaError_t launch_metadata(const int32_t *seqlens, int batch, int ovh, int num_parts, int32_t *tile_md,
                             int32_t *num_splits, cudaStream_t stream) {
   const size_t smem = size_t(batch + 1) * sizeof(long long);
   if (smem > 48 * 1024) {
@@ -121,7 +120,7 @@ cudaError_t launch_metadata(const int32_t *seqlens, int batch, int num_parts, in
                                   int((MLA_MAX_BATCH + 1) * sizeof(long long)));
     if (e != cudaSuccess) return e;
   }
-  metadata_kernel<<<1, kMetaThreads, smem, stream>>>(seqlens, batch, num_parts, tile_md, num_splits);
+  metadata_kernel<<<1, kMetaThreads, smem, stream>>>(seqlens, batch, ovh, num_parts, tile_md, num_splits);
   return cudaGetLastError();
 }
 

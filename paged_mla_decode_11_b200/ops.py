@@ -29,6 +29,8 @@ MLA_OK = 0
 MLA_ERR_TIMEOUT = -4
 MLA_FLAG_SKIP_COMBINE = 1
 MLA_FLAG_WARP_MMA = 2
+MLA_FLAG_TCGEN05 = 4
+KERNELS = {"auto": 0, "warp_mma": MLA_FLAG_WARP_MMA, "tcgen05": MLA_FLAG_TCGEN05}
 PAGE = 64
 D_QK = 576
 D_V = 512
@@ -63,7 +65,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         sig = {
             "mla_device_sm_count": [I, P],
             "mla_num_parts": [I, I, I, P],
-            "mla_get_metadata": [P, I, I, P, P, P],
+            "mla_get_metadata": [P, I, I, I, P, P, P],
             "mla_workspace_size": [I, I, I, I, I, P],
             "mla_decode_paged": [P, P, I, I, I, I, P, I64, I, I, P, I64, P, I, P, I, P,
                                  ctypes.c_float, I, P, P, P, ctypes.c_size_t, ctypes.c_uint, P],
@@ -130,7 +132,7 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, rows_per_kv_head: int, h_kv: i
     batch = cache_seqlens.shape[0]
     tile = torch.empty(num_parts, TILE_FIELDS, dtype=torch.int32, device=dev)
     splits = torch.empty(batch + 1, dtype=torch.int32, device=dev)
-    _check(load_library().mla_get_metadata(cache_seqlens.data_ptr(), batch, num_parts,
+    _check(load_library().mla_get_metadata(cache_seqlens.data_ptr(), batch, rows_per_kv_head, num_parts,
                                            tile.data_ptr(), splits.data_ptr(), _stream_ptr(dev)))
     return tile, splits
 
@@ -163,14 +165,15 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
                      num_splits: torch.Tensor, softmax_scale: Optional[float] = None,
                      causal: bool = False, workspace: Optional[torch.Tensor] = None,
                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                     skip_combine: bool = False, warp_mma: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+                     skip_combine: bool = False, kernel: str = "auto") -> Tuple[torch.Tensor, torch.Tensor]:
     """Paged MLA decode.  q [b, s_q, h_q, 576] bf16, k_cache [pages, 64, h_kv, 576] bf16,
     block_table [b, w] int32, cache_seqlens [b] int32.  Returns (out [b, s_q, h_q, dv]
     bf16, lse [b, h_q, s_q] fp32).  The default softmax_scale is 576 ** -0.5.
 
     Without ``workspace`` a per-(device, stream) scratch buffer is reused; calls that may
-    run concurrently on one stream's buffer must pass their own.  ``warp_mma`` selects the
-    warp-MMA (mma.sync) kernel instead of the tcgen05 one, as a baseline."""
+    run concurrently on one stream's buffer must pass their own.  ``kernel`` is "auto"
+    (the library's choice by shape), "warp_mma" or "tcgen05" (up to 64 rows per latent
+    head)."""
     _require_cuda(q, "q", torch.bfloat16)
     _require_cuda(k_cache, "k_cache", torch.bfloat16)
     _require_cuda(block_table, "block_table", torch.int32)
@@ -210,7 +213,9 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
     if workspace is None:
         workspace = _default_workspace(need, dev)
     strides = (ctypes.c_int64 * 3)(q.stride(0), q.stride(1), q.stride(2))
-    flags = (MLA_FLAG_SKIP_COMBINE if skip_combine else 0) | (MLA_FLAG_WARP_MMA if warp_mma else 0)
+    if kernel not in KERNELS:
+        raise ValueError(f"kernel must be one of {sorted(KERNELS)}")
+    flags = (MLA_FLAG_SKIP_COMBINE if skip_combine else 0) | KERNELS[kernel]
     _check(load_library().mla_decode_paged(
         q.data_ptr(), strides, b, s_q, h_q, d, k_cache.data_ptr(), num_pages, page, h_kv,
         block_table.data_ptr(), block_table.stride(0), cache_seqlens.data_ptr(), dv,

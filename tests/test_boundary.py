@@ -57,7 +57,7 @@ def test_host_side_rejections(lib):
     assert lib.mla_workspace_size(0, 1, 16, 1, 10, ctypes.byref(out)) == -1
     n = ctypes.c_int(0)
     assert lib.mla_num_parts(0, 16, 1, ctypes.byref(n)) == -1
-    assert lib.mla_get_metadata(None, 4, 10, None, None, None) == -1
+    assert lib.mla_get_metadata(None, 4, 16, 10, None, None, None) == -1
     strides = (ctypes.c_int64 * 3)(576, 576, 576)
     # d != 576 and dv != 512 are refused before anything touches a device
     rc = lib.mla_decode_paged(16, strides, 1, 1, 16, 512, 16, 1, 64, 1, 16, 1, 16, 512, 16, 1, 16,

@@ -19,16 +19,17 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 def test_hand_worked_cases():
     spec = json.load(open(os.path.join(GOLDEN, "metadata_cases.json")))
     for case in spec["cases"]:
-        tiles, splits = M.schedule(case["seqlens"], case["num_parts"])
+        tiles, splits = M.schedule(case["seqlens"], case["num_parts"], case["rows_per_kv_head"])
         assert tiles == case["tiles"], case["work"]
         assert splits == case["num_splits"], case["work"]
 
 
-def check_plan(lens, num_parts, tiles, splits):
+def check_plan(lens, num_parts, tiles, splits, R=16):
     """Coverage: every page of every sequence exactly once, in order; split counts agree;
     no part does more than payload + OVH units of work; ordinals count earlier parts
     touching a sequence."""
-    payload = M.payload_of(lens, num_parts) + M.OVH
+    OVH = M.overhead_pages(R)
+    payload = M.payload_of(lens, num_parts, R) + OVH
     assert len(tiles) == num_parts and len(splits) == len(lens) + 1 and splits[0] == 0
     segs = M.segments(tiles, lens)
     cursor = {}
@@ -45,7 +46,7 @@ def check_plan(lens, num_parts, tiles, splits):
             seen_ord[b] += 1
             touched[b] += 1
             cursor[b] = t1
-            cost += -(-(t1 - t0) // M.PAGE) + M.OVH
+            cost += -(-(t1 - t0) // M.PAGE) + OVH
         assert cost <= payload
     for b, L in enumerate(lens):
         assert cursor.get(b, None) == L, f"sequence {b} not fully covered"
@@ -61,8 +62,9 @@ def test_random_plans_cover_everything(seed):
     B = rng.randint(1, 40)
     lens = [rng.choice([0, 1, 63, 64, 65, rng.randint(1, 5000), rng.randint(1, 70000)]) for _ in range(B)]
     num_parts = rng.randint(1, 160)
-    tiles, splits = M.schedule(lens, num_parts)
-    check_plan(lens, num_parts, tiles, splits)
+    R = rng.choice([1, 16, 33, 64, 128, 256, 1000])
+    tiles, splits = M.schedule(lens, num_parts, R)
+    check_plan(lens, num_parts, tiles, splits, R)
 
 
 def test_workload_plans():
@@ -70,8 +72,8 @@ def test_workload_plans():
     for w in W.WORKLOADS.values():
         lens = W._draw_seqlens(w, __import__("torch").Generator().manual_seed(0)).tolist()
         parts = M.num_parts_for(148, w.rows_per_kv_head, w.h_kv)
-        tiles, splits = M.schedule(lens, parts)
-        check_plan(lens, parts, tiles, splits)
+        tiles, splits = M.schedule(lens, parts, w.rows_per_kv_head)
+        check_plan(lens, parts, tiles, splits, w.rows_per_kv_head)
 
 
 def test_num_parts_formula():
@@ -81,3 +83,7 @@ def test_num_parts_formula():
     assert M.num_parts_for(148, 256, 1) == 37
     assert M.num_parts_for(148, 128, 2) == 37
     assert M.num_parts_for(4, 4096, 1) == 1
+
+
+def test_overhead_pages():
+    assert [M.overhead_pages(r) for r in (1, 16, 32, 33, 64, 128, 256)] == [1, 1, 1, 2, 2, 4, 8]
