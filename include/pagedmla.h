@@ -193,6 +193,35 @@ MLA_API int mla_query_status(void *workspace, mla_stream_t stream);
  */
 MLA_API int mla_watchdog_selftest(void *workspace, uint64_t timeout_ns, mla_stream_t stream);
 
+/*
+ * mla_decode_paged_static -- mla_decode_paged for callers that cannot allocate device
+ * memory (a framework that owns the whole memory budget, a server that reserves all
+ * memory at start-up, a real-time loop where an allocation could block or fail).  It
+ * allocates nothing: instead of a caller-provided workspace it uses one fixed device
+ * array of 8 MiB (MLA_STATIC_SCRATCH_BYTES) that the library carries and that every
+ * device which loads the library holds until the process exits.  Arguments, layouts and
+ * errors are those of mla_decode_paged without workspace/workspace_bytes; the caller
+ * still provides all inputs and outputs.  The pages describe no such variant; it exists
+ * for deployment only.
+ *   - A shape whose split scratch (mla_workspace_size) exceeds 8 MiB is rejected with
+ *     MLA_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call made while a device is current looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Each call clears the array's 256-byte status block on `stream`, then runs the
+ *     decode; the partial results in the array are overwritten by every call.
+ *   - All calls share the one array: calls that can overlap on the GPU (different
+ *     streams without ordering between them) race and corrupt each other's results.
+ *   - A device-side time-out is recorded in the array's status block and not reported.
+ */
+#define MLA_STATIC_SCRATCH_BYTES (8u << 20)
+MLA_API int mla_decode_paged_static(const void *q, const int64_t q_strides[3], int batch, int s_q,
+                                    int h_q, int d, const void *k_cache, int64_t num_pages,
+                                    int page_size, int h_kv, const int32_t *block_table,
+                                    int64_t block_table_stride, const int32_t *cache_seqlens,
+                                    int dv, const int32_t *tile_metadata, int num_parts,
+                                    const int32_t *num_splits, float softmax_scale, int causal,
+                                    void *out, float *lse, unsigned flags, mla_stream_t stream);
+
 /* Thread-local description of this thread's last error ("" when none). */
 MLA_API const char *mla_last_error_string(void);
 

@@ -134,6 +134,8 @@ int check_common(int batch, int s_q, int h_q, int h_kv, int dv) {
 
 namespace pagedmla {
 
+int record_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
 cudaError_t set_smem_once(const void *kernel, int bytes) {
   static std::mutex mu;
   static std::vector<std::pair<const void *, int>> done;  // (kernel, device)

@@ -9,6 +9,9 @@
 
 namespace pagedmla {
 
+// Records an error for mla_last_error_string() on this thread and returns `code`.
+int record_error(int code, const char *msg);
+
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device), so that
 // launches inside CUDA-graph capture make no attribute calls.
 cudaError_t set_smem_once(const void *kernel, int bytes);

@@ -39,7 +39,7 @@ TILE_FIELDS = 8
 EXPORTED = (
     "mla_device_sm_count", "mla_num_parts", "mla_get_metadata", "mla_workspace_size",
     "mla_decode_paged", "mla_combine", "mla_query_status", "mla_watchdog_selftest",
-    "mla_last_error_string",
+    "mla_last_error_string", "mla_decode_paged_static",
 )
 
 _lib = None
