@@ -347,44 +347,52 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
 // ---------------------------------------------------------------------------------------
 // Up to 16 query rows: the memory-bound decode shape.  mma.sync's 16-row tile fits these
 // rows exactly (a tcgen05 MMA pads them to 128 and costs at least a 128x128x16 tile).
-//   - Keys stream as 32-token half pages through a 5-deep TMA ring (two and a half pages
-//     per SM in flight from HBM).
-//   - QK warps 0-3: warp (kh, kn) keeps the A fragments of half the 576 columns of Q in
-//     registers for a whole sequence and computes the partial scores of 16 keys; the two
-//     column halves are summed through shared memory, then the online softmax runs and
-//     the kh = 0 warps write the bf16 P tile and the per-row rescale factors.
-//   - PV warps 4-7: O (16 rows x 128 value columns each) += P V from the same chunk.
-//   P tiles are double-buffered between the two groups with producer/consumer named
-//   barriers, so QK of chunk n+1 overlaps PV of chunk n.
+// Keys stream as 32-token half pages through a 5-deep TMA ring (two and a half pages per
+// SM in flight from HBM).  Three warp stages overlap across chunks:
+//   - S warps 0-3: warp (kh, kn) keeps the A fragments of half the 576 columns of Q in
+//     registers for a whole sequence and computes the partial scores of 16 keys of each
+//     chunk into a double-buffered shared-memory tile;
+//   - softmax warp 4: sums the two column halves, runs the online softmax (running max,
+//     rescale factor, row sums) and writes the bf16 P tile, double-buffered;
+//   - PV warps 5-8: O (16 rows x 128 value columns each) += P V from the same chunk.
+// Each hand-off is a producer/consumer named barrier pair (full / empty), so the S warps
+// run up to two chunks ahead of the softmax, which runs up to two chunks ahead of PV.
 // ---------------------------------------------------------------------------------------
 struct Mma16 {
   static constexpr int KC = 32;                           // keys per chunk
   static constexpr int NS = 5;                            // ring depth
-  static constexpr int kQKWarps = 4;
-  static constexpr int kPVWarps = 4;
-  static constexpr int kThreads = (kQKWarps + kPVWarps + 1) * 32;  // + producer warp
+  static constexpr int kSWarps = 4, kSmWarp = 4, kPVWarp0 = 5, kPVWarps = 4, kProducer = 9;
+  static constexpr int kThreads = 10 * 32;
   static constexpr int kChunkBlock = KC * 128;            // one 64-column block: 4 KB
   static constexpr int kChunkBytes = kColBlocks * kChunkBlock;
   static constexpr int kOffRing = 0;
   static constexpr int kOffQ = NS * kChunkBytes;          // 16 rows x 576, 9 blocks of 2 KB
-  static constexpr int kOffP = kOffQ + kColBlocks * 16 * 128;   // 2 x [16 rows x 32 keys]
-  static constexpr int kOffXS = kOffP + 2 * 16 * 128;           // score exchange [4][8][32] f32
-  static constexpr int kOffRed = kOffXS + 4 * 8 * 32 * 4;       // red_max[2][16]
-  static constexpr int kOffAlpha = kOffRed + 2 * 16 * 4;        // alpha[2][16]
-  static constexpr int kOffL = kOffAlpha + 2 * 16 * 4;          // l[2 segs][2 halves][16]
-  static constexpr int kOffM = kOffL + 2 * 2 * 16 * 4;          // m[2 segs][16]
+  static constexpr int kOffP = kOffQ + kColBlocks * 16 * 128;   // 2 x [16 rows x 32 keys] bf16
+  static constexpr int kOffS = kOffP + 2 * 16 * 128;            // 2 x [4 warps][8][32] f32 partial S
+  static constexpr int kOffAlpha = kOffS + 2 * 4 * 8 * 32 * 4;  // alpha[2][16]
+  static constexpr int kOffL = kOffAlpha + 2 * 16 * 4;          // l[2 segs][16]
+  static constexpr int kOffM = kOffL + 2 * 16 * 4;              // m[2 segs][16]
   static constexpr int kOffBar = kOffM + 2 * 16 * 4;
   enum { FULL = 0, EMPTY = FULL + NS, QFULL = EMPTY + NS, QFREE = QFULL + 1, NBARS = QFREE + 1 };
   static constexpr int kOffAbort = kOffBar + NBARS * 8;
   static constexpr int kSmemBytes = kOffAbort + 16 + 1024;
-  // named barriers: 1 = QK warps; 2, 3 = P tile full; 4, 5 = P tile empty
-  static constexpr int kBarQK = 1, kBarPFull = 2, kBarPEmpty = 4;
-  static constexpr int kPairThreads = (kQKWarps + kPVWarps) * 32;
+  // named barriers (id, id + 1 for the two buffers): S tile full / empty, P tile full / empty
+  static constexpr int kBarSFull = 1, kBarSEmpty = 3, kBarPFull = 5, kBarPEmpty = 7;
+  static constexpr int kSPair = (kSWarps + 1) * 32, kPPair = (kPVWarps + 1) * 32;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Token range and 32-key chunk count of sequence `seq` within part `pc`.
+__device__ __forceinline__ int chunk_range(const DecodeParams &p, const PartCursor &pc, int seq, int &L,
+                                           int &t0, int &t1) {
+  L = p.seqlens[seq];
+  t0 = seq == pc.bi ? pc.bt : 0;
+  t1 = seq == pc.ei ? pc.et : L;
+  return t1 > t0 ? (t1 - t0 + Mma16::KC - 1) / Mma16::KC : 0;
 }
 
 __global__ void __launch_bounds__(Mma16::kThreads, 1)
@@ -401,8 +409,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
   volatile int *abort = reinterpret_cast<volatile int *>(smem + T::kOffAbort);
   const uint32_t sRing = sbase + T::kOffRing, sQ = sbase + T::kOffQ, sP = sbase + T::kOffP;
-  float *xs = reinterpret_cast<float *>(smem + T::kOffXS);
-  float *red_max = reinterpret_cast<float *>(smem + T::kOffRed);
+  float *sbuf = reinterpret_cast<float *>(smem + T::kOffS);
   float *alpha_sm = reinterpret_cast<float *>(smem + T::kOffAlpha);
   float *l_sm = reinterpret_cast<float *>(smem + T::kOffL);
   float *m_sm = reinterpret_cast<float *>(smem + T::kOffM);
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
       mbar_init(bar(T::EMPTY + s), T::kPVWarps);
     }
     mbar_init(bar(T::QFULL), 1);
-    mbar_init(bar(T::QFREE), T::kQKWarps);
+    mbar_init(bar(T::QFREE), T::kSWarps);
     *abort = 0;
     fence_barrier_init();
   }
@@ -422,7 +429,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
   const PartCursor pc = load_part(p.tile_md, part);
   const int g4 = lane >> 2, c4 = lane & 3;
 
-  if (warp == T::kQKWarps + T::kPVWarps) {
+  if (warp == T::kProducer) {
     // ------------------------- producer: query tiles and key chunks -------------------------
     if (lane == 0) {
       prefetch_tensormap(&kv_map);
@@ -434,10 +441,8 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
     for (int s = 0; s < T::NS; ++s) last_chunk[s] = -1;
     bool ok = true;
     for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
-      const int L = p.seqlens[seq];
-      const int t0 = seq == pc.bi ? pc.bt : 0;
-      const int t1 = seq == pc.ei ? pc.et : L;
-      const int nch = t1 > t0 ? (t1 - t0 + T::KC - 1) / T::KC : 0;
+      int L, t0, t1;
+      const int nch = chunk_range(p, pc, seq, L, t0, t1);
       if (nch == 0) continue;
       int good = 1;
       if (lane == 0) {
@@ -486,24 +491,16 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
       if (last_q >= 0) mbar_wait(bar(T::QFULL), last_q & 1, &never, p.status, lim_ns);
     }
     __syncwarp();
-  } else if (warp < T::kQKWarps) {
-    // ------------------------- QK + softmax warps -------------------------
+  } else if (warp < T::kSWarps) {
+    // ------------------------- S warps: partial scores -------------------------
     const int kh = warp >> 1, kn = warp & 1;
     uint32_t qf[kD / 32][4];  // A fragments of this warp's 288 columns of Q
     int it = 0, qs = 0;
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
-      const int L = p.seqlens[seq];
-      const int t0 = seq == pc.bi ? pc.bt : 0;
-      const int t1 = seq == pc.ei ? pc.et : L;
-      const int nch = t1 > t0 ? (t1 - t0 + T::KC - 1) / T::KC : 0;
+      int L, t0, t1;
+      const int nch = chunk_range(p, pc, seq, L, t0, t1);
       if (nch == 0) continue;
-      int lim[2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int row = g4 + 8 * r;
-        lim[r] = row < p.R ? min(t1, p.causal ? L - (p.s_q - 1 - row / p.g) : L) : -1;
-      }
       ok = ok && mbar_wait(bar(T::QFULL), qs & 1, abort, p.status, lim_ns);
       if (ok) {
 #pragma unroll
@@ -515,152 +512,147 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(T::QFREE));
-
-      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-      // S partial of one chunk: 16 rows x this warp's 16 keys over its 288 columns; key
-      // fragments loaded one k-step ahead, four independent accumulator chains
-      auto qk_chunk = [&](int cidx, float(&out)[2][4]) {
-        const uint32_t chunk = sRing + (cidx % T::NS) * T::kChunkBytes;
-        float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) out[0][e] = out[1][e] = 0.f;
-        auto kaddr = [&](int k) {
-          return chunk + (k >> 2) * T::kChunkBlock +
-                 sw128(kn * 16 + (lane & 7) + (lane >> 4) * 8, (k & 3) * 2 + ((lane >> 3) & 1));
-        };
-        uint32_t b[2][4];
-        ldsm_x4(kaddr(kh * (kD / 32)), b[0][0], b[0][1], b[0][2], b[0][3]);
-#pragma unroll
-        for (int kk = 0; kk < kD / 32; ++kk) {
-          if (kk + 1 < kD / 32)
-            ldsm_x4(kaddr(kh * (kD / 32) + kk + 1), b[(kk + 1) & 1][0], b[(kk + 1) & 1][1],
-                    b[(kk + 1) & 1][2], b[(kk + 1) & 1][3]);
-          float(&a0)[4] = (kk & 1) ? sd[0] : out[0];
-          float(&a1)[4] = (kk & 1) ? sd[1] : out[1];
-          mma_bf16_16816(a0, qf[kk], b[kk & 1][0], b[kk & 1][1]);
-          mma_bf16_16816(a1, qf[kk], b[kk & 1][2], b[kk & 1][3]);
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          out[0][e] += sd[0][e];
-          out[1][e] += sd[1][e];
-        }
-      };
-      float sc[2][4];
-      ok = ok && mbar_wait(bar(T::FULL + it % T::NS), (it / T::NS) & 1, abort, p.status, lim_ns);
-      if (ok) qk_chunk(it, sc);
       for (int n = 0; n < nch; ++n, ++it) {
-        const int pb = it & 1;
-        // issue the next chunk's QK before this chunk's softmax, so the tensor work of
-        // chunk n+1 overlaps the exchange, softmax and hand-off of chunk n
-        float sn[2][4];
-        if (n + 1 < nch) {
-          ok = ok && mbar_wait(bar(T::FULL + (it + 1) % T::NS), ((it + 1) / T::NS) & 1, abort, p.status, lim_ns);
-          if (ok) qk_chunk(it + 1, sn);
-        }
-        // sum the two column halves
+        const int sb = it & 1;
+        ok = ok && mbar_wait(bar(T::FULL + it % T::NS), (it / T::NS) & 1, abort, p.status, lim_ns);
+        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if (ok) {
+          // key fragments loaded one k-step ahead; four independent accumulator chains
+          const uint32_t chunk = sRing + (it % T::NS) * T::kChunkBytes;
+          float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          auto kaddr = [&](int k) {
+            return chunk + (k >> 2) * T::kChunkBlock +
+                   sw128(kn * 16 + (lane & 7) + (lane >> 4) * 8, (k & 3) * 2 + ((lane >> 3) & 1));
+          };
+          uint32_t b[2][4];
+          ldsm_x4(kaddr(kh * (kD / 32)), b[0][0], b[0][1], b[0][2], b[0][3]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) xs[(warp * 8 + e) * 32 + lane] = sc[e >> 2][e & 3];
-        named_bar_sync(T::kBarQK, T::kQKWarps * 32);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sc[e >> 2][e & 3] += xs[((warp ^ 2) * 8 + e) * 32 + lane];
-        // mask, log2-domain scale, row maximum over the chunk's 32 keys
-        const int key0 = t0 + n * T::KC + kn * 16 + c4 * 2;
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
+          for (int kk = 0; kk < kD / 32; ++kk) {
+            if (kk + 1 < kD / 32)
+              ldsm_x4(kaddr(kh * (kD / 32) + kk + 1), b[(kk + 1) & 1][0], b[(kk + 1) & 1][1],
+                      b[(kk + 1) & 1][2], b[(kk + 1) & 1][3]);
+            float(&a0)[4] = (kk & 1) ? sd[0] : sc[0];
+            float(&a1)[4] = (kk & 1) ? sd[1] : sc[1];
+            mma_bf16_16816(a0, qf[kk], b[kk & 1][0], b[kk & 1][1]);
+            mma_bf16_16816(a1, qf[kk], b[kk & 1][2], b[kk & 1][3]);
+          }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int r = e >> 1;
-            const float v = key0 + t * 8 + (e & 1) < lim[r] ? sc[t][e] * p.scale_log2 : -INFINITY;
-            sc[t][e] = v;
+            sc[0][e] += sd[0][e];
+            sc[1][e] += sd[1][e];
+          }
+        }
+        if (it >= 2) named_bar_sync(T::kBarSEmpty + sb, T::kSPair);
+        float *dst = sbuf + (sb * 4 + warp) * 8 * 32;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dst[e * 32 + lane] = sc[e >> 2][e & 3];
+        named_bar_arrive(T::kBarSFull + sb, T::kSPair);
+      }
+      ++qs;
+    }
+    for (int c = max(it - 2, 0); c < it; ++c) named_bar_sync(T::kBarSEmpty + (c & 1), T::kSPair);
+  } else if (warp == T::kSmWarp) {
+    // ------------------------- softmax warp -------------------------
+    int it = 0, qs = 0;
+    for (int seq = pc.bi; part_has(pc, seq); ++seq) {
+      int L, t0, t1;
+      const int nch = chunk_range(p, pc, seq, L, t0, t1);
+      if (nch == 0) continue;
+      int lim[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = g4 + 8 * r;
+        lim[r] = row < p.R ? min(t1, p.causal ? L - (p.s_q - 1 - row / p.g) : L) : -1;
+      }
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      for (int n = 0; n < nch; ++n, ++it) {
+        const int sb = it & 1, pb = it & 1;
+        named_bar_sync(T::kBarSFull + sb, T::kSPair);
+        // this thread's 16 scores: key halves kn = 0, 1; per half 2 key tiles x 4 values
+        float sc[2][8];
+        const float *src = sbuf + sb * 4 * 8 * 32;
+#pragma unroll
+        for (int kn = 0; kn < 2; ++kn)
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            sc[kn][e] = src[(kn * 8 + e) * 32 + lane] + src[((2 + kn) * 8 + e) * 32 + lane];
+        named_bar_arrive(T::kBarSEmpty + sb, T::kSPair);
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int kn = 0; kn < 2; ++kn)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int r = (e >> 1) & 1;
+            const int key = t0 + n * T::KC + kn * 16 + (e >> 2) * 8 + c4 * 2 + (e & 1);
+            const float v = key < lim[r] ? sc[kn][e] * p.scale_log2 : -INFINITY;
+            sc[kn][e] = v;
             mx[r] = fmaxf(mx[r], v);
           }
+        float alpha[2], base[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
           mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-        }
-        if (kh == 0 && c4 == 0) {
-          red_max[kn * 16 + g4] = mx[0];
-          red_max[kn * 16 + g4 + 8] = mx[1];
-        }
-        named_bar_sync(T::kBarQK, T::kQKWarps * 32);
-        float alpha[2], base[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const float mn = fmaxf(m[r], fmaxf(red_max[g4 + 8 * r], red_max[16 + g4 + 8 * r]));
+          const float mn = fmaxf(m[r], mx[r]);
           base[r] = mn == -INFINITY ? 0.f : mn;
           alpha[r] = fast_exp2(m[r] - base[r]);
           m[r] = mn;
+          l[r] *= alpha[r];
         }
-        // P tile (and the rescale factors) into buffer pb once the PV warps are done with it
-        if (it >= 2) named_bar_sync(T::kBarPEmpty + pb, T::kPairThreads);
-        if (kh == 0) {
-          const uint32_t ptile = sP + pb * (16 * 128);
+        if (it >= 2) named_bar_sync(T::kBarPEmpty + pb, T::kPPair);
+        const uint32_t ptile = sP + pb * (16 * 128);
+#pragma unroll
+        for (int kn = 0; kn < 2; ++kn)
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            const float p0 = fast_exp2(sc[t][0] - base[0]), p1 = fast_exp2(sc[t][1] - base[0]);
-            const float p2 = fast_exp2(sc[t][2] - base[1]), p3 = fast_exp2(sc[t][3] - base[1]);
-            l[0] = (t == 0 ? l[0] * alpha[0] : l[0]) + p0 + p1;
-            l[1] = (t == 0 ? l[1] * alpha[1] : l[1]) + p2 + p3;
+            const float p0 = fast_exp2(sc[kn][t * 4 + 0] - base[0]), p1 = fast_exp2(sc[kn][t * 4 + 1] - base[0]);
+            const float p2 = fast_exp2(sc[kn][t * 4 + 2] - base[1]), p3 = fast_exp2(sc[kn][t * 4 + 3] - base[1]);
+            l[0] += p0 + p1;
+            l[1] += p2 + p3;
             const int kl = kn * 16 + t * 8 + c4 * 2;
             asm volatile("st.shared.b32 [%0], %1;" ::"r"(ptile + sw128(g4, kl / 8) + (kl % 8) * 2),
                          "r"(pack_bf16x2(p0, p1)));
             asm volatile("st.shared.b32 [%0], %1;" ::"r"(ptile + sw128(g4 + 8, kl / 8) + (kl % 8) * 2),
                          "r"(pack_bf16x2(p2, p3)));
           }
-          if (kn == 0 && c4 == 0) {
-            alpha_sm[pb * 16 + g4] = alpha[0];
-            alpha_sm[pb * 16 + g4 + 8] = alpha[1];
-          }
-          if (n == nch - 1) {
-            // per-half row sums and the row maximum for the epilogue of this sequence
-            float lr[2] = {l[0], l[1]};
+        if (c4 == 0) {
+          alpha_sm[pb * 16 + g4] = alpha[0];
+          alpha_sm[pb * 16 + g4 + 8] = alpha[1];
+        }
+        if (n == nch - 1) {
+          // row sums and the row maximum for the epilogue of this sequence
+          float lr[2] = {l[0], l[1]};
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              lr[r] += __shfl_xor_sync(0xffffffffu, lr[r], 1);
-              lr[r] += __shfl_xor_sync(0xffffffffu, lr[r], 2);
-            }
-            if (c4 == 0) {
-              l_sm[((qs & 1) * 2 + kn) * 16 + g4] = lr[0];
-              l_sm[((qs & 1) * 2 + kn) * 16 + g4 + 8] = lr[1];
-              if (kn == 0) {
-                m_sm[(qs & 1) * 16 + g4] = m[0];
-                m_sm[(qs & 1) * 16 + g4 + 8] = m[1];
-              }
-            }
+          for (int r = 0; r < 2; ++r) {
+            lr[r] += __shfl_xor_sync(0xffffffffu, lr[r], 1);
+            lr[r] += __shfl_xor_sync(0xffffffffu, lr[r], 2);
+          }
+          if (c4 == 0) {
+            l_sm[(qs & 1) * 16 + g4] = lr[0];
+            l_sm[(qs & 1) * 16 + g4 + 8] = lr[1];
+            m_sm[(qs & 1) * 16 + g4] = m[0];
+            m_sm[(qs & 1) * 16 + g4 + 8] = m[1];
           }
         }
-        named_bar_arrive(T::kBarPFull + pb, T::kPairThreads);
-        if (n + 1 < nch) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            sc[0][e] = sn[0][e];
-            sc[1][e] = sn[1][e];
-          }
-        }
+        named_bar_arrive(T::kBarPFull + pb, T::kPPair);
       }
       ++qs;
     }
-    // consume the last two P-empty signals so every named-barrier arrival is matched
-    for (int c = max(it - 2, 0); c < it; ++c) named_bar_sync(T::kBarPEmpty + (c & 1), T::kPairThreads);
+    for (int c = max(it - 2, 0); c < it; ++c) named_bar_sync(T::kBarPEmpty + (c & 1), T::kPPair);
   } else {
     // ------------------------- PV warps -------------------------
-    const int v = warp - T::kQKWarps;  // value columns 128 v .. 128 v + 127
+    const int v = warp - T::kPVWarp0;  // value columns 128 v .. 128 v + 127
     int it = 0, qs = 0;
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
-      const int L = p.seqlens[seq];
-      const int t0 = seq == pc.bi ? pc.bt : 0;
-      const int t1 = seq == pc.ei ? pc.et : L;
-      const int nch = t1 > t0 ? (t1 - t0 + T::KC - 1) / T::KC : 0;
+      int L, t0, t1;
+      const int nch = chunk_range(p, pc, seq, L, t0, t1);
       const int ns0 = p.num_splits[seq];
       const int nsplit = p.num_splits[seq + 1] - ns0;
       const int ord = seq == pc.bi ? pc.bord : 0;
       const int64_t acc_row0 = ((int64_t)(ns0 + ord) * p.h_kv + kvh) * p.R;
       if (nch == 0) {
-        const int tid = threadIdx.x - T::kQKWarps * 32;
+        const int tid = threadIdx.x - T::kPVWarp0 * 32;
         for (int idx = tid; idx < p.R * kDV; idx += T::kPVWarps * 32) {
           const int c = idx / kDV, dv = idx % kDV;
           if (nsplit == 1)
@@ -680,10 +672,19 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
       float o[16][4];
 #pragma unroll
       for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+      float lt[2] = {0.f, 0.f}, mr[2] = {-INFINITY, -INFINITY};
       for (int n = 0; n < nch; ++n, ++it) {
         const int s = it % T::NS, pb = it & 1;
-        named_bar_sync(T::kBarPFull + pb, T::kPairThreads);
+        named_bar_sync(T::kBarPFull + pb, T::kPPair);
         const float a0 = alpha_sm[pb * 16 + g4], a1 = alpha_sm[pb * 16 + g4 + 8];
+        if (n == nch - 1) {
+          // this sequence's row sums and maxima, read before the P tile is released
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            lt[r] = l_sm[(qs & 1) * 16 + g4 + 8 * r];
+            mr[r] = m_sm[(qs & 1) * 16 + g4 + 8 * r];
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           o[j][0] *= a0;
@@ -714,7 +715,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
             }
           }
         }
-        named_bar_arrive(T::kBarPEmpty + pb, T::kPairThreads);
+        named_bar_arrive(T::kBarPEmpty + pb, T::kPPair);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(T::EMPTY + s));
       }
@@ -723,11 +724,9 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
       for (int r = 0; r < 2; ++r) {
         const int row = g4 + 8 * r;
         if (row >= p.R || !ok) continue;
-        const float lt = l_sm[((qs & 1) * 2) * 16 + row] + l_sm[((qs & 1) * 2 + 1) * 16 + row];
-        const float mr = m_sm[(qs & 1) * 16 + row];
-        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const float inv = lt[r] > 0.f ? 1.f / lt[r] : 0.f;
         const int sq = row / p.g, h = kvh * p.g + row % p.g;
-        const float lse_v = lt > 0.f ? (mr + fast_log2(lt)) * 0.69314718055994531f : -INFINITY;
+        const float lse_v = lt[r] > 0.f ? (mr[r] + fast_log2(lt[r])) * 0.69314718055994531f : -INFINITY;
         if (nsplit == 1) {
           __nv_bfloat16 *orow = p.out + (((int64_t)seq * p.s_q + sq) * p.h_q + h) * kDV + v * 128 + c4 * 2;
 #pragma unroll
