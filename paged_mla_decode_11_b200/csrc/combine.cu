@@ -15,6 +15,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
     combine_kernel(const int32_t *__restrict__ num_splits, int s_q, int h_q, int h_kv, int R,
                    const float *__restrict__ lse_accum, const float *__restrict__ o_accum,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+  grid_dependency_wait();  // partials come from the decode kernel just before
   const int b = blockIdx.x, kvh = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int row = blockIdx.y * kCombineWarps + warp;
@@ -25,6 +26,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
   const int64_t stride = int64_t(h_kv) * R;  // between consecutive splits
   const int64_t base = (int64_t(ns0) * h_kv + kvh) * R + row;
 
+  // merged LSE: max over splits, then ln sum exp
   float mx = -INFINITY;
   for (int k = lane; k < n; k += 32) mx = fmaxf(mx, lse_accum[base + k * stride]);
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -38,16 +40,23 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (tot != -INFINITY) {
-    for (int k = 0; k < n; ++k) {
-      const float w = expf(lse_accum[base + k * stride] - tot);
-      const float4 *src = reinterpret_cast<const float4 *>(o_accum + (base + k * stride) * kDV);
+    for (int k0 = 0; k0 < n; k0 += 32) {
+      // lane j holds the weight of split k0 + j; the partial rows are then read with
+      // four independent 16-byte loads per lane and split
+      const float wl = k0 + lane < n ? expf(lse_accum[base + (k0 + lane) * stride] - tot) : 0.f;
+      const int kn = min(32, n - k0);
+#pragma unroll 4
+      for (int j = 0; j < kn; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wl, j);
+        const float4 *src = reinterpret_cast<const float4 *>(o_accum + (base + (k0 + j) * stride) * kDV);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = src[lane + 32 * i];
-        acc[i].x += w * v.x;
-        acc[i].y += w * v.y;
-        acc[i].z += w * v.z;
-        acc[i].w += w * v.w;
+        for (int i = 0; i < 4; ++i) {
+          const float4 v = src[lane + 32 * i];
+          acc[i].x += w * v.x;
+          acc[i].y += w * v.y;
+          acc[i].z += w * v.z;
+          acc[i].w += w * v.w;
+        }
       }
     }
   }
@@ -68,9 +77,8 @@ cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_
                            float *lse, cudaStream_t stream) {
   const int R = s_q * (h_q / h_kv);
   dim3 grid(batch, (R + kCombineWarps - 1) / kCombineWarps, h_kv);
-  combine_kernel<<<grid, kCombineWarps * 32, 0, stream>>>(num_splits, s_q, h_q, h_kv, R, lse_accum,
-                                                          o_accum, out, lse);
-  return cudaGetLastError();
+  return launch_early(combine_kernel, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv, R,
+                      lse_accum, o_accum, out, lse);
 }
 
 // A CTA that waits on a barrier nothing completes, with the decode kernels' bounded

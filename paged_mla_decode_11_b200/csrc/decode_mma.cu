@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  grid_dependency_wait();  // the plan comes from the scheduler kernel just before
   const PartCursor pc = load_part(p.tile_md, part);
 
   if (warp == T::NCW) {
@@ -341,6 +342,7 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
       }
     }
   }
+  grid_launch_dependents();
   __syncthreads();
 }
 
@@ -426,6 +428,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  grid_dependency_wait();  // the plan comes from the scheduler kernel just before
   const PartCursor pc = load_part(p.tile_md, part);
   const int g4 = lane >> 2, c4 = lane & 3;
 
@@ -744,6 +747,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
       ++qs;
     }
   }
+  grid_launch_dependents();
   __syncthreads();
 }
 
@@ -753,8 +757,7 @@ cudaError_t launch_decode_mma16(const CUtensorMap &kv_map, const CUtensorMap &q_
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(decode_mma16_kernel), T::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_parts, 1, p.h_kv);
-  decode_mma16_kernel<<<grid, T::kThreads, T::kSmemBytes, stream>>>(kv_map, q_map, p);
-  return cudaGetLastError();
+  return launch_early(decode_mma16_kernel, grid, dim3(T::kThreads), T::kSmemBytes, stream, kv_map, q_map, p);
 }
 
 template <int BM, int DVS>
@@ -765,8 +768,7 @@ static cudaError_t launch_mma(const CUtensorMap &map, const DecodeParams &p, int
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), T::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_parts, m_blocks, p.h_kv);
-  kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(map, p);
-  return cudaGetLastError();
+  return launch_early(kern, grid, dim3(T::kThreads), T::kSmemBytes, stream, map, p);
 }
 
 cudaError_t launch_decode_mma(const CUtensorMap &map, const DecodeParams &p, cudaStream_t stream) {

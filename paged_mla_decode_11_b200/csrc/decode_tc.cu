@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + T::kOffTmem);
+  grid_dependency_wait();  // the plan comes from the scheduler kernel just before
   const PartCursor pc = load_part(p.tile_md, part);
   const unsigned long long lim_ns = p.watchdog_ns;
 
@@ -471,6 +472,7 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
       ++qs;
     }
   }
+  grid_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -485,8 +487,7 @@ static cudaError_t launch_tc(const CUtensorMap &kv_map, const CUtensorMap &q_map
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), T::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_parts, 1, p.h_kv);
-  kern<<<grid, T::kThreads, T::kSmemBytes, stream>>>(kv_map, q_map, p);
-  return cudaGetLastError();
+  return launch_early(kern, grid, dim3(T::kThreads), T::kSmemBytes, stream, kv_map, q_map, p);
 }
 
 cudaError_t launch_decode_tc_narrow(const CUtensorMap &kv_map, const CUtensorMap &q_map,

@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(kMetaThreads)
                     int32_t *__restrict__ tile_md, int32_t *__restrict__ num_splits) {
   extern __shared__ long long start[];  // [batch + 1]
   __shared__ long long scratch[32];
+  grid_launch_dependents();  // the decode kernel may start its prologue now
   const int per = (batch + kMetaThreads - 1) / kMetaThreads;
   const int lo = threadIdx.x * per, hi = min(batch, lo + per);
 
