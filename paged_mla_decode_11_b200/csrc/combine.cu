@@ -1,82 +1,112 @@
 // Log-sum-exp combine of split-KV partials (the method's merge of the partial results
 // of one sequence's splits): lse = ln sum_k exp(lse_k), out = sum_k exp(lse_k - lse) o_k.
 //
-// One warp per (sequence, latent head, query row); sequences with a single split are
-// skipped (the decode kernel wrote them directly).  Each lane owns 16 of the 512 value
-// columns as four float4s strided 128 apart, so every warp-wide access covers 512
-// contiguous bytes.
+// One warp per (sequence, latent head, query row, half of the value columns); sequences
+// with a single split are skipped (the decode kernel wrote them directly).  In its 256
+// columns each lane owns 8 as two float4s strided 128 apart, so every warp-wide access
+// covers 512 contiguous bytes.  CTAs are small (4 warps, few registers) so that they fit
+// beside a running decode CTA and are resident before the decode kernel ends.
+//
+// The kernel is launched early (programmatic dependent launch) and runs after the decode
+// kernel's last CTA, so its latency is the tail of every decode call.  It therefore reads
+// the plan before waiting for the decode kernel (the scheduler kernel wrote num_splits and
+// had completed before any decode CTA passed its own dependency wait), and after the wait
+// issues the split LSEs and the partial rows of the first kBatch splits in one round trip.
 #include "launch.h"
 
 namespace pagedmla {
 
-constexpr int kCombineWarps = 8;
+constexpr int kCombineWarps = 4;           // two rows x two column halves
+constexpr int kBatch = 4;                  // splits whose partial rows are loaded together
 
-__global__ void __launch_bounds__(kCombineWarps * 32)
+// 6 CTAs per SM bound the registers to 80 per thread: one CTA then fits beside a decode
+// CTA's 320 threads x 168 registers.
+__global__ void __launch_bounds__(kCombineWarps * 32, 6)
     combine_kernel(const int32_t *__restrict__ num_splits, int s_q, int h_q, int h_kv, int R,
                    const float *__restrict__ lse_accum, const float *__restrict__ o_accum,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-  grid_dependency_wait();  // partials come from the decode kernel just before
   const int b = blockIdx.x, kvh = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int row = blockIdx.y * kCombineWarps + warp;
+  const int row = blockIdx.y * (kCombineWarps / 2) + warp / 2, half = warp % 2;
   const int ns0 = num_splits[b];
   const int n = num_splits[b + 1] - ns0;
   if (n <= 1 || row >= R) return;
   const int g = h_q / h_kv;
   const int64_t stride = int64_t(h_kv) * R;  // between consecutive splits
   const int64_t base = (int64_t(ns0) * h_kv + kvh) * R + row;
+  auto part_row = [&](int k) {
+    return reinterpret_cast<const float4 *>(o_accum + (base + k * stride) * kDV + half * (kDV / 2));
+  };
+  grid_dependency_wait();  // partials come from the decode kernel just before
+
+  // one round trip: split `lane`'s LSE and the first kBatch splits' partial rows
+  const float lk = lane < n ? lse_accum[base + lane * stride] : -INFINITY;
+  float4 v[kBatch][2];
+#pragma unroll
+  for (int j = 0; j < kBatch; ++j)
+    if (j < n)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) v[j][i] = part_row(j)[lane + 32 * i];
 
   // merged LSE: max over splits, then ln sum exp
-  float mx = -INFINITY;
-  for (int k = lane; k < n; k += 32) mx = fmaxf(mx, lse_accum[base + k * stride]);
+  float mx = lk;
+  for (int k = lane + 32; k < n; k += 32) mx = fmaxf(mx, lse_accum[base + k * stride]);
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float sum = 0.f;
-  if (mx != -INFINITY)
-    for (int k = lane; k < n; k += 32) sum += expf(lse_accum[base + k * stride] - mx);
+  if (mx != -INFINITY) {
+    sum = expf(lk - mx);
+    for (int k = lane + 32; k < n; k += 32) sum += expf(lse_accum[base + k * stride] - mx);
+  }
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float tot = mx == -INFINITY ? -INFINITY : mx + logf(sum);
 
-  float4 acc[4];
+  float4 acc[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (tot != -INFINITY) {
-    for (int k0 = 0; k0 < n; k0 += 32) {
-      // lane j holds the weight of split k0 + j; the partial rows are then read with
-      // four independent 16-byte loads per lane and split
-      const float wl = k0 + lane < n ? expf(lse_accum[base + (k0 + lane) * stride] - tot) : 0.f;
-      const int kn = min(32, n - k0);
-#pragma unroll 4
-      for (int j = 0; j < kn; ++j) {
-        const float w = __shfl_sync(0xffffffffu, wl, j);
-        const float4 *src = reinterpret_cast<const float4 *>(o_accum + (base + (k0 + j) * stride) * kDV);
+  for (int i = 0; i < 2; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k0 = 0; k0 < n; k0 += 32) {
+    // lane j holds the weight of split k0 + j
+    const float l = k0 == 0 ? lk : (k0 + lane < n ? lse_accum[base + (k0 + lane) * stride] : -INFINITY);
+    const float wl = tot != -INFINITY && k0 + lane < n ? expf(l - tot) : 0.f;
+    const int kn = min(32, n - k0);
+    for (int j0 = 0; j0 < kn; j0 += kBatch) {
+      if (k0 + j0 > 0) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 v = src[lane + 32 * i];
-          acc[i].x += w * v.x;
-          acc[i].y += w * v.y;
-          acc[i].z += w * v.z;
-          acc[i].w += w * v.w;
+        for (int j = 0; j < kBatch; ++j)
+          if (j0 + j < kn)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) v[j][i] = part_row(k0 + j0 + j)[lane + 32 * i];
+      }
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (j0 + j >= kn) break;
+        const float w = __shfl_sync(0xffffffffu, wl, j0 + j);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          acc[i].x += w * v[j][i].x;
+          acc[i].y += w * v[j][i].y;
+          acc[i].z += w * v[j][i].z;
+          acc[i].w += w * v[j][i].w;
         }
       }
     }
   }
   const int s = row / g, h = kvh * g + row % g;
-  __nv_bfloat16 *dst = out + ((int64_t(b) * s_q + s) * h_q + h) * kDV;
+  __nv_bfloat16 *dst = out + ((int64_t(b) * s_q + s) * h_q + h) * kDV + half * (kDV / 2);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint2 v;
-    v.x = pack_bf16x2(acc[i].x, acc[i].y);
-    v.y = pack_bf16x2(acc[i].z, acc[i].w);
-    *reinterpret_cast<uint2 *>(dst + 4 * (lane + 32 * i)) = v;
+  for (int i = 0; i < 2; ++i) {
+    uint2 u;
+    u.x = pack_bf16x2(acc[i].x, acc[i].y);
+    u.y = pack_bf16x2(acc[i].z, acc[i].w);
+    *reinterpret_cast<uint2 *>(dst + 4 * (lane + 32 * i)) = u;
   }
-  if (lane == 0) lse[(int64_t(b) * h_q + h) * s_q + s] = tot;
+  if (lane == 0 && half == 0) lse[(int64_t(b) * h_q + h) * s_q + s] = tot;
 }
 
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,
                            const float *lse_accum, const float *o_accum, __nv_bfloat16 *out,
                            float *lse, cudaStream_t stream) {
   const int R = s_q * (h_q / h_kv);
-  dim3 grid(batch, (R + kCombineWarps - 1) / kCombineWarps, h_kv);
+  dim3 grid(batch, (R + kCombineWarps / 2 - 1) / (kCombineWarps / 2), h_kv);
   return launch_early(combine_kernel, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv, R,
                       lse_accum, o_accum, out, lse);
 }
