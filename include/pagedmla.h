@@ -66,8 +66,9 @@ extern "C" {
 
 #define MLA_FLAG_SKIP_COMBINE 1u  /* mla_decode_paged: leave split partials unmerged */
 #define MLA_FLAG_WARP_MMA 2u      /* mla_decode_paged: force the warp-MMA (mma.sync) kernels */
-#define MLA_FLAG_TCGEN05 4u       /* mla_decode_paged: force the tcgen05 kernel (rows per
-                                     latent head <= 64 only) */
+#define MLA_FLAG_TCGEN05 4u       /* mla_decode_paged: force the tcgen05 kernels (above 16
+                                     rows per latent head h_q / h_kv must be a multiple or a
+                                     divisor of 64) */
 
 typedef struct CUstream_st *mla_stream_t; /* identical to cudaStream_t */
 
@@ -152,7 +153,8 @@ MLA_API int mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int num_pa
  *                  the workspace for a later mla_combine) and at most one kernel choice:
  *                  MLA_FLAG_WARP_MMA or MLA_FLAG_TCGEN05.  By default the kernel follows
  *                  the measured costs on B200: up to 16 rows per latent head the 16-row
- *                  warp-MMA kernel, above that the 64-row-tile warp-MMA kernel.
+ *                  warp-MMA kernel; above that the 64-row tcgen05 kernel when h_q / h_kv
+ *                  is a multiple or a divisor of 64, else the 64-row warp-MMA kernel.
  * Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.  A device
  * wait that times out (never in correct use) sets the workspace status word; read it
  * with mla_query_status.

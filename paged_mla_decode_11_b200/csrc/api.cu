@@ -101,9 +101,9 @@ int encode_kv_map(CUtensorMap *map, const void *k_cache, int64_t num_pages, int 
 }
 
 // Query [batch][s_q][h_q][576] bf16 with element strides (sb, ss, sh) as a 4-D map
-// (columns, head, s_q, batch); one box = 64 columns (128-byte swizzle) x the g heads of one
-// latent head x all s_q positions, i.e. the R query rows of one tile in row order s*g + h.
-int encode_q_map(CUtensorMap *map, const void *q, int batch, int s_q, int h_q, int g,
+// (columns, head, s_q, batch); one box = 64 columns (128-byte swizzle) x box_heads heads x
+// box_s positions, i.e. box_heads * box_s query rows of a tile in row order s*g + h.
+int encode_q_map(CUtensorMap *map, const void *q, int batch, int s_q, int h_q, int box_heads, int box_s,
                  const int64_t strides[3]) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
@@ -111,7 +111,7 @@ int encode_q_map(CUtensorMap *map, const void *q, int batch, int s_q, int h_q, i
   cuuint64_t gstr[3] = {cuuint64_t(strides[2]) * 2, cuuint64_t(strides[1]) * 2, cuuint64_t(strides[0]) * 2};
   for (int i = 0; i < 3; ++i)
     if (gstr[i] == 0) gstr[i] = 16;  // a dimension of extent 1 may carry stride 0
-  cuuint32_t box[4] = {64, cuuint32_t(g), cuuint32_t(s_q), 1};
+  cuuint32_t box[4] = {64, cuuint32_t(box_heads), cuuint32_t(box_s), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), dims, gstr, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -237,15 +237,22 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   if (workspace_bytes < wl.total)
     return fail(MLA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, wl.total);
 
-  // Kernel choice.  Measured on B200: a tcgen05 MMA costs at least a 128x128x16 tile, so for
-  // few query rows the 16-row warp-MMA tiles do the same work in fewer tensor cycles.
-  enum { kMma16, kMma64, kTc } kind = R <= 16 ? kMma16 : kMma64;
-  if (flags & MLA_FLAG_TCGEN05) {
-    if (R > 64) return fail(MLA_ERR_UNSUPPORTED, "the tcgen05 kernel handles up to 64 rows per latent head");
-    kind = kTc;
+  // Kernel choice.  Measured on B200: a tcgen05 MMA costs at least a 128x128x16 tile (an
+  // M = 64 one as much as M = 128), so up to 16 query rows the 16-row warp-MMA tiles do the
+  // same work in fewer tensor cycles; above that the 64-row tcgen05 kernel, or the 64-row
+  // warp-MMA kernel for query tiles one TMA box cannot cover.
+  enum { kMma16, kMma64, kTc, kWide } kind;
+  if (flags & MLA_FLAG_WARP_MMA) {
+    kind = R <= 16 ? kMma16 : kMma64;
+  } else if (flags & MLA_FLAG_TCGEN05) {
+    if (R > 16 && !wide_supported(R, g))
+      return fail(MLA_ERR_UNSUPPORTED, "the tcgen05 kernels take g = h_q / h_kv a multiple or a divisor of 64");
+    kind = R <= 16 ? kTc : kWide;
+  } else {
+    kind = R <= 16 ? kMma16 : (wide_supported(R, g) ? kWide : kMma64);
   }
   CUtensorMap map;
-  rc = encode_kv_map(&map, k_cache, num_pages, h_kv, kind == kMma64 ? kPage : 32);
+  rc = encode_kv_map(&map, k_cache, num_pages, h_kv, kind == kMma64 || kind == kWide ? kPage : 32);
   if (rc) return rc;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -281,9 +288,15 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   cudaError_t e;
   if (kind == kMma64) {
     e = launch_decode_mma(map, p, st);
+  } else if (kind == kWide) {
+    // a 64-row tile: 64 heads of one position, or 64 / g positions of all g heads
+    CUtensorMap qmap;
+    rc = encode_q_map(&qmap, q, batch, s_q, h_q, g >= 64 ? 64 : g, g >= 64 ? 1 : 64 / g, q_strides);
+    if (rc) return rc;
+    e = launch_decode_wide(map, qmap, p, st);
   } else {
     CUtensorMap qmap;
-    rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, q_strides);
+    rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, s_q, q_strides);
     if (rc) return rc;
     e = kind == kTc ? launch_decode_tc_narrow(map, qmap, p, st) : launch_decode_mma16(map, qmap, p, st);
   }

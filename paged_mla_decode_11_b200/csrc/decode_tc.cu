@@ -1,5 +1,6 @@
 // Paged MLA decode on 5th-generation tensor cores (tcgen05, TMEM accumulators) for up to
-// 64 query rows per latent head -- the memory-bound decode shapes.
+// 16 query rows per latent head (MLA_FLAG_TCGEN05; the 16-row warp-MMA kernel is the
+// default there, and decode_wide.cu takes more rows).  The template covers up to 64 rows.
 //
 // Per CTA: one split-KV part of the scheduler's plan, all R = s_q * h_q / h_kv query rows
 // of one latent head.  Warp roles:
@@ -492,14 +493,9 @@ static cudaError_t launch_tc(const CUtensorMap &kv_map, const CUtensorMap &q_map
 
 cudaError_t launch_decode_tc_narrow(const CUtensorMap &kv_map, const CUtensorMap &q_map,
                                     const DecodeParams &p, cudaStream_t stream) {
-  const int rp = (p.R + 15) / 16 * 16;
-  switch (rp) {
-    case 16: return launch_tc<16>(kv_map, q_map, p, stream);
-    case 32: return launch_tc<32>(kv_map, q_map, p, stream);
-    case 48: return launch_tc<48>(kv_map, q_map, p, stream);
-    case 64: return launch_tc<64>(kv_map, q_map, p, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  // above 16 rows per latent head the 64-row tcgen05 kernel takes over
+  if (p.R > 16) return cudaErrorInvalidValue;
+  return launch_tc<16>(kv_map, q_map, p, stream);
 }
 
 }  // namespace pagedmla

@@ -89,19 +89,49 @@ SMALL_CASES = [
 ]
 
 
+def tcgen05_takes(s_q, h_q, h_kv):
+    """The tcgen05 kernels: up to 16 rows per latent head, or g = h_q / h_kv a multiple or a
+    divisor of 64 (one TMA box per 64-row query tile)."""
+    g = h_q // h_kv
+    return s_q * g <= 16 or g % 64 == 0 or 64 % g == 0
+
+
 @pytest.mark.parametrize("kernel", ["auto", "warp_mma", "tcgen05"])
 @pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: f"b{c[0]}sq{c[1]}h{c[2]}kv{c[3]}")
 def test_parity_small(case, kernel):
     b, s_q, h_q, h_kv, lens, causal = case
-    if kernel == "tcgen05" and s_q * h_q // h_kv > 64:
-        pytest.skip("the tcgen05 kernel covers up to 64 rows per latent head")
+    if kernel == "tcgen05" and not tcgen05_takes(s_q, h_q, h_kv):
+        pytest.skip("query tile not one TMA box")
     x = W.make_inputs(W.custom(b, s_q, h_q, h_kv, lens, causal=causal), seed=sum(lens) % 97)
     full_parity(x, kernel=kernel)
+
+
+WIDE_CASES = [
+    # (batch, s_q, h_q, seqlens, causal): the 64-row tcgen05 kernel
+    (3, 1, 64, [1, 64, 700], True),           # one 64-row block, ragged pages
+    (2, 1, 128, [5000, 33], True),            # two row blocks, a long split sequence
+    (2, 2, 128, [700, 2], True),              # causal multi-token: blocks see different key ends
+    (3, 3, 32, [129, 1000, 64], True),        # g = 32: a block holds 2 positions x 32 heads
+    (2, 4, 16, [300, 65], True),              # g = 16: a block holds 4 positions x 16 heads
+    (2, 1, 256, [640, 100], False),           # g = 256: four blocks of 64 heads
+    (3, 1, 64, [0, 4000, 0], True),           # empty sequences around a long one
+    (1, 2, 64, [1], True),                    # a causal row with no visible key
+]
+
+
+@pytest.mark.parametrize("case", WIDE_CASES, ids=lambda c: f"b{c[0]}sq{c[1]}h{c[2]}")
+@pytest.mark.parametrize("num_parts", [None, 3])
+def test_parity_tcgen05_64_row_tiles(case, num_parts):
+    b, s_q, h_q, lens, causal = case
+    x = W.make_inputs(W.custom(b, s_q, h_q, 1, lens, causal=causal), seed=len(lens) * 13 + h_q)
+    full_parity(x, kernel="tcgen05", num_parts=num_parts)
 
 
 @pytest.mark.parametrize("kernel", ["auto", "tcgen05"])
 @pytest.mark.parametrize("h_q,s_q", [(16, 1), (8, 2), (4, 1), (24, 1), (32, 1), (12, 3), (48, 1), (64, 1), (16, 4)])
 def test_parity_row_paddings(h_q, s_q, kernel):
+    if kernel == "tcgen05" and not tcgen05_takes(s_q, h_q, 1):
+        pytest.skip("query tile not one TMA box")
     # every padded tile height of the kernels (16, 32, 48, 64 rows), ragged row counts
     x = W.make_inputs(W.custom(3, s_q, h_q, 1, [1, 200, 1000], causal=True), seed=h_q * 7 + s_q)
     full_parity(x, kernel=kernel)
