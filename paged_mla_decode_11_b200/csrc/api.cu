@@ -239,14 +239,11 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
 
   // Kernel choice.  Measured on B200: a tcgen05 MMA costs at least a 128x128x16 tile (an
   // M = 64 one as much as M = 128), so up to 16 query rows the 16-row warp-MMA tiles do the
-  // same work in fewer tensor cycles; above that the 64-row tcgen05 kernel, or the 64-row
-  // warp-MMA kernel for query tiles one TMA box cannot cover.
+  // same work in fewer tensor cycles; above that the 64-row tcgen05 kernel.
   enum { kMma16, kMma64, kTc, kWide } kind;
   if (flags & MLA_FLAG_WARP_MMA) {
     kind = R <= 16 ? kMma16 : kMma64;
   } else if (flags & MLA_FLAG_TCGEN05) {
-    if (R > 16 && !wide_supported(R, g))
-      return fail(MLA_ERR_UNSUPPORTED, "the tcgen05 kernels take g = h_q / h_kv a multiple or a divisor of 64");
     kind = R <= 16 ? kTc : kWide;
   } else {
     kind = R <= 16 ? kMma16 : (wide_supported(R, g) ? kWide : kMma64);
@@ -289,11 +286,7 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   if (kind == kMma64) {
     e = launch_decode_mma(map, p, st);
   } else if (kind == kWide) {
-    // a 64-row tile: 64 heads of one position, or 64 / g positions of all g heads
-    CUtensorMap qmap;
-    rc = encode_q_map(&qmap, q, batch, s_q, h_q, g >= 64 ? 64 : g, g >= 64 ? 1 : 64 / g, q_strides);
-    if (rc) return rc;
-    e = launch_decode_wide(map, qmap, p, st);
+    e = launch_decode_wide(map, p, st);  // reads the query rows itself (any g)
   } else {
     CUtensorMap qmap;
     rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, s_q, q_strides);

@@ -2,27 +2,35 @@
 // than 16 query rows per latent head: the mixed and compute-bound decode shapes.
 //
 // One CTA per (split-KV part, block of 64 query rows, latent head).  The 64-row tile is
-// what fits: the fp32 output accumulator of 64 rows x 512 value columns takes half of
-// TMEM when it is held as two M = 64 accumulators interleaved in the lane halves of each
-// 32-lane sub-partition (value columns 0-255 in lanes 0-15, 256-511 in lanes 16-31, both
-// in TMEM columns 0-255), which leaves room for the score tiles; 128 rows would need all of
-// TMEM for the output alone.  Per 64-token page (one tile, "OpenSourceWeek Day 1 - FlashMLA",
-// section II.1: fixed 64-token blocks):
-//     S = Q K^T          M = 64 rows, N = 64 keys, K = 576 (absorbed-query score over the
-//                        whole latent row, dpshk.com notes 2.1); S double-buffered in TMEM
+// what fits: 64 rows x 512 value columns of fp32 output take one lane half of TMEM.  An
+// M = 64 accumulator occupies lanes 0-15 of each 32-lane sub-partition (row 16q + i on lane
+// 32q + i) or, placed at lane 16, lanes 16-31; 128 rows of output would need all of TMEM.
+// TMEM map (512 columns):
+//     lanes 0-15 of each sub-partition    S double buffer (columns 0-127) and the 64-row
+//                                         query tile as the MMA's A operand (columns
+//                                         224-511: 576 bf16 = 288 packed columns)
+//     lanes 16-31                         O: value columns 0-255 in TMEM columns 0-255,
+//                                         256-511 in columns 256-511
+// With Q in TMEM, shared memory holds a three-page ring and the P tile.  Per 64-token page
+// (one tile, "OpenSourceWeek Day 1 - FlashMLA", section II.1: fixed 64-token blocks):
+//     S = Q K^T          M = 64 rows, N = 64 keys, K = 576, A from TMEM (absorbed-query
+//                        score over the whole latent row, dpshk.com notes 2.1)
 //     online softmax     running maximum refreshed only when it grows by more than 8 in
 //                        log2 units (same notes 2.2); P -> bf16 tile in shared memory
 //     O += P V           M = 64, N = 256 (two halves of the 512 value columns), K = 64
 //                        keys, V = the page's first 512 columns read in place as an
 //                        MN-major operand
 // Warp roles:
-//   warp 0      TMA producer: the 64-row query tile (once per sequence piece) and the pages
-//               gathered through block_table into a two-page ring
-//   warp 1      TMEM owner and MMA issuer (one thread); QK of page n+1 is issued before PV
-//               of page n, so the softmax of one page overlaps tensor-core work on the next
-//   warps 2-5   softmax, O rescale and epilogue: lanes 0-15 of the warp on sub-partition q
-//               own rows 16q..16q+15 of the score tile; for the output both lane halves work,
-//               each on one half of the value columns of the same row
+//   warp 0      TMA producer: pages gathered through block_table into the ring, pages three
+//               ahead prefetched into L2
+//   warp 1      TMEM owner and MMA issuer (one thread): QK runs up to two pages ahead of PV
+//               and each step issues whichever group is ready, so the softmax of one page
+//               overlaps tensor-core work on the next
+//   warps 2-5   softmax, O rescale and epilogue.  The warp on sub-partition q owns rows
+//               16q..16q+15; lane i and lane i + 16 share row 16q + i: keys 0-31 / 32-63 of
+//               the score tile, value columns 0-255 / 256-511 of the output
+//   warps 6-9   query loaders: the next sequence piece's query rows are read into registers
+//               while the current piece runs and written to TMEM once its last QK is done
 // Every mbarrier wait is bounded (pagedmla watchdog); a warp whose wait gives up keeps
 // walking the same barrier sequence without work.
 #include "common.cuh"
@@ -31,14 +39,12 @@
 namespace pagedmla {
 
 struct Wide64 {
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
   static constexpr int BM = 64;                             // query rows per CTA
-  static constexpr int NS = 2;                              // page ring depth
-  static constexpr int kQBlock = BM * 128;                  // 64 rows x 64 columns: 8 KB
-  static constexpr int kQBytes = kColBlocks * kQBlock;      // 73,728 B
+  static constexpr int NS = 3;                              // page ring depth
+  static constexpr int kAhead = 3;                          // pages prefetched into L2 ahead
   static constexpr int kPBytes = BM * 128;                  // 64 rows x 64 keys bf16
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffRing = kOffQ + kQBytes;          // 1 KB aligned
+  static constexpr int kOffRing = 0;
   static constexpr int kOffP = kOffRing + NS * kPageBytes;
   enum {
     FULL = 0, EMPTY = FULL + NS, QFULL = EMPTY + NS, QFREE = QFULL + 1, SFULL = QFREE + 1,
@@ -50,15 +56,16 @@ struct Wide64 {
   static constexpr int kOffAbort = kOffTmem + 8;
   static constexpr int kSmemBytes = kOffAbort + 8 + 1024;   // + slack for 1 KB alignment
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTmemS = 256;                   // S buffers: columns 256 and 320
-  static constexpr uint32_t kHalf1 = 16u << 16;             // lane offset of the second atom
-  static_assert(kOffRing % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static constexpr uint32_t kTmemS = 0;                     // S buffers: columns 0 and 64
+  static constexpr uint32_t kTmemQ = kTmemCols - kD / 2;    // query tile: columns 224-511
+  static constexpr uint32_t kHalf1 = 16u << 16;             // lane offset of the O accumulators
+  static_assert(kOffP % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kTmemS + 128 <= kTmemQ, "tensor memory map");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-// Shapes the 64-row tensor-core kernel takes: more than 16 rows per latent head, and a
-// query tile of 64 rows that one 4-D TMA box covers (g a multiple or a divisor of 64).
-bool wide_supported(int R, int g) { return R > 16 && (g % 64 == 0 || 64 % g == 0); }
+// Shapes the 64-row tensor-core kernel takes: more than 16 rows per latent head.
+bool wide_supported(int R, int g) { return R > 16 && g > 0; }
 
 struct WidePiece {
   int seq, L, t0, t1, ntiles;  // ntiles = 64-token pages in [t0, t1); t0 is page aligned
@@ -82,9 +89,67 @@ __device__ __forceinline__ WidePiece wide_piece(const DecodeParams &p, const Par
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
+// 16-lane TMEM accesses (.16x32bx2): lane i < 16 of the warp reaches TMEM lane base + i at
+// column c + j, lane i + 16 the same TMEM lane at column c + OFF + j.  Both lane halves of a
+// warp work on one 16-row half of its sub-partition, which is how an M = 64 accumulator
+// (16 rows per sub-partition) is read without touching the other 16 lanes.
+template <int OFF>
+__device__ __forceinline__ void tmem_ld_half32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32], %33;\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr), "n"(OFF)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int OFF>
+__device__ __forceinline__ void tmem_st_half32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
+      "{%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, "
+      "%18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33};" ::"r"(taddr),
+      "n"(OFF), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+template <int OFF>
+__device__ __forceinline__ void tmem_st_half16(uint32_t taddr, const uint4 (&v)[4]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, "
+      "{%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17};" ::"r"(taddr),
+      "n"(OFF), "r"(v[0].x), "r"(v[0].y), "r"(v[0].z), "r"(v[0].w), "r"(v[1].x), "r"(v[1].y), "r"(v[1].z),
+      "r"(v[1].w), "r"(v[2].x), "r"(v[2].y), "r"(v[2].z), "r"(v[2].w), "r"(v[3].x), "r"(v[3].y), "r"(v[3].z),
+      "r"(v[3].w)
+      : "memory");
+}
+
+// L2 prefetch of one latent page (64 tokens of a single latent head: contiguous).
+__device__ __forceinline__ void prefetch_page(const DecodeParams &p, int phys) {
+  if (p.h_kv == 1) prefetch_l2_bulk(p.kv_base + (int64_t)phys * kPage * p.kv_token_bytes, uint32_t(kPage * p.kv_token_bytes));
+}
+
 __global__ void __launch_bounds__(Wide64::kThreads, 1)
-    decode_wide_kernel(const __grid_constant__ CUtensorMap kv_map, const __grid_constant__ CUtensorMap q_map,
-                       const DecodeParams p) {
+    decode_wide_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeParams p) {
   using T = Wide64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -96,14 +161,14 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
   const uint32_t bar0 = sbase + T::kOffBar;
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
   volatile int *abort = reinterpret_cast<volatile int *>(smem + T::kOffAbort);
-  const uint32_t sQ = sbase + T::kOffQ, sRing = sbase + T::kOffRing, sP = sbase + T::kOffP;
+  const uint32_t sRing = sbase + T::kOffRing, sP = sbase + T::kOffP;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::NS; ++s) {
       mbar_init(bar(T::FULL + s), 1);
       mbar_init(bar(T::EMPTY + s), 1);
     }
-    mbar_init(bar(T::QFULL), 1);
+    mbar_init(bar(T::QFULL), 4);
     mbar_init(bar(T::QFREE), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(T::SFULL + i), 1);
@@ -127,14 +192,9 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
   const unsigned long long lim_ns = p.watchdog_ns;
 
   if (warp == 0) {
-    // ------------------------- producer: query tiles and pages -------------------------
-    if (lane == 0) {
-      prefetch_tensormap(&kv_map);
-      prefetch_tensormap(&q_map);
-    }
-    // the query tile of this block: rows row0.. in the order s * g + h
-    const int s0 = row0 / p.g, h0 = kvh * p.g + row0 % p.g;
-    int it = 0, qs = 0, last_q = -1;
+    // ------------------------- producer: pages -------------------------
+    if (lane == 0) prefetch_tensormap(&kv_map);
+    int it = 0;
     int last_page[T::NS];
 #pragma unroll
     for (int s = 0; s < T::NS; ++s) last_page[s] = -1;
@@ -142,26 +202,17 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
     for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
       const WidePiece w = wide_piece(p, pc, seq, row0);
       if (w.ntiles == 0) continue;
-      int good = 1;
-      if (lane == 0) {
-        if (!mbar_wait(bar(T::QFREE), (qs & 1) ^ 1, abort, p.status, lim_ns)) {
-          good = 0;
-        } else {
-          mbar_arrive_expect_tx(bar(T::QFULL), uint32_t(T::kQBytes));
-#pragma unroll
-          for (int c = 0; c < kColBlocks; ++c)
-            tma_load_4d(sQ + c * T::kQBlock, &q_map, bar(T::QFULL), c * 64, h0, s0, seq);
-          last_q = qs;
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, good, 0) != 0;
-      ++qs;
       const int32_t *bt_row = p.block_table + (int64_t)seq * p.bt_stride + w.t0 / kPage;
       for (int base = 0; ok && base < w.ntiles; base += 32) {
         const int mine = base + lane < w.ntiles ? bt_row[base + lane] : 0;
         const int cnt = min(32, w.ntiles - base);
+        // With two pages in the ring a slot refills only after the page before it is done;
+        // pages kAhead ahead are pulled into L2 first so that the refill reads L2, not HBM.
+        if (lane < min(T::kAhead, cnt)) prefetch_page(p, mine);
         for (int i = 0; ok && i < cnt; ++i, ++it) {
           const int phys = __shfl_sync(0xffffffffu, mine, i);
+          const int ahead = __shfl_sync(0xffffffffu, mine, min(i + T::kAhead, 31));
+          if (lane == 0 && i + T::kAhead < cnt) prefetch_page(p, ahead);
           const int s = it % T::NS;
           int g2 = 1;
           if (lane == 0) {
@@ -186,68 +237,107 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       for (int s = 0; s < T::NS; ++s)
         if (last_page[s] >= 0)
           mbar_wait(bar(T::FULL + s), (last_page[s] / T::NS) & 1, &never, p.status, lim_ns);
-      if (last_q >= 0) mbar_wait(bar(T::QFULL), last_q & 1, &never, p.status, lim_ns);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------- MMA issuer (one thread) -------------------------
+    // Two cursors walk the part's pages: QK runs up to two pages ahead of PV (the S buffers
+    // and the ring bound it).  Each step issues whichever MMA group is ready, PV first: it
+    // frees a ring slot and the P tile sooner.  A fixed QK(n+1)-then-PV(n) order would hold
+    // PV behind a QK that waits for a page whose load could only start after the PV before.
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(64, 64, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(64, 256, false, true);
-      int it = 0, qs = 0;
-      bool ok = true;
-      // O += P V for global page j; `first` = first page of a sequence piece (overwrites O,
-      // after the previous piece's epilogue has read it)
-      auto issue_pv = [&](int j, bool first) -> bool {
-        if (!mbar_wait(bar(T::PFULL), j & 1, abort, p.status, lim_ns)) return false;
-        if (first && qs > 0 && !mbar_wait(bar(T::OFREE), (qs - 1) & 1, abort, p.status, lim_ns)) return false;
-        tc_fence_after();
-        const uint32_t page = sRing + (j % T::NS) * kPageBytes;
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
-#pragma unroll
-          for (int ks = 0; ks < kPage / 16; ++ks) {
-            // V: value columns 256 half.. (4 column blocks, 8 KB apart), keys 16 ks.. (two
-            // 8-row groups, 1 KB apart); P: keys 16 ks.. of the 64-row tile
-            const uint64_t b = smem_desc_sw128(page + half * 4 * kPageBlockBytes + ks * 2048, kPageBlockBytes, 1024);
-            const uint64_t a = smem_desc_sw128(sP + ks * 32, 16, 1024);
-            umma_bf16(tmem + (half ? T::kHalf1 : 0u), a, b, idesc_pv, (!first || ks > 0) ? 1u : 0u);
+      // first piece at or after `seq` with pages; -1 at the end of the part
+      auto seek = [&](int seq, int &nt) -> int {
+        for (; part_has(pc, seq); ++seq) {
+          const int n = wide_piece(p, pc, seq, row0).ntiles;
+          if (n > 0) {
+            nt = n;
+            return seq;
           }
-        umma_commit(bar(T::PFREE));
-        umma_commit(bar(T::EMPTY + j % T::NS));
-        return true;
+        }
+        return -1;
       };
-      for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
-        const WidePiece w = wide_piece(p, pc, seq, row0);
-        if (w.ntiles == 0) continue;
-        if (!mbar_wait(bar(T::QFULL), qs & 1, abort, p.status, lim_ns)) {
-          ok = false;
-          break;
-        }
-        for (int n = 0; ok && n < w.ntiles; ++n) {
-          const int cur = it + n, s = cur % T::NS, sb = cur & 1;
-          if (!mbar_wait(bar(T::FULL + s), (cur / T::NS) & 1, abort, p.status, lim_ns) ||
-              (cur >= 2 && !mbar_wait(bar(T::SFREE + sb), ((cur >> 1) - 1) & 1, abort, p.status, lim_ns))) {
-            ok = false;
-            break;
+      int qk_nt = 0, qk_n = 0, qk_t = 0, qk_piece = 0;
+      int qk_seq = seek(pc.bi, qk_nt);
+      int pv_nt = qk_nt, pv_n = 0, pv_t = 0, pv_piece = 0;
+      int pv_seq = qk_seq;
+      bool have_q = false, ok = true;
+      unsigned long long idle_since = 0;
+      uint32_t spins = 0;
+      while (ok && pv_seq >= 0) {
+        bool progressed = false;
+        if (pv_t < qk_t) {
+          // O += P V for page pv_t; the first page of a piece overwrites O once the previous
+          // piece's epilogue has read it
+          const bool first = pv_n == 0;
+          if (mbar_test_wait(bar(T::PFULL), pv_t & 1) &&
+              (!first || pv_piece == 0 || mbar_test_wait(bar(T::OFREE), (pv_piece - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t page = sRing + (pv_t % T::NS) * kPageBytes;
+#pragma unroll
+            for (int half = 0; half < 2; ++half)
+#pragma unroll
+              for (int ks = 0; ks < kPage / 16; ++ks) {
+                // V: value columns 256 half.. (4 column blocks, 8 KB apart), keys 16 ks.. (two
+                // 8-row groups, 1 KB apart); P: keys 16 ks.. of the 64-row tile
+                const uint64_t b = smem_desc_sw128(page + half * 4 * kPageBlockBytes + ks * 2048, kPageBlockBytes, 1024);
+                const uint64_t a = smem_desc_sw128(sP + ks * 32, 16, 1024);
+                umma_bf16(tmem + T::kHalf1 + half * 256, a, b, idesc_pv, (!first || ks > 0) ? 1u : 0u);
+              }
+            umma_commit(bar(T::PFREE));
+            umma_commit(bar(T::EMPTY + pv_t % T::NS));
+            if (++pv_n == pv_nt) {
+              umma_commit(bar(T::OFULL));
+              pv_seq = seek(pv_seq + 1, pv_nt);
+              pv_n = 0;
+              ++pv_piece;
+            }
+            ++pv_t;
+            progressed = true;
           }
-          tc_fence_after();
-          const uint32_t page = sRing + s * kPageBytes;
+        }
+        if (!progressed && qk_seq >= 0) {
+          // S = Q K^T for page qk_t: its page has landed and its S buffer has been read
+          if (!have_q) have_q = mbar_test_wait(bar(T::QFULL), qk_piece & 1);
+          const int s = qk_t % T::NS, sb = qk_t & 1;
+          if (have_q && mbar_test_wait(bar(T::FULL + s), (qk_t / T::NS) & 1) &&
+              (qk_t < 2 || mbar_test_wait(bar(T::SFREE + sb), ((qk_t >> 1) - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t page = sRing + s * kPageBytes;
 #pragma unroll 4
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kPageBlockBytes + (kk & 3) * 32;
-            const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * T::kQBlock + (kk & 3) * 32, 16, 1024);
-            const uint64_t b = smem_desc_sw128(page + off, 16, 1024);
-            umma_bf16(tmem + T::kTmemS + sb * 64, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint64_t b = smem_desc_sw128(page + (kk >> 2) * kPageBlockBytes + (kk & 3) * 32, 16, 1024);
+              umma_bf16_ts(tmem + T::kTmemS + sb * 64, tmem + T::kTmemQ + kk * 8, b, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bar(T::SFULL + sb));
+            if (++qk_n == qk_nt) {
+              umma_commit(bar(T::QFREE));  // the query tile may be replaced by the next piece's
+              have_q = false;
+              qk_seq = seek(qk_seq + 1, qk_nt);
+              qk_n = 0;
+              ++qk_piece;
+            }
+            ++qk_t;
+            progressed = true;
           }
-          umma_commit(bar(T::SFULL + sb));
-          if (n == w.ntiles - 1) umma_commit(bar(T::QFREE));
-          if (n > 0 && !issue_pv(cur - 1, n == 1)) ok = false;
         }
-        if (ok && !issue_pv(it + w.ntiles - 1, w.ntiles == 1)) ok = false;
-        if (ok) umma_commit(bar(T::OFULL));
-        it += w.ntiles;
-        ++qs;
+        // watchdog: give up after lim_ns without progress, or when another warp has
+        if (progressed) {
+          idle_since = 0;
+        } else if ((++spins & 255u) == 0) {
+          const unsigned long long now = global_ns();
+          if (*abort) {
+            ok = false;
+          } else if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > lim_ns) {
+            *abort = 1;
+            report_timeout(p.status);
+            ok = false;
+          }
+        }
       }
       // all issued tensor-core work completes before TMEM is released
       umma_commit(bar(T::FINAL));
@@ -255,15 +345,16 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       mbar_wait(bar(T::FINAL), 0, &never, p.status, lim_ns);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     // ------------------------- softmax / O rescale / epilogue -------------------------
     const int q = warp & 3;                   // TMEM sub-partition of this warp
-    const int hf = lane >> 4;                 // 0: score row and value columns 0-255; 1: columns 256-511
+    const int hf = lane >> 4;                 // keys 32 hf.. of the score row; value columns 256 hf..
     const int rl = 16 * q + (lane & 15);      // row within the 64-row block
     const int row = row0 + rl;
     const bool active = row < p.R;
     const int s_row = row / p.g, h_row = kvh * p.g + row % p.g;
-    const uint32_t lanes = tmem + (uint32_t(32 * q) << 16);
+    const uint32_t lanes = tmem + (uint32_t(32 * q) << 16);   // S rows of this warp
+    const uint32_t olanes = lanes + T::kHalf1;                // O rows of this warp
     int it = 0, qs = 0;
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
@@ -289,34 +380,30 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       }
       // rows past R and rows without a visible key get P = 0 (every key masked)
       const int lim = active ? min(w.t1, p.causal ? w.L - (p.s_q - 1 - s_row) : w.L) : -1;
-      float m_used = -INFINITY, l = 0.f;
+      float m_used = -INFINITY, l = 0.f;  // l: this lane's half of the row sum
 
       for (int n = 0; n < w.ntiles; ++n) {
         const int cur = it + n, sb = cur & 1;
         ok = warp_all(ok && mbar_wait(bar(T::SFULL + sb), (cur >> 1) & 1, abort, p.status, lim_ns));
         tc_fence_after();
-        float sa[32], sc[32];
-        if (ok) {
-          tmem_ld32(lanes + T::kTmemS + sb * 64, sa);
-          tmem_ld32(lanes + T::kTmemS + sb * 64 + 32, sc);
-        }
+        float sv[32];
+        if (ok) tmem_ld_half32<32>(lanes + T::kTmemS + sb * 64, sv);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(T::SFREE + sb));
 
         bool need = false;
         float alpha = 1.f;
-        if (ok && hf == 0) {
-          const int key0 = w.t0 + n * kPage;
+        if (ok) {
+          const int key0 = w.t0 + n * kPage + 32 * hf;
           float mx = -INFINITY;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float va = key0 + i < lim ? sa[i] * p.scale_log2 : -INFINITY;
-            const float vc = key0 + 32 + i < lim ? sc[i] * p.scale_log2 : -INFINITY;
-            sa[i] = va;
-            sc[i] = vc;
-            mx = fmaxf(mx, fmaxf(va, vc));
+            const float v = key0 + i < lim ? sv[i] * p.scale_log2 : -INFINITY;
+            sv[i] = v;
+            mx = fmaxf(mx, v);
           }
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           const float m_new = fmaxf(m_used, mx);
           need = m_new > m_used + 8.f;
           if (need) {
@@ -327,38 +414,33 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
           float sum = 0.f;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            sa[i] = fast_exp2(sa[i] - base);
-            sc[i] = fast_exp2(sc[i] - base);
-            sum += sa[i] + sc[i];
+            sv[i] = fast_exp2(sv[i] - base);
+            sum += sv[i];
           }
           l = l * alpha + sum;
         }
-        // both lane halves hold the row's output; they share its rescale factor
-        const float alpha_o = __shfl_sync(0xffffffffu, alpha, lane & 15);
         const bool rescale = __any_sync(0xffffffffu, need && n > 0);
         // P and O may be touched once the previous page's PV has completed
         if (cur > 0) ok = warp_all(ok && mbar_wait(bar(T::PFREE), (cur - 1) & 1, abort, p.status, lim_ns));
         if (ok && rescale) {
           tc_fence_after();
 #pragma unroll 1
-          for (int c0 = 0; c0 < 256; c0 += 16) {
-            float v[16];
-            tmem_ld16(lanes + c0, v);
+          for (int c0 = 0; c0 < 256; c0 += 32) {
+            float v[32];
+            tmem_ld_half32<256>(olanes + c0, v);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] *= alpha_o;
-            tmem_st16(lanes + c0, v);
+            for (int k = 0; k < 32; ++k) v[k] *= alpha;
+            tmem_st_half32<256>(olanes + c0, v);
           }
           tmem_st_wait();
         }
-        if (ok && hf == 0) {
+        if (ok) {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float *src = c < 4 ? sa + 8 * c : sc + 8 * (c - 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sP + sw128(rl, c)),
-                         "r"(pack_bf16x2(src[0], src[1])), "r"(pack_bf16x2(src[2], src[3])),
-                         "r"(pack_bf16x2(src[4], src[5])), "r"(pack_bf16x2(src[6], src[7]))
+          for (int c = 0; c < 4; ++c)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sP + sw128(rl, 4 * hf + c)),
+                         "r"(pack_bf16x2(sv[8 * c], sv[8 * c + 1])), "r"(pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3])),
+                         "r"(pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5])), "r"(pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]))
                          : "memory");
-          }
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -367,15 +449,14 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       }
 
       // ---- epilogue: O / l -> output (or fp32 split partial), natural-log LSE ----
-      const float l_row = __shfl_sync(0xffffffffu, l, lane & 15);
-      const float m_row = __shfl_sync(0xffffffffu, m_used, lane & 15);
+      const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
       ok = warp_all(ok && mbar_wait(bar(T::OFULL), qs & 1, abort, p.status, lim_ns));
       tc_fence_after();
       if (ok) {
         const float inv = l_row > 0.f ? 1.f / l_row : 0.f;
         for (int c0 = 0; c0 < 256; c0 += 32) {
           float v[32];
-          tmem_ld32(lanes + c0, v);
+          tmem_ld_half32<256>(olanes + c0, v);
           if (!active) continue;
           if (nsplit == 1) {
             uint4 *o = reinterpret_cast<uint4 *>(p.out + (((int64_t)seq * p.s_q + s_row) * p.h_q + h_row) * kDV +
@@ -394,7 +475,7 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
           }
         }
         if (active && hf == 0) {
-          const float lse_v = l_row > 0.f ? (m_row + fast_log2(l_row)) * 0.69314718055994531f : -INFINITY;
+          const float lse_v = l_row > 0.f ? (m_used + fast_log2(l_row)) * 0.69314718055994531f : -INFINITY;
           if (nsplit == 1)
             p.lse[((int64_t)seq * p.h_q + h_row) * p.s_q + s_row] = lse_v;
           else
@@ -407,6 +488,41 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       it += w.ntiles;
       ++qs;
     }
+  } else {
+    // ------------------------- query loaders -------------------------
+    // Lane i and lane i + 16 of the warp on sub-partition q carry row 16q + i: query
+    // elements 0-287 and 288-575 (144 packed bf16 pairs each).
+    const int q = warp & 3;
+    const int hf = lane >> 4;
+    const int row = row0 + 16 * q + (lane & 15);
+    const bool active = row < p.R;
+    const uint32_t lanes = tmem + (uint32_t(32 * q) << 16);
+    uint4 qv[36];
+    int qs = 0;
+    bool ok = true;
+    for (int seq = pc.bi; part_has(pc, seq); ++seq) {
+      if (wide_piece(p, pc, seq, row0).ntiles == 0) continue;
+      // read this piece's rows while the previous piece still uses the tile in TMEM
+      const uint4 *src = reinterpret_cast<const uint4 *>(
+          p.q + (int64_t)seq * p.q_sb + (int64_t)(row / p.g) * p.q_ss + (int64_t)(kvh * p.g + row % p.g) * p.q_sh) +
+          hf * 36;
+#pragma unroll
+      for (int i = 0; i < 36; ++i) qv[i] = active ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      if (qs > 0) ok = warp_all(ok && mbar_wait(bar(T::QFREE), (qs - 1) & 1, abort, p.status, lim_ns));
+      tc_fence_after();
+      if (ok) {
+#pragma unroll
+        for (int j = 0; j < 9; ++j) {
+          const uint4 v4[4] = {qv[4 * j], qv[4 * j + 1], qv[4 * j + 2], qv[4 * j + 3]};
+          tmem_st_half16<144>(lanes + T::kTmemQ + 16 * j, v4);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(T::QFULL));
+      ++qs;
+    }
   }
   grid_launch_dependents();
   tc_fence_before();
@@ -415,13 +531,12 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, T::kTmemCols);
 }
 
-cudaError_t launch_decode_wide(const CUtensorMap &kv_map, const CUtensorMap &q_map, const DecodeParams &p,
-                               cudaStream_t stream) {
+cudaError_t launch_decode_wide(const CUtensorMap &kv_map, const DecodeParams &p, cudaStream_t stream) {
   using T = Wide64;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(decode_wide_kernel), T::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_parts, (p.R + T::BM - 1) / T::BM, p.h_kv);
-  return launch_early(decode_wide_kernel, grid, dim3(T::kThreads), T::kSmemBytes, stream, kv_map, q_map, p);
+  return launch_early(decode_wide_kernel, grid, dim3(T::kThreads), T::kSmemBytes, stream, kv_map, p);
 }
 
 }  // namespace pagedmla

@@ -21,11 +21,9 @@ cudaError_t launch_metadata(const int32_t *seqlens, int batch, int ovh, int num_
 cudaError_t launch_decode_mma(const CUtensorMap &map, const DecodeParams &p, cudaStream_t stream);
 cudaError_t launch_decode_mma16(const CUtensorMap &kv_map, const CUtensorMap &q_map, const DecodeParams &p,
                                 cudaStream_t stream);
-// The 64-row tcgen05 kernel takes R > 16 rows per latent head with g a multiple or a
-// divisor of 64 (one 4-D TMA box then covers a 64-row query tile).
+// The 64-row tcgen05 kernel takes more than 16 rows per latent head.
 bool wide_supported(int R, int g);
-cudaError_t launch_decode_wide(const CUtensorMap &kv_map, const CUtensorMap &q_map, const DecodeParams &p,
-                               cudaStream_t stream);
+cudaError_t launch_decode_wide(const CUtensorMap &kv_map, const DecodeParams &p, cudaStream_t stream);
 cudaError_t launch_decode_tc_narrow(const CUtensorMap &kv_map, const CUtensorMap &q_map,
                                     const DecodeParams &p, cudaStream_t stream);
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,

@@ -89,19 +89,10 @@ SMALL_CASES = [
 ]
 
 
-def tcgen05_takes(s_q, h_q, h_kv):
-    """The tcgen05 kernels: up to 16 rows per latent head, or g = h_q / h_kv a multiple or a
-    divisor of 64 (one TMA box per 64-row query tile)."""
-    g = h_q // h_kv
-    return s_q * g <= 16 or g % 64 == 0 or 64 % g == 0
-
-
 @pytest.mark.parametrize("kernel", ["auto", "warp_mma", "tcgen05"])
 @pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: f"b{c[0]}sq{c[1]}h{c[2]}kv{c[3]}")
 def test_parity_small(case, kernel):
     b, s_q, h_q, h_kv, lens, causal = case
-    if kernel == "tcgen05" and not tcgen05_takes(s_q, h_q, h_kv):
-        pytest.skip("query tile not one TMA box")
     x = W.make_inputs(W.custom(b, s_q, h_q, h_kv, lens, causal=causal), seed=sum(lens) % 97)
     full_parity(x, kernel=kernel)
 
@@ -116,6 +107,9 @@ WIDE_CASES = [
     (2, 1, 256, [640, 100], False),           # g = 256: four blocks of 64 heads
     (3, 1, 64, [0, 4000, 0], True),           # empty sequences around a long one
     (1, 2, 64, [1], True),                    # a causal row with no visible key
+    (2, 1, 48, [900, 70], True),              # 48 rows: one block with 16 padding rows
+    (2, 2, 96, [333, 1200], True),            # g = 96: blocks straddle the two positions
+    (3, 3, 24, [64, 2, 777], True),           # g = 24, 72 rows: a second block of 8 rows
 ]
 
 
@@ -130,8 +124,6 @@ def test_parity_tcgen05_64_row_tiles(case, num_parts):
 @pytest.mark.parametrize("kernel", ["auto", "tcgen05"])
 @pytest.mark.parametrize("h_q,s_q", [(16, 1), (8, 2), (4, 1), (24, 1), (32, 1), (12, 3), (48, 1), (64, 1), (16, 4)])
 def test_parity_row_paddings(h_q, s_q, kernel):
-    if kernel == "tcgen05" and not tcgen05_takes(s_q, h_q, 1):
-        pytest.skip("query tile not one TMA box")
     # every padded tile height of the kernels (16, 32, 48, 64 rows), ragged row counts
     x = W.make_inputs(W.custom(3, s_q, h_q, 1, [1, 200, 1000], causal=True), seed=h_q * 7 + s_q)
     full_parity(x, kernel=kernel)
