@@ -49,7 +49,7 @@ from paged_mla_decode_11_b200 import workloads as W  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["common.cuh", "decode_tc.cu", "decode_mma.cu"]
+KERNEL_SOURCES = ["common.cuh", "decode_tc.cu", "decode_mma.cu", "decode_wide.cu"]
 
 
 # ----------------------------------------------------------------------------------------
@@ -194,12 +194,19 @@ def pick_sample(x, w, seconds):
 
 
 def cpu_baseline(x, w, unit, seconds=10.0):
+    """The oracle as it stands on the host cores: whole sequences worth about `seconds` of
+    work; a batch the oracle finishes sooner is decoded again until that much has run."""
     import oracle
     seqs = pick_sample(x, w, seconds)
-    dt, nb, fl = oracle_sample(x, w, seqs)
-    val = nb / dt / 1e9 if unit == "GB/s" else fl / dt / 1e12
+    tot_t = tot_b = tot_f = 0.0
+    runs = 0
+    while runs == 0 or (tot_t < 0.8 * seconds and runs < 200):
+        dt, nb, fl = oracle_sample(x, w, seqs)
+        tot_t, tot_b, tot_f, runs = tot_t + dt, tot_b + nb, tot_f + fl, runs + 1
+    val = tot_b / tot_t / 1e9 if unit == "GB/s" else tot_f / tot_t / 1e12
     return {"value": val, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{len(seqs)} of {w.batch} sequences (all query rows), {dt:.1f} s of fp64 oracle work"}
+            "sample": f"{len(seqs)} of {w.batch} sequences (all query rows) decoded {runs} time(s), "
+                      f"{tot_t:.1f} s of fp64 oracle work"}
 
 
 def run_reference(args):
