@@ -1,0 +1,37 @@
+"""The split-KV scheduler on the GPU against the oracle's specification, bit-exact.
+
+The 512-thread scheduler gives each thread ceil(batch / 512) consecutive sequences; the cases
+straddle those boundaries, with empty sequences, one-page and long sequences, and part counts
+from 1 to more than the batch.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import metadata as spec
+from paged_mla_decode_11_b200 import ops
+
+pytestmark = pytest.mark.gpu
+
+
+def lengths(batch, seed):
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, 5000, size=batch)
+    lens[rng.random(batch) < 0.1] = 0          # empty sequences
+    lens[rng.random(batch) < 0.05] = 64        # exactly one page
+    if batch > 3:
+        lens[batch // 3] = 70000               # one long sequence
+    return lens.astype(np.int32)
+
+
+@pytest.mark.parametrize("batch", [1, 2, 31, 32, 33, 95, 1000, 1023, 1024, 1025, 3000])
+@pytest.mark.parametrize("rows", [16, 128])
+def test_plan_matches_specification(batch, rows):
+    for num_parts in (1, 7, 148, batch + 5):
+        lens = lengths(batch, seed=batch * 7 + rows + num_parts)
+        tile, splits = ops.get_mla_metadata(torch.from_numpy(lens).cuda(), rows, 1, num_parts=num_parts)
+        torch.cuda.synchronize()
+        want_tiles, want_splits = spec.schedule(lens.tolist(), num_parts, rows)
+        assert tile.cpu().tolist() == want_tiles
+        assert splits.cpu().tolist() == want_splits
