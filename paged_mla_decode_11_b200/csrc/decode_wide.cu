@@ -21,8 +21,7 @@
 //                        keys, V = the page's first 512 columns read in place as an
 //                        MN-major operand
 // Warp roles:
-//   warp 0      TMA producer: pages gathered through block_table into the ring, pages three
-//               ahead prefetched into L2
+//   warp 0      TMA producer: pages gathered through block_table into the ring
 //   warp 1      TMEM owner and MMA issuer (one thread): QK runs up to two pages ahead of PV
 //               and each step issues whichever group is ready, so the softmax of one page
 //               overlaps tensor-core work on the next
@@ -42,7 +41,6 @@ struct Wide64 {
   static constexpr int kThreads = 320;
   static constexpr int BM = 64;                             // query rows per CTA
   static constexpr int NS = 3;                              // page ring depth
-  static constexpr int kAhead = 3;                          // pages prefetched into L2 ahead
   static constexpr int kPBytes = BM * 128;                  // 64 rows x 64 keys bf16
   static constexpr int kOffRing = 0;
   static constexpr int kOffP = kOffRing + NS * kPageBytes;
@@ -143,10 +141,6 @@ __device__ __forceinline__ void tmem_st_half16(uint32_t taddr, const uint4 (&v)[
       : "memory");
 }
 
-// L2 prefetch of one latent page (64 tokens of a single latent head: contiguous).
-__device__ __forceinline__ void prefetch_page(const DecodeParams &p, int phys) {
-  if (p.h_kv == 1) prefetch_l2_bulk(p.kv_base + (int64_t)phys * kPage * p.kv_token_bytes, uint32_t(kPage * p.kv_token_bytes));
-}
 
 __global__ void __launch_bounds__(Wide64::kThreads, 1)
     decode_wide_kernel(const __grid_constant__ CUtensorMap kv_map, const DecodeParams p) {
@@ -206,13 +200,8 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       for (int base = 0; ok && base < w.ntiles; base += 32) {
         const int mine = base + lane < w.ntiles ? bt_row[base + lane] : 0;
         const int cnt = min(32, w.ntiles - base);
-        // With two pages in the ring a slot refills only after the page before it is done;
-        // pages kAhead ahead are pulled into L2 first so that the refill reads L2, not HBM.
-        if (lane < min(T::kAhead, cnt)) prefetch_page(p, mine);
         for (int i = 0; ok && i < cnt; ++i, ++it) {
           const int phys = __shfl_sync(0xffffffffu, mine, i);
-          const int ahead = __shfl_sync(0xffffffffu, mine, min(i + T::kAhead, 31));
-          if (lane == 0 && i + T::kAhead < cnt) prefetch_page(p, ahead);
           const int s = it % T::NS;
           int g2 = 1;
           if (lane == 0) {
