@@ -438,6 +438,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
       prefetch_tensormap(&kv_map);
       prefetch_tensormap(&q_map);
     }
+    const uint64_t policy = l2_evict_first_policy();  // pages are read once
     int it = 0, qs = 0, last_q = -1;
     int last_chunk[T::NS];
 #pragma unroll
@@ -478,7 +479,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
               const int row = phys * kPage + ((base + i) & 1) * T::KC;
 #pragma unroll
               for (int c = 0; c < kColBlocks; ++c)
-                tma_load_3d(dst + c * T::kChunkBlock, &kv_map, bar(T::FULL + s), c * 64, kvh, row);
+                tma_load_3d_hint(dst + c * T::kChunkBlock, &kv_map, bar(T::FULL + s), c * 64, kvh, row, policy);
               last_chunk[s] = it;
             }
           }

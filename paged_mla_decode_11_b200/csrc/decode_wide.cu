@@ -188,6 +188,9 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
   if (warp == 0) {
     // ------------------------- producer: pages -------------------------
     if (lane == 0) prefetch_tensormap(&kv_map);
+    // pages are read once, unless another 64-row block of the same latent head reads them
+    // too (from L2, shortly after)
+    const uint64_t policy = gridDim.y == 1 ? l2_evict_first_policy() : l2_evict_normal_policy();
     int it = 0;
     int last_page[T::NS];
 #pragma unroll
@@ -212,7 +215,8 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
               const uint32_t dst = sRing + s * kPageBytes;
 #pragma unroll
               for (int c = 0; c < kColBlocks; ++c)
-                tma_load_3d(dst + c * kPageBlockBytes, &kv_map, bar(T::FULL + s), c * 64, kvh, phys * kPage);
+                tma_load_3d_hint(dst + c * kPageBlockBytes, &kv_map, bar(T::FULL + s), c * 64, kvh, phys * kPage,
+                                 policy);
               last_page[s] = it;
             }
           }
