@@ -108,7 +108,12 @@ MLA_API int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_
  *   num_splits     device int32 [batch + 1], written: prefix sums of the number of parts
  *                  touching each sequence (num_splits[0] = 0)
  *   rows_per_kv_head  s_q * h_q / h_kv (sets OVH); num_parts from mla_num_parts.
- * Launches one small kernel on `stream`.  Errors: MLA_ERR_ARG (null pointer, batch < 1
+ * Launches one small kernel on `stream`, as a programmatic dependent launch: it reads
+ * cache_seqlens and computes the plan while the kernel before it in the stream is still
+ * finishing, and writes tile_metadata and num_splits only after that kernel has completed.
+ * So a kernel that writes cache_seqlens and signals programmatic dependents
+ * (griddepcontrol.launch_dependents) must do so after those writes; ordinary launches and
+ * copies are always waited for.  Errors: MLA_ERR_ARG (null pointer, batch < 1
  * or > MLA_MAX_BATCH, rows_per_kv_head < 1, num_parts < 1), MLA_ERR_CUDA.  Negative lengths are not detected
  * on the device; mla_decode_paged's callers must pass lengths >= 0.
  */

@@ -25,6 +25,9 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 6)
     combine_kernel(const int32_t *__restrict__ num_splits, int s_q, int h_q, int h_kv, int R,
                    const float *__restrict__ lse_accum, const float *__restrict__ o_accum,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+  // the next kernel may start its prologue; the scheduler kernel of a next step computes its
+  // plan meanwhile and writes it only after this kernel has completed
+  grid_launch_dependents();
   const int b = blockIdx.x, kvh = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int row = blockIdx.y * (kCombineWarps / 2) + warp / 2, half = warp % 2;

@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(kMetaThreads)
   const long long payload = (T + num_parts - 1) / num_parts;
 
   // 2. one thread per part: both cuts -> cursors by binary search over start[]
-  for (int p = threadIdx.x; p < num_parts; p += kMetaThreads) {
+  auto part_entry = [&](int p, int32_t (&t)[8]) {
     int ci[2];
     long long ck[2];
 #pragma unroll
@@ -88,27 +88,44 @@ __global__ void __launch_bounds__(kMetaThreads)
         ck[e] = max(0ll, x - start[a] - ovh);
       }
     }
-    const int ord = ck[0] > 0 ? int(p - (start[ci[0]] + ovh) / payload) : 0;
-    int32_t *t = tile_md + p * 8;
     t[0] = ci[0];
     t[1] = int32_t(ck[0] * kPage);
     t[2] = ci[1];
     t[3] = int32_t(ck[1] * kPage);
-    t[4] = ord;
-    t[5] = 0;
-    t[6] = 0;
-    t[7] = 0;
-  }
+    t[4] = ck[0] > 0 ? int(p - (start[ci[0]] + ovh) / payload) : 0;
+    t[5] = t[6] = t[7] = 0;
+  };
+  int32_t held[8];
+  const bool one_pass = num_parts <= kMetaThreads;
+  if (one_pass && threadIdx.x < num_parts) part_entry(threadIdx.x, held);
 
   // 3. parts touching sequence b: 1 + cuts strictly inside its page units
+  auto splits_of = [&](int b) { return 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + ovh) / payload); };
   long long cnt = 0;
-  for (int b = lo; b < hi; ++b)
-    cnt += 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + ovh) / payload);
+  for (int b = lo; b < hi; ++b) cnt += splits_of(b);
   long long all;
   run = block_exclusive_scan(cnt, scratch, &all);
+
+  // The plan is complete; the kernel before this one in the stream may still read the
+  // buffers it is written to (a previous step's plan), so wait for it before writing.  All
+  // of the above, the length reads included, overlapped that kernel's tail.
+  grid_dependency_wait();
+  if (one_pass) {
+    if (threadIdx.x < num_parts) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) tile_md[threadIdx.x * 8 + k] = held[k];
+    }
+  } else {
+    for (int p = threadIdx.x; p < num_parts; p += kMetaThreads) {
+      int32_t t[8];
+      part_entry(p, t);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) tile_md[p * 8 + k] = t[k];
+    }
+  }
   if (threadIdx.x == 0) num_splits[0] = 0;
   for (int b = lo; b < hi; ++b) {
-    run += 1 + max(0ll, (start[b + 1] - 1) / payload - (start[b] + ovh) / payload);
+    run += splits_of(b);
     num_splits[b + 1] = int32_t(run);
   }
 }
@@ -121,8 +138,9 @@ cudaError_t launch_metadata(const int32_t *seqlens, int batch, int ovh, int num_
                                   int((MLA_MAX_BATCH + 1) * sizeof(long long)));
     if (e != cudaSuccess) return e;
   }
-  metadata_kernel<<<1, kMetaThreads, smem, stream>>>(seqlens, batch, ovh, num_parts, tile_md, num_splits);
-  return cudaGetLastError();
+  // launched early: the plan is computed while the previous kernel finishes (see above)
+  return launch_early(metadata_kernel, dim3(1), dim3(kMetaThreads), smem, stream, seqlens, batch, ovh, num_parts,
+                      tile_md, num_splits);
 }
 
 }  // namespace pagedmla
