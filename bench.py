@@ -60,6 +60,51 @@ def dist_env():
         int(os.environ.get("WORLD_SIZE", "1"))
 
 
+class RankGroup:
+    """One process per GPU (torchrun environment).  Sequences are independent, so the data
+    path has no collective; the group only aligns the ranks (barrier) and reduces the timings
+    (maximum over ranks).  `backend` is "nccl" on GPUs, "gloo" for the CPU tests."""
+
+    def __init__(self, backend: str, device: torch.device):
+        self.rank, self.local_rank, self.world = dist_env()
+        self.device = device
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+            self.pg = dist
+
+    def _sync(self):
+        if self.device.type == "cuda":
+            torch.cuda.synchronize(self.device)
+
+    def barrier(self):
+        if self.pg is not None:
+            t = torch.zeros(1, device=self.device)
+            self.pg.all_reduce(t)
+        self._sync()
+
+    def max(self, v: float) -> float:
+        if self.pg is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg is not None:
+            self.pg.destroy_process_group()
+            self.pg = None
+
+
+def aggregate_throughput(units_per_rank: float, world: int, seconds_per_step: float) -> float:
+    """Whole-job throughput: the units every rank processed in one step over the slowest
+    rank's step time (weak scaling: each rank decodes its own batch)."""
+    return units_per_rank * world / seconds_per_step
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -273,25 +318,8 @@ def run_ours(args):
         raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} processes (launch with torchrun)")
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
-
-    def barrier():
-        if pg is not None:
-            t = torch.zeros(1, device=dev)
-            pg.all_reduce(t)
-        torch.cuda.synchronize(dev)
-
-    def max_over_ranks(v: float) -> float:
-        if pg is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        return float(t.item())
+    group = RankGroup("nccl", dev)
+    barrier, max_over_ranks = group.barrier, group.max
 
     w = W.WORKLOADS[args.workload]
     R = w.rows_per_kv_head
@@ -376,8 +404,8 @@ def run_ours(args):
     elapsed = max_over_ranks(start.elapsed_time(end) * 1e-3)
     kernel_s = max_over_ranks(k0.elapsed_time(k1) * 1e-3 / args.steps)
     per_step = elapsed / args.steps
-    total_bytes = nbytes * world
-    total_flops = flops * world
+    total_bytes = aggregate_throughput(nbytes, world, 1.0)
+    total_flops = aggregate_throughput(flops, world, 1.0)
     value = (total_bytes / per_step / 1e9) if unit == "GB/s" else (total_flops / per_step / 1e12)
 
     peaks, peak_kind = load_peaks()
@@ -435,8 +463,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(x, w, unit)
 
-    if pg is not None:
-        pg.destroy_process_group()
+    group.close()
     if rank != 0:
         return
     cfg = workload_config(w)
