@@ -4,8 +4,8 @@
 // One warp per (sequence, latent head, query row, half of the value columns); sequences
 // with a single split are skipped (the decode kernel wrote them directly).  In its 256
 // columns each lane owns 8 as two float4s strided 128 apart, so every warp-wide access
-// covers 512 contiguous bytes.  CTAs are small (4 warps, few registers) so that they fit
-// beside a running decode CTA and are resident before the decode kernel ends.
+// covers 512 contiguous bytes.  CTAs are small (4 warps) so that many of them are resident
+// as soon as the decode kernel's CTAs exit.
 //
 // The kernel is launched early (programmatic dependent launch) and runs after the decode
 // kernel's last CTA, so its latency is the tail of every decode call.  It therefore reads
@@ -17,22 +17,26 @@
 namespace pagedmla {
 
 constexpr int kCombineWarps = 4;           // two rows x two column halves
-constexpr int kBatch = 4;                  // splits whose partial rows are loaded together
+constexpr int kBatch = 8;                  // splits whose partial rows are loaded together
 
-// 6 CTAs per SM bound the registers to 80 per thread: one CTA then fits beside a decode
-// CTA's 320 threads x 168 registers.
-__global__ void __launch_bounds__(kCombineWarps * 32, 6)
+// 4 CTAs per SM bound the registers to 128 per thread (eight splits' rows in flight).
+__global__ void __launch_bounds__(kCombineWarps * 32, 4)
     combine_kernel(const int32_t *__restrict__ num_splits, int s_q, int h_q, int h_kv, int R,
                    const float *__restrict__ lse_accum, const float *__restrict__ o_accum,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
   // the next kernel may start its prologue; the scheduler kernel of a next step computes its
   // plan meanwhile and writes it only after this kernel has completed
   grid_launch_dependents();
-  const int b = blockIdx.x, kvh = blockIdx.z;
+  // row pairs of a sequence are the fastest grid index, so all rows of a long sequence (tens
+  // of splits) are scheduled in the first wave rather than spread over the whole grid
+  const int b = blockIdx.y, kvh = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int row = blockIdx.y * (kCombineWarps / 2) + warp / 2, half = warp % 2;
-  const int ns0 = num_splits[b];
-  const int n = num_splits[b + 1] - ns0;
+  const int row = blockIdx.x * (kCombineWarps / 2) + warp / 2, half = warp % 2;
+  // Everything this kernel reads comes from kernels that may still be running when it
+  // starts (programmatic dependent launch), so it reads through L2 (ld.global.cg), never
+  // through the non-coherent read-only path.
+  const int ns0 = __ldcg(num_splits + b);
+  const int n = __ldcg(num_splits + b + 1) - ns0;
   if (n <= 1 || row >= R) return;
   const int g = h_q / h_kv;
   const int64_t stride = int64_t(h_kv) * R;  // between consecutive splits
@@ -40,25 +44,26 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 6)
   auto part_row = [&](int k) {
     return reinterpret_cast<const float4 *>(o_accum + (base + k * stride) * kDV + half * (kDV / 2));
   };
+  auto lse_of = [&](int k) { return __ldcg(lse_accum + base + k * stride); };
   grid_dependency_wait();  // partials come from the decode kernel just before
 
   // one round trip: split `lane`'s LSE and the first kBatch splits' partial rows
-  const float lk = lane < n ? lse_accum[base + lane * stride] : -INFINITY;
+  const float lk = lane < n ? lse_of(lane) : -INFINITY;
   float4 v[kBatch][2];
 #pragma unroll
   for (int j = 0; j < kBatch; ++j)
     if (j < n)
 #pragma unroll
-      for (int i = 0; i < 2; ++i) v[j][i] = part_row(j)[lane + 32 * i];
+      for (int i = 0; i < 2; ++i) v[j][i] = __ldcg(part_row(j) + lane + 32 * i);
 
   // merged LSE: max over splits, then ln sum exp
   float mx = lk;
-  for (int k = lane + 32; k < n; k += 32) mx = fmaxf(mx, lse_accum[base + k * stride]);
+  for (int k = lane + 32; k < n; k += 32) mx = fmaxf(mx, lse_of(k));
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float sum = 0.f;
   if (mx != -INFINITY) {
     sum = expf(lk - mx);
-    for (int k = lane + 32; k < n; k += 32) sum += expf(lse_accum[base + k * stride] - mx);
+    for (int k = lane + 32; k < n; k += 32) sum += expf(lse_of(k) - mx);
   }
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   const float tot = mx == -INFINITY ? -INFINITY : mx + logf(sum);
@@ -68,7 +73,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 6)
   for (int i = 0; i < 2; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int k0 = 0; k0 < n; k0 += 32) {
     // lane j holds the weight of split k0 + j
-    const float l = k0 == 0 ? lk : (k0 + lane < n ? lse_accum[base + (k0 + lane) * stride] : -INFINITY);
+    const float l = k0 == 0 ? lk : (k0 + lane < n ? lse_of(k0 + lane) : -INFINITY);
     const float wl = tot != -INFINITY && k0 + lane < n ? expf(l - tot) : 0.f;
     const int kn = min(32, n - k0);
     for (int j0 = 0; j0 < kn; j0 += kBatch) {
@@ -77,7 +82,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 6)
         for (int j = 0; j < kBatch; ++j)
           if (j0 + j < kn)
 #pragma unroll
-            for (int i = 0; i < 2; ++i) v[j][i] = part_row(k0 + j0 + j)[lane + 32 * i];
+            for (int i = 0; i < 2; ++i) v[j][i] = __ldcg(part_row(k0 + j0 + j) + lane + 32 * i);
       }
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
@@ -109,7 +114,7 @@ cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_
                            const float *lse_accum, const float *o_accum, __nv_bfloat16 *out,
                            float *lse, cudaStream_t stream) {
   const int R = s_q * (h_q / h_kv);
-  dim3 grid(batch, (R + kCombineWarps / 2 - 1) / (kCombineWarps / 2), h_kv);
+  dim3 grid((R + kCombineWarps / 2 - 1) / (kCombineWarps / 2), batch, h_kv);
   return launch_early(combine_kernel, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv, R,
                       lse_accum, o_accum, out, lse);
 }

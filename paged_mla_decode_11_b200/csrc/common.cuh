@@ -420,10 +420,15 @@ struct PartCursor {
   int bi, bt, ei, et, bord;
 };
 
+// The plan is written by the scheduler kernel, which may still be running when a decode
+// kernel starts (programmatic dependent launch): after griddepcontrol.wait it is read
+// through L2 (ld.global.cg), never through the non-coherent read-only path.
 __device__ __forceinline__ PartCursor load_part(const int32_t *tile_md, int part) {
   const int32_t *m = tile_md + part * 8;
-  return PartCursor{m[0], m[1], m[2], m[3], m[4]};
+  return PartCursor{__ldcg(m), __ldcg(m + 1), __ldcg(m + 2), __ldcg(m + 3), __ldcg(m + 4)};
 }
+
+__device__ __forceinline__ int split_base(const int32_t *num_splits, int seq) { return __ldcg(num_splits + seq); }
 
 __device__ __forceinline__ bool part_has(const PartCursor &c, int seq) {
   return seq < c.ei || (seq == c.ei && c.et > 0);

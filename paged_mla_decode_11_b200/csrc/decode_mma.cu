@@ -307,8 +307,8 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
         red_sum[(rg * DVS + wd) * 16 + g4 + 8] = l[1];
       }
       named_bar_sync(group_bar, DVS * 32);
-      const int ns0 = p.num_splits[seq];
-      const int nsplit = p.num_splits[seq + 1] - ns0;
+      const int ns0 = split_base(p.num_splits, seq);
+      const int nsplit = split_base(p.num_splits, seq + 1) - ns0;
       const int ord = seq == pc.bi ? pc.bord : 0;
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
@@ -651,8 +651,8 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
       int L, t0, t1;
       const int nch = chunk_range(p, pc, seq, L, t0, t1);
-      const int ns0 = p.num_splits[seq];
-      const int nsplit = p.num_splits[seq + 1] - ns0;
+      const int ns0 = split_base(p.num_splits, seq);
+      const int nsplit = split_base(p.num_splits, seq + 1) - ns0;
       const int ord = seq == pc.bi ? pc.bord : 0;
       const int64_t acc_row0 = ((int64_t)(ns0 + ord) * p.h_kv + kvh) * p.R;
       if (nch == 0) {

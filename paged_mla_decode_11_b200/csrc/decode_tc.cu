@@ -321,8 +321,8 @@ __global__ void __launch_bounds__(TcNarrow<RP>::kThreads, 1)
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
       const Segment sg = make_segment(p, pc, seq);
-      const int ns0 = p.num_splits[seq];
-      const int nsplit = p.num_splits[seq + 1] - ns0;
+      const int ns0 = split_base(p.num_splits, seq);
+      const int nsplit = split_base(p.num_splits, seq + 1) - ns0;
       const int ord = seq == pc.bi ? pc.bord : 0;
       const int64_t acc_row0 = ((int64_t)(ns0 + ord) * p.h_kv + kvh) * p.R;
       if (sg.nch == 0) {

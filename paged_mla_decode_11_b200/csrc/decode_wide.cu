@@ -352,8 +352,8 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
       const WidePiece w = wide_piece(p, pc, seq, row0);
-      const int ns0 = p.num_splits[seq];
-      const int nsplit = p.num_splits[seq + 1] - ns0;
+      const int ns0 = split_base(p.num_splits, seq);
+      const int nsplit = split_base(p.num_splits, seq + 1) - ns0;
       const int ord = seq == pc.bi ? pc.bord : 0;
       const int64_t acc_row = ((int64_t)(ns0 + ord) * p.h_kv + kvh) * p.R + row;
       if (w.ntiles == 0) {
