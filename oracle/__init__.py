@@ -131,8 +131,10 @@ def mla_decode(q, k_cache, block_table, cache_seqlens, dv: int = 512,
 
 
 def combine(lse_parts, o_parts):
-    """Log-sum-exp merge of split partials (the benchmark spec: split-KV partials are merged by
-    a log-sum-exp combine).
+    """Log-sum-exp merge of split partials: the online-softmax rescaling of partial
+    results by a later maximum (dpshk.com notes, section 2.2) applied across the splits
+    that get_mla_metadata's num_splits counts ("OpenSourceWeek Day 1 - FlashMLA", section
+    V.2).
 
     lse_parts [k, ...], o_parts [k, ..., dv] float64.  lse = ln sum_k exp(lse_k),
     out = sum_k exp(lse_k - lse) o_k.  Partials with lse_k = -inf carry no weight; when

@@ -121,6 +121,13 @@ def test_parity_tcgen05_64_row_tiles(case, num_parts):
     full_parity(x, kernel="tcgen05", num_parts=num_parts)
 
 
+@pytest.mark.parametrize("s_q,h_q,h_kv", [(1, 128, 2), (2, 64, 2), (1, 96, 3)], ids=["R64x2", "R64x2-mtp", "R32x3"])
+def test_parity_tcgen05_several_latent_heads(s_q, h_q, h_kv):
+    # the 64-row kernel with more than one latent head: grid z, page rows of head kvh
+    x = W.make_inputs(W.custom(3, s_q, h_q, h_kv, [700, 65, 3000], causal=True), seed=h_q + h_kv)
+    full_parity(x)
+
+
 @pytest.mark.parametrize("kernel", ["auto", "tcgen05"])
 @pytest.mark.parametrize("h_q,s_q", [(16, 1), (8, 2), (4, 1), (24, 1), (32, 1), (12, 3), (48, 1), (64, 1), (16, 4)])
 def test_parity_row_paddings(h_q, s_q, kernel):
