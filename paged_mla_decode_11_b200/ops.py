@@ -113,11 +113,17 @@ def device_sm_count(device: Optional[torch.device] = None) -> int:
     return _sm_count[dev]
 
 
+_parts_cache: dict = {}
+
+
 def num_parts_for(num_sms: int, rows_per_kv_head: int, h_kv: int) -> int:
-    lib = load_library()
-    n = ctypes.c_int(0)
-    _check(lib.mla_num_parts(num_sms, rows_per_kv_head, h_kv, ctypes.byref(n)))
-    return n.value
+    key = (num_sms, rows_per_kv_head, h_kv)
+    if key not in _parts_cache:  # a pure function of its arguments: asked once per shape
+        lib = load_library()
+        n = ctypes.c_int(0)
+        _check(lib.mla_num_parts(num_sms, rows_per_kv_head, h_kv, ctypes.byref(n)))
+        _parts_cache[key] = n.value
+    return _parts_cache[key]
 
 
 def get_mla_metadata(cache_seqlens: torch.Tensor, rows_per_kv_head: int, h_kv: int,
@@ -137,10 +143,16 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, rows_per_kv_head: int, h_kv: i
     return tile, splits
 
 
+_ws_size_cache: dict = {}
+
+
 def workspace_size(batch: int, s_q: int, h_q: int, h_kv: int, num_parts: int) -> int:
-    n = ctypes.c_size_t(0)
-    _check(load_library().mla_workspace_size(batch, s_q, h_q, h_kv, num_parts, ctypes.byref(n)))
-    return n.value
+    key = (batch, s_q, h_q, h_kv, num_parts)
+    if key not in _ws_size_cache:  # a pure function of the shape: asked once per shape
+        n = ctypes.c_size_t(0)
+        _check(load_library().mla_workspace_size(batch, s_q, h_q, h_kv, num_parts, ctypes.byref(n)))
+        _ws_size_cache[key] = n.value
+    return _ws_size_cache[key]
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
