@@ -174,6 +174,32 @@ def test_separate_combine_matches_fused():
     assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
 
 
+@pytest.mark.parametrize("h_q", [16, 64], ids=["16-row-kernel", "64-row-kernel"])
+def test_many_short_sequences_sampled(h_q):
+    # 2048 sequences of 1..256 tokens: parts hold many sequence pieces, so the query reload,
+    # the per-piece epilogue and the scheduler's block path all run many times
+    rng = np.random.default_rng(3)
+    lens = rng.integers(1, 257, size=2048).tolist()
+    x = W.make_inputs(W.custom(2048, 1, h_q, 1, lens, causal=True), seed=21)
+    out, lse, tile, splits = run_gpu(x)
+    check_metadata(x, tile, splits)
+    rows = sample_rows(x, per_seq=1, seed=4)[::7]
+    ro, rl = oracle.mla_decode_rows(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], rows,
+                                    dv=512, softmax_scale=x["softmax_scale"], causal=True)
+    o = out.double().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    l = lse.double().cpu().numpy()[rows[:, 0], rows[:, 2], rows[:, 1]]
+    assert np.abs(o - ro).max() <= OUT_TOL * np.abs(ro).max()
+    assert (np.abs(l - rl) / np.maximum(np.abs(rl), 1.0)).max() <= LSE_RTOL
+
+
+@pytest.mark.parametrize("h_q", [16, 64], ids=["16-row-kernel", "64-row-kernel"])
+def test_all_sequences_empty(h_q):
+    x = W.make_inputs(W.custom(3, 1, h_q, 1, [0, 0, 0], causal=True), seed=2)
+    out, lse, _, _ = run_gpu(x)
+    assert torch.isneginf(lse).all()
+    assert (out == 0).all()
+
+
 def test_deterministic():
     x = W.make_inputs(W.custom(4, 1, 128, 1, [4000, 100, 2500, 64], causal=True), seed=10)
     a = run_gpu(x)
