@@ -6,14 +6,21 @@
 // M = 64 accumulator occupies lanes 0-15 of each 32-lane sub-partition (row 16q + i on lane
 // 32q + i) or, placed at lane 16, lanes 16-31; 128 rows of output would need all of TMEM.
 // TMEM map (512 columns):
-//     lanes 0-15 of each sub-partition    S double buffer (columns 0-127) and the 64-row
-//                                         query tile as the MMA's A operand (columns
-//                                         224-511: 576 bf16 = 288 packed columns)
+//     lanes 0-15 of each sub-partition    score buffers A (columns 0-127, a page pair) and
+//                                         B (columns 128-191, one page); the 64-row query
+//                                         tile as the MMA's A operand (columns 224-511:
+//                                         576 bf16 = 288 packed columns)
 //     lanes 16-31                         O: value columns 0-255 in TMEM columns 0-255,
 //                                         256-511 in columns 256-511
-// With Q in TMEM, shared memory holds a three-page ring and the P tile.  Per 64-token page
-// (one tile, "OpenSourceWeek Day 1 - FlashMLA", section II.1: fixed 64-token blocks):
-//     S = Q K^T          M = 64 rows, N = 64 keys, K = 576, A from TMEM (absorbed-query
+// Shared memory holds a three-page ring laid out column block by column block across the
+// slots: block c (64 columns) of slot s at c * 24 KB + s * 8 KB.  Slots 0-1 and 1-2 are
+// then one 128-key operand with a uniform row stride, and an M = 64 MMA costs the same for
+// N = 64 and N = 128, so the score of a page pair is one MMA per 16-column step at half the
+// cost per key.  Each page's P tile is written into its own rope block (columns 512-575),
+// which no MMA reads once the page's score is done.
+// Per page ("OpenSourceWeek Day 1 - FlashMLA", section II.1: fixed 64-token blocks):
+//     S = Q K^T          M = 64 rows, N = 128 keys (a page pair in slots 0-1 or 1-2 of one
+//                        sequence piece) or 64 keys, K = 576, A from TMEM (absorbed-query
 //                        score over the whole latent row, dpshk.com notes 2.1)
 //     online softmax     running maximum refreshed only when it grows by more than 8 in
 //                        log2 units (same notes 2.2); P -> bf16 tile in shared memory
@@ -22,12 +29,12 @@
 //                        MN-major operand
 // Warp roles:
 //   warp 0      TMA producer: pages gathered through block_table into the ring
-//   warp 1      TMEM owner and MMA issuer (one thread): QK runs up to two pages ahead of PV
-//               and each step issues whichever group is ready, so the softmax of one page
-//               overlaps tensor-core work on the next
+//   warp 1      TMEM owner and MMA issuer (one thread): scores run up to two groups ahead
+//               of PV and each step issues whichever group is ready, so the softmax of one
+//               group overlaps tensor-core work on the next
 //   warps 2-5   softmax, O rescale and epilogue.  The warp on sub-partition q owns rows
-//               16q..16q+15; lane i and lane i + 16 share row 16q + i: keys 0-31 / 32-63 of
-//               the score tile, value columns 0-255 / 256-511 of the output
+//               16q..16q+15; lane i and lane i + 16 share row 16q + i: the two pages of a
+//               pair (keys 0-31 / 32-63 of a single page), value columns 0-255 / 256-511
 //   warps 6-9   query loaders: the next sequence piece's query rows are read into registers
 //               while the current piece runs and written to TMEM once its last QK is done
 // Every mbarrier wait is bounded (pagedmla watchdog); a warp whose wait gives up keeps
@@ -41,26 +48,34 @@ struct Wide64 {
   static constexpr int kThreads = 320;
   static constexpr int BM = 64;                             // query rows per CTA
   static constexpr int NS = 3;                              // page ring depth
-  static constexpr int kPBytes = BM * 128;                  // 64 rows x 64 keys bf16
+  static constexpr int kBoxStride = NS * kPageBlockBytes;   // one column block of every slot
   static constexpr int kOffRing = 0;
-  static constexpr int kOffP = kOffRing + NS * kPageBytes;
+  static constexpr int kOffRope = kOffRing + (kColBlocks - 1) * kBoxStride;  // P tiles
   enum {
     FULL = 0, EMPTY = FULL + NS, QFULL = EMPTY + NS, QFREE = QFULL + 1, SFULL = QFREE + 1,
-    SFREE = SFULL + 2, PFULL = SFREE + 2, PFREE = PFULL + 1, OFULL = PFREE + 1, OFREE = OFULL + 1,
+    SFREE = SFULL + 2, PFULL = SFREE + 2, PVDONE = PFULL + 1, OFULL = PVDONE + 1, OFREE = OFULL + 1,
     FINAL = OFREE + 1, NBARS = FINAL + 1
   };
-  static constexpr int kOffBar = kOffP + kPBytes;
+  static constexpr int kOffBar = kOffRing + NS * kPageBytes;
   static constexpr int kOffTmem = kOffBar + NBARS * 8;
   static constexpr int kOffAbort = kOffTmem + 8;
   static constexpr int kSmemBytes = kOffAbort + 8 + 1024;   // + slack for 1 KB alignment
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTmemS = 0;                     // S buffers: columns 0 and 64
+  static constexpr uint32_t kTmemSA = 0;                    // score of a page pair: 128 columns
+  static constexpr uint32_t kTmemSB = 128;                  // score of a single page: 64 columns
   static constexpr uint32_t kTmemQ = kTmemCols - kD / 2;    // query tile: columns 224-511
   static constexpr uint32_t kHalf1 = 16u << 16;             // lane offset of the O accumulators
-  static_assert(kOffP % 1024 == 0, "swizzled tiles need 1 KB alignment");
-  static_assert(kTmemS + 128 <= kTmemQ, "tensor memory map");
+  static_assert(kOffRope % 1024 == 0 && kPageBlockBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  static_assert(kTmemSB + 64 <= kTmemQ, "tensor memory map");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
+
+// Pages in the score group that starts at page n of a piece with ntiles pages, `it` being
+// the CTA-wide page counter (slot it % 3): a pair when the page sits in slot 0 or 1 and
+// the piece has a next page (the two slots are adjacent in every column block), else one.
+__device__ __forceinline__ int wide_group(int it, int n, int ntiles) {
+  return (it % Wide64::NS != Wide64::NS - 1 && n + 1 < ntiles) ? 2 : 1;
+}
 
 // Shapes the 64-row tensor-core kernel takes: more than 16 rows per latent head.
 bool wide_supported(int R, int g) { return R > 16 && g > 0; }
@@ -155,7 +170,7 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
   const uint32_t bar0 = sbase + T::kOffBar;
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
   volatile int *abort = reinterpret_cast<volatile int *>(smem + T::kOffAbort);
-  const uint32_t sRing = sbase + T::kOffRing, sP = sbase + T::kOffP;
+  const uint32_t sRing = sbase + T::kOffRing, sRope = sbase + T::kOffRope;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::NS; ++s) {
@@ -169,7 +184,7 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       mbar_init(bar(T::SFREE + i), 4);
     }
     mbar_init(bar(T::PFULL), 4);
-    mbar_init(bar(T::PFREE), 1);
+    mbar_init(bar(T::PVDONE), 1);
     mbar_init(bar(T::OFULL), 1);
     mbar_init(bar(T::OFREE), 4);
     mbar_init(bar(T::FINAL), 1);
@@ -212,10 +227,10 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
               g2 = 0;
             } else {
               mbar_arrive_expect_tx(bar(T::FULL + s), kPageBytes);
-              const uint32_t dst = sRing + s * kPageBytes;
+              const uint32_t dst = sRing + s * kPageBlockBytes;
 #pragma unroll
               for (int c = 0; c < kColBlocks; ++c)
-                tma_load_3d_hint(dst + c * kPageBlockBytes, &kv_map, bar(T::FULL + s), c * 64, kvh, phys * kPage,
+                tma_load_3d_hint(dst + c * T::kBoxStride, &kv_map, bar(T::FULL + s), c * 64, kvh, phys * kPage,
                                  policy);
               last_page[s] = it;
             }
@@ -234,12 +249,14 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------- MMA issuer (one thread) -------------------------
-    // Two cursors walk the part's pages: QK runs up to two pages ahead of PV (the S buffers
-    // and the ring bound it).  Each step issues whichever MMA group is ready, PV first: it
-    // frees a ring slot and the P tile sooner.  A fixed QK(n+1)-then-PV(n) order would hold
-    // PV behind a QK that waits for a page whose load could only start after the PV before.
+    // Two cursors walk the part's score groups (wide_group): QK runs up to two groups ahead
+    // of PV (the two score buffers and the ring bound it).  Each step issues whichever MMA
+    // group is ready, PV first: it frees ring slots sooner.  A fixed QK(n+1)-then-PV(n)
+    // order would hold PV behind a QK that waits for a page whose load could only start
+    // after the PV before.
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(64, 64, false, false);
+      const uint32_t idesc_qk1 = idesc_bf16_f32(64, 64, false, false);
+      const uint32_t idesc_qk2 = idesc_bf16_f32(64, 128, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(64, 256, false, true);
       // first piece at or after `seq` with pages; -1 at the end of the part
       auto seek = [&](int seq, int &nt) -> int {
@@ -252,67 +269,83 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
         }
         return -1;
       };
-      int qk_nt = 0, qk_n = 0, qk_t = 0, qk_piece = 0;
+      auto landed = [&](int it) { return mbar_test_wait(bar(T::FULL + it % T::NS), (it / T::NS) & 1); };
+      int qk_nt = 0, qk_n = 0, qk_it = 0, qk_g = 0, qk_piece = 0;
+      int uses_a = 0, uses_b = 0;  // score groups issued into buffer A (pairs) and B (single pages)
       int qk_seq = seek(pc.bi, qk_nt);
-      int pv_nt = qk_nt, pv_n = 0, pv_t = 0, pv_piece = 0;
+      int pv_nt = qk_nt, pv_n = 0, pv_it = 0, pv_g = 0, pv_piece = 0;
       int pv_seq = qk_seq;
       bool have_q = false, ok = true;
       unsigned long long idle_since = 0;
       uint32_t spins = 0;
       while (ok && pv_seq >= 0) {
         bool progressed = false;
-        if (pv_t < qk_t) {
-          // O += P V for page pv_t; the first page of a piece overwrites O once the previous
-          // piece's epilogue has read it
+        if (pv_g < qk_g) {
+          // O += P V for the pages of group pv_g; the first page of a piece overwrites O
+          // once the previous piece's epilogue has read it
+          const int gsz = wide_group(pv_it, pv_n, pv_nt);
           const bool first = pv_n == 0;
-          if (mbar_test_wait(bar(T::PFULL), pv_t & 1) &&
+          if (mbar_test_wait(bar(T::PFULL), pv_g & 1) &&
               (!first || pv_piece == 0 || mbar_test_wait(bar(T::OFREE), (pv_piece - 1) & 1))) {
             tc_fence_after();
-            const uint32_t page = sRing + (pv_t % T::NS) * kPageBytes;
+            for (int j = 0; j < gsz; ++j) {
+              const int s = (pv_it + j) % T::NS;
 #pragma unroll
-            for (int half = 0; half < 2; ++half)
+              for (int half = 0; half < 2; ++half)
 #pragma unroll
-              for (int ks = 0; ks < kPage / 16; ++ks) {
-                // V: value columns 256 half.. (4 column blocks, 8 KB apart), keys 16 ks.. (two
-                // 8-row groups, 1 KB apart); P: keys 16 ks.. of the 64-row tile
-                const uint64_t b = smem_desc_sw128(page + half * 4 * kPageBlockBytes + ks * 2048, kPageBlockBytes, 1024);
-                const uint64_t a = smem_desc_sw128(sP + ks * 32, 16, 1024);
-                umma_bf16(tmem + T::kHalf1 + half * 256, a, b, idesc_pv, (!first || ks > 0) ? 1u : 0u);
-              }
-            umma_commit(bar(T::PFREE));
-            umma_commit(bar(T::EMPTY + pv_t % T::NS));
-            if (++pv_n == pv_nt) {
+                for (int ks = 0; ks < kPage / 16; ++ks) {
+                  // V: value columns 256 half.. (4 column blocks, kBoxStride apart), keys
+                  // 16 ks.. (two 8-row groups, 1 KB apart); P: keys 16 ks.. of the page's tile
+                  const uint64_t b = smem_desc_sw128(sRing + s * kPageBlockBytes + half * 4 * T::kBoxStride + ks * 2048,
+                                                     T::kBoxStride, 1024);
+                  const uint64_t a = smem_desc_sw128(sRope + s * kPageBlockBytes + ks * 32, 16, 1024);
+                  umma_bf16(tmem + T::kHalf1 + half * 256, a, b, idesc_pv, (!first || j > 0 || ks > 0) ? 1u : 0u);
+                }
+              umma_commit(bar(T::EMPTY + s));
+            }
+            umma_commit(bar(T::PVDONE));
+            pv_n += gsz;
+            pv_it += gsz;
+            ++pv_g;
+            if (pv_n == pv_nt) {
               umma_commit(bar(T::OFULL));
               pv_seq = seek(pv_seq + 1, pv_nt);
               pv_n = 0;
               ++pv_piece;
             }
-            ++pv_t;
             progressed = true;
           }
         }
         if (!progressed && qk_seq >= 0) {
-          // S = Q K^T for page qk_t: its page has landed and its S buffer has been read
+          // S = Q K^T for group qk_g: its pages have landed and its score buffer has been read
           if (!have_q) have_q = mbar_test_wait(bar(T::QFULL), qk_piece & 1);
-          const int s = qk_t % T::NS, sb = qk_t & 1;
-          if (have_q && mbar_test_wait(bar(T::FULL + s), (qk_t / T::NS) & 1) &&
-              (qk_t < 2 || mbar_test_wait(bar(T::SFREE + sb), ((qk_t >> 1) - 1) & 1))) {
+          const int gsz = wide_group(qk_it, qk_n, qk_nt);
+          const int sb = gsz == 2 ? 0 : 1;
+          const int uses = sb == 0 ? uses_a : uses_b;
+          if (have_q && landed(qk_it) && (gsz == 1 || landed(qk_it + 1)) &&
+              (uses == 0 || mbar_test_wait(bar(T::SFREE + sb), (uses - 1) & 1))) {
             tc_fence_after();
-            const uint32_t page = sRing + s * kPageBytes;
+            const uint32_t keys = sRing + (qk_it % T::NS) * kPageBlockBytes;
+            const uint32_t d = tmem + (sb == 0 ? T::kTmemSA : T::kTmemSB);
+            const uint32_t idesc = gsz == 2 ? idesc_qk2 : idesc_qk1;
 #pragma unroll 4
             for (int kk = 0; kk < kD / 16; ++kk) {
-              const uint64_t b = smem_desc_sw128(page + (kk >> 2) * kPageBlockBytes + (kk & 3) * 32, 16, 1024);
-              umma_bf16_ts(tmem + T::kTmemS + sb * 64, tmem + T::kTmemQ + kk * 8, b, idesc_qk, kk > 0 ? 1u : 0u);
+              // keys of the group: 8-row groups 1 KB apart, running on into the next slot
+              const uint64_t b = smem_desc_sw128(keys + (kk >> 2) * T::kBoxStride + (kk & 3) * 32, 16, 1024);
+              umma_bf16_ts(d, tmem + T::kTmemQ + kk * 8, b, idesc, kk > 0 ? 1u : 0u);
             }
             umma_commit(bar(T::SFULL + sb));
-            if (++qk_n == qk_nt) {
+            if (sb == 0) ++uses_a; else ++uses_b;
+            qk_n += gsz;
+            qk_it += gsz;
+            ++qk_g;
+            if (qk_n == qk_nt) {
               umma_commit(bar(T::QFREE));  // the query tile may be replaced by the next piece's
               have_q = false;
               qk_seq = seek(qk_seq + 1, qk_nt);
               qk_n = 0;
               ++qk_piece;
             }
-            ++qk_t;
             progressed = true;
           }
         }
@@ -341,14 +374,15 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
   } else if (warp < 6) {
     // ------------------------- softmax / O rescale / epilogue -------------------------
     const int q = warp & 3;                   // TMEM sub-partition of this warp
-    const int hf = lane >> 4;                 // keys 32 hf.. of the score row; value columns 256 hf..
+    const int hf = lane >> 4;                 // page hf of a pair (keys 32 hf.. of a single page); value columns 256 hf..
     const int rl = 16 * q + (lane & 15);      // row within the 64-row block
     const int row = row0 + rl;
     const bool active = row < p.R;
     const int s_row = row / p.g, h_row = kvh * p.g + row % p.g;
     const uint32_t lanes = tmem + (uint32_t(32 * q) << 16);   // S rows of this warp
     const uint32_t olanes = lanes + T::kHalf1;                // O rows of this warp
-    int it = 0, qs = 0;
+    int it = 0, g = 0, qs = 0;  // pages, score groups and pieces done
+    int uses_a = 0, uses_b = 0;  // score groups read from buffer A (pairs) and B (single pages)
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
       const WidePiece w = wide_piece(p, pc, seq, row0);
@@ -375,27 +409,43 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       const int lim = active ? min(w.t1, p.causal ? w.L - (p.s_q - 1 - s_row) : w.L) : -1;
       float m_used = -INFINITY, l = 0.f;  // l: this lane's half of the row sum
 
-      for (int n = 0; n < w.ntiles; ++n) {
-        const int cur = it + n, sb = cur & 1;
-        ok = warp_all(ok && mbar_wait(bar(T::SFULL + sb), (cur >> 1) & 1, abort, p.status, lim_ns));
+      for (int n = 0; n < w.ntiles;) {
+        const int gsz = wide_group(it, n, w.ntiles);
+        const int sb = gsz == 2 ? 0 : 1;
+        ok = warp_all(ok && mbar_wait(bar(T::SFULL + sb), (sb == 0 ? uses_a : uses_b) & 1, abort, p.status, lim_ns));
         tc_fence_after();
-        float sv[32];
-        if (ok) tmem_ld_half32<32>(lanes + T::kTmemS + sb * 64, sv);
+        // pair: lane i < 16 takes the first page (columns 0-63), lane i + 16 the second
+        // (64-127); single page: keys 0-31 / 32-63
+        float sv[2][32];
+        if (ok) {
+          if (gsz == 2) {
+            tmem_ld_half32<64>(lanes + T::kTmemSA, sv[0]);
+            tmem_ld_half32<64>(lanes + T::kTmemSA + 32, sv[1]);
+          } else {
+            tmem_ld_half32<32>(lanes + T::kTmemSB, sv[0]);
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(T::SFREE + sb));
+        if (sb == 0) ++uses_a; else ++uses_b;
 
+        const int nh = gsz;  // 32-key halves this lane holds
         bool need = false;
         float alpha = 1.f;
         if (ok) {
-          const int key0 = w.t0 + n * kPage + 32 * hf;
+          const int key0 = w.t0 + n * kPage + 32 * gsz * hf;
           float mx = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float v = key0 + i < lim ? sv[i] * p.scale_log2 : -INFINITY;
-            sv[i] = v;
-            mx = fmaxf(mx, v);
-          }
+          for (int h = 0; h < 2; ++h)
+            if (h < nh) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float v = key0 + 32 * h + i < lim ? sv[h][i] * p.scale_log2 : -INFINITY;
+                sv[h][i] = v;
+                mx = fmaxf(mx, v);
+              }
+            }
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           const float m_new = fmaxf(m_used, mx);
           need = m_new > m_used + 8.f;
@@ -406,15 +456,20 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
           const float base = m_used == -INFINITY ? 0.f : m_used;
           float sum = 0.f;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            sv[i] = fast_exp2(sv[i] - base);
-            sum += sv[i];
-          }
+          for (int h = 0; h < 2; ++h)
+            if (h < nh) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                sv[h][i] = fast_exp2(sv[h][i] - base);
+                sum += sv[h][i];
+              }
+            }
           l = l * alpha + sum;
         }
         const bool rescale = __any_sync(0xffffffffu, need && n > 0);
-        // P and O may be touched once the previous page's PV has completed
-        if (cur > 0) ok = warp_all(ok && mbar_wait(bar(T::PFREE), (cur - 1) & 1, abort, p.status, lim_ns));
+        // O may be rescaled once the previous group's PV has completed.  The wait is taken
+        // for every group (before P is published) so that the parity walk never skips a phase.
+        if (g > 0) ok = warp_all(ok && mbar_wait(bar(T::PVDONE), (g - 1) & 1, abort, p.status, lim_ns));
         if (ok && rescale) {
           tc_fence_after();
 #pragma unroll 1
@@ -428,17 +483,30 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
           tmem_st_wait();
         }
         if (ok) {
+          // P into the rope block of the page's slot (128-byte swizzle, 64 keys per row)
+          const int slot = (it + (gsz == 2 ? hf : 0)) % T::NS;
+          const int chunk0 = gsz == 2 ? 0 : 4 * hf;
+          const uint32_t dst = sRope + slot * kPageBlockBytes;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sP + sw128(rl, 4 * hf + c)),
-                         "r"(pack_bf16x2(sv[8 * c], sv[8 * c + 1])), "r"(pack_bf16x2(sv[8 * c + 2], sv[8 * c + 3])),
-                         "r"(pack_bf16x2(sv[8 * c + 4], sv[8 * c + 5])), "r"(pack_bf16x2(sv[8 * c + 6], sv[8 * c + 7]))
-                         : "memory");
+          for (int h = 0; h < 2; ++h)
+            if (h < nh) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + sw128(rl, chunk0 + 4 * h + c)),
+                             "r"(pack_bf16x2(sv[h][8 * c], sv[h][8 * c + 1])),
+                             "r"(pack_bf16x2(sv[h][8 * c + 2], sv[h][8 * c + 3])),
+                             "r"(pack_bf16x2(sv[h][8 * c + 4], sv[h][8 * c + 5])),
+                             "r"(pack_bf16x2(sv[h][8 * c + 6], sv[h][8 * c + 7]))
+                             : "memory");
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(T::PFULL));
+        ++g;
+        n += gsz;
+        it += gsz;
       }
 
       // ---- epilogue: O / l -> output (or fp32 split partial), natural-log LSE ----
@@ -478,7 +546,6 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(T::OFREE));
-      it += w.ntiles;
       ++qs;
     }
   } else {
