@@ -425,6 +425,10 @@ def run_ours(args):
     sched_s = max_over_ranks(graph_time(mgraph))
     combine_s = max_over_ranks(graph_time(cgraph))
     clocks = sampler.stop()
+    # a device-side wait that gave up invalidates the run: its kernels returned early
+    for d in reps:
+        if ops.query_status(d["ws"]) != ops.MLA_OK:
+            raise RuntimeError("a device-side wait timed out during the timed region")
     elapsed = max_over_ranks(start.elapsed_time(end) * 1e-3)
     per_step = elapsed / args.steps
     total_bytes = aggregate_throughput(nbytes, world, 1.0)

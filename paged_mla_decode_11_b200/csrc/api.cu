@@ -85,7 +85,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // Page pool [num_pages * 64 tokens][h_kv][576] bf16 as a 3-D map (columns, latent head,
 // token); one box = 64 columns (128 bytes, 128-byte swizzle) x 1 head x box_tokens tokens
-// (64 = a page for the warp-MMA kernel, 32 = half a page for the tcgen05 kernel).
+// (64 = a page for the 64-row kernels, 32 = half a page for the 16-row kernels).
 int encode_kv_map(CUtensorMap *map, const void *k_cache, int64_t num_pages, int h_kv, int box_tokens) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");

@@ -106,16 +106,18 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits until the phase with the given parity has completed.  Gives up after
-// `limit_ns` (checked every 256 polls) or as soon as *abort is set by another thread;
-// on giving up it records the time-out and raises *abort.  Returns true on success.
+// Waits until the phase with the given parity has completed.  Each poll is a try_wait,
+// which suspends the thread in hardware until the phase completes or a short time slice
+// ends, so waiting warps take no issue slots from the ones doing work.  Gives up after
+// `limit_ns` (checked every 16 polls) or as soon as *abort is set by another thread; on
+// giving up it records the time-out and raises *abort.  Returns true on success.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           int *status, unsigned long long limit_ns) {
-  if (mbar_test_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((i & 255u) == 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 0) {
       if (*abort) return false;
       if (global_ns() - t0 > limit_ns) {
         *abort = 1;

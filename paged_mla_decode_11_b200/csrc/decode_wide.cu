@@ -48,12 +48,13 @@ struct Wide64 {
   static constexpr int kThreads = 320;
   static constexpr int BM = 64;                             // query rows per CTA
   static constexpr int NS = 3;                              // page ring depth
+  static constexpr int kPrefetchAhead = 3;                  // L2 prefetch distance in pages
   static constexpr int kBoxStride = NS * kPageBlockBytes;   // one column block of every slot
   static constexpr int kOffRing = 0;
   static constexpr int kOffRope = kOffRing + (kColBlocks - 1) * kBoxStride;  // P tiles
   enum {
     FULL = 0, EMPTY = FULL + NS, QFULL = EMPTY + NS, QFREE = QFULL + 1, SFULL = QFREE + 1,
-    SFREE = SFULL + 2, PFULL = SFREE + 2, PVDONE = PFULL + 1, OFULL = PVDONE + 1, OFREE = OFULL + 1,
+    SFREE = SFULL + 2, PFULL = SFREE + 2, PVDONE = PFULL + 2, OFULL = PVDONE + 2, OFREE = OFULL + 1,
     FINAL = OFREE + 1, NBARS = FINAL + 1
   };
   static constexpr int kOffBar = kOffRing + NS * kPageBytes;
@@ -183,8 +184,10 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       mbar_init(bar(T::SFULL + i), 1);
       mbar_init(bar(T::SFREE + i), 4);
     }
-    mbar_init(bar(T::PFULL), 4);
-    mbar_init(bar(T::PVDONE), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(T::PFULL + i), 4);
+      mbar_init(bar(T::PVDONE + i), 1);
+    }
     mbar_init(bar(T::OFULL), 1);
     mbar_init(bar(T::OFREE), 4);
     mbar_init(bar(T::FINAL), 1);
@@ -206,6 +209,10 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
     // pages are read once, unless another 64-row block of the same latent head reads them
     // too (from L2, shortly after)
     const uint64_t policy = gridDim.y == 1 ? l2_evict_first_policy() : l2_evict_normal_policy();
+    // With one latent head a page's 64 token rows are one contiguous 72 KB range: the first
+    // 64-row block of the part also asks L2 for the page kPrefetchAhead pages ahead, so that
+    // the ring's copies, which can start only when a slot frees, mostly hit L2.
+    const bool prefetch = p.h_kv == 1 && mb == 0;
     int it = 0;
     int last_page[T::NS];
 #pragma unroll
@@ -217,9 +224,11 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
       const int32_t *bt_row = p.block_table + (int64_t)seq * p.bt_stride + w.t0 / kPage;
       for (int base = 0; ok && base < w.ntiles; base += 32) {
         const int mine = base + lane < w.ntiles ? bt_row[base + lane] : 0;
+        const int ahead = prefetch && base + lane + T::kPrefetchAhead < w.ntiles ? bt_row[base + lane + T::kPrefetchAhead] : -1;
         const int cnt = min(32, w.ntiles - base);
         for (int i = 0; ok && i < cnt; ++i, ++it) {
           const int phys = __shfl_sync(0xffffffffu, mine, i);
+          const int pf = __shfl_sync(0xffffffffu, ahead, i);
           const int s = it % T::NS;
           int g2 = 1;
           if (lane == 0) {
@@ -232,6 +241,7 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
               for (int c = 0; c < kColBlocks; ++c)
                 tma_load_3d_hint(dst + c * T::kBoxStride, &kv_map, bar(T::FULL + s), c * 64, kvh, phys * kPage,
                                  policy);
+              if (pf >= 0) prefetch_l2_bulk(p.kv_base + (int64_t)pf * kPage * p.kv_token_bytes, kPageBytes);
               last_page[s] = it;
             }
           }
@@ -249,11 +259,15 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------- MMA issuer (one thread) -------------------------
-    // Two cursors walk the part's score groups (wide_group): QK runs up to two groups ahead
-    // of PV (the two score buffers and the ring bound it).  Each step issues whichever MMA
-    // group is ready, PV first: it frees ring slots sooner.  A fixed QK(n+1)-then-PV(n)
-    // order would hold PV behind a QK that waits for a page whose load could only start
-    // after the PV before.
+    // Two cursors walk the part's score groups (wide_group): QK of group g is issued only
+    // once PV of group g - 2 has been, so QK runs at most two groups ahead of PV.  The four
+    // softmax warps publish P independently, and a warp may finish group g + 1 before a
+    // slower one finishes group g; P hand-offs therefore alternate between two barriers by
+    // group parity, and the bound keeps any warp from reaching group g + 2 before PV(g) is
+    // issued (which needs all four arrivals for g).  Each step issues whichever MMA group
+    // is ready, PV first: it frees ring slots sooner.  A fixed QK(n+1)-then-PV(n) order
+    // would hold PV behind a QK that waits for a page whose load could only start after
+    // the PV before.
     if (lane == 0) {
       const uint32_t idesc_qk1 = idesc_bf16_f32(64, 64, false, false);
       const uint32_t idesc_qk2 = idesc_bf16_f32(64, 128, false, false);
@@ -285,7 +299,7 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
           // once the previous piece's epilogue has read it
           const int gsz = wide_group(pv_it, pv_n, pv_nt);
           const bool first = pv_n == 0;
-          if (mbar_test_wait(bar(T::PFULL), pv_g & 1) &&
+          if (mbar_test_wait(bar(T::PFULL + (pv_g & 1)), (pv_g >> 1) & 1) &&
               (!first || pv_piece == 0 || mbar_test_wait(bar(T::OFREE), (pv_piece - 1) & 1))) {
             tc_fence_after();
             for (int j = 0; j < gsz; ++j) {
@@ -303,7 +317,7 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
                 }
               umma_commit(bar(T::EMPTY + s));
             }
-            umma_commit(bar(T::PVDONE));
+            umma_commit(bar(T::PVDONE + (pv_g & 1)));
             pv_n += gsz;
             pv_it += gsz;
             ++pv_g;
@@ -316,7 +330,7 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
             progressed = true;
           }
         }
-        if (!progressed && qk_seq >= 0) {
+        if (!progressed && qk_seq >= 0 && qk_g < pv_g + 2) {
           // S = Q K^T for group qk_g: its pages have landed and its score buffer has been read
           if (!have_q) have_q = mbar_test_wait(bar(T::QFULL), qk_piece & 1);
           const int gsz = wide_group(qk_it, qk_n, qk_nt);
@@ -467,9 +481,13 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
           l = l * alpha + sum;
         }
         const bool rescale = __any_sync(0xffffffffu, need && n > 0);
-        // O may be rescaled once the previous group's PV has completed.  The wait is taken
-        // for every group (before P is published) so that the parity walk never skips a phase.
-        if (g > 0) ok = warp_all(ok && mbar_wait(bar(T::PVDONE), (g - 1) & 1, abort, p.status, lim_ns));
+        // O may be rescaled once the previous group's PV has completed.  Groups alternate
+        // between two PV-done barriers, and the score of group g (so this softmax) can only
+        // have been issued after PV(g - 3) completed: its pages took slots that PV freed.
+        // The barrier of group g - 1 is therefore at most one phase behind, and the wait is
+        // needed only when rescaling.
+        if (rescale)
+          ok = warp_all(ok && mbar_wait(bar(T::PVDONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort, p.status, lim_ns));
         if (ok && rescale) {
           tc_fence_after();
 #pragma unroll 1
@@ -503,7 +521,7 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(T::PFULL));
+        if (lane == 0) mbar_arrive(bar(T::PFULL + (g & 1)));
         ++g;
         n += gsz;
         it += gsz;

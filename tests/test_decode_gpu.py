@@ -29,14 +29,20 @@ def to_dev(x):
 
 
 def run_gpu(x, num_parts=None, q=None, skip_combine=False, kernel="auto"):
+    """One decode call on its own workspace; also checks that no device-side wait gave up
+    (a pipeline that stalls shows up as a time-out here, not only as wrong values)."""
     d = to_dev(x)
     R = x["s_q"] * x["h_q"] // x["h_kv"]
     tile, splits = ops.get_mla_metadata(d["cache_seqlens"], R, x["h_kv"], num_parts=num_parts)
     qq = d["q"] if q is None else q
+    b, s_q, h_q, _ = qq.shape
+    ws = ops.new_workspace(ops.workspace_size(b, s_q, h_q, x["h_kv"], tile.shape[0]), qq.device)
     out, lse = ops.mla_decode_paged(qq, d["k_cache"], d["block_table"], d["cache_seqlens"], x["dv"],
                                     tile, splits, softmax_scale=x["softmax_scale"],
-                                    causal=x["causal"], skip_combine=skip_combine, kernel=kernel)
+                                    causal=x["causal"], workspace=ws, skip_combine=skip_combine,
+                                    kernel=kernel)
     torch.cuda.synchronize()
+    assert ops.query_status(ws) == ops.MLA_OK, "a device-side wait timed out"
     return out, lse, tile, splits
 
 
