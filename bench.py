@@ -51,7 +51,17 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # nominal B200 figures, reported beside the measured-peak fractions
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
-KERNEL_SOURCES = ["common.cuh", "decode_tc.cu", "decode_mma.cu", "decode_wide.cu"]
+# sources of the decode kernel the library picks for a workload (16 rows or fewer per latent
+# head: the warp-MMA kernel; more: the 64-row tcgen05 kernel); a committed ncu summary stays
+# valid while these are unchanged
+KERNEL_SOURCES = {
+    "decode_mma16_kernel": ["common.cuh", "decode_mma.cu"],
+    "decode_wide_kernel": ["common.cuh", "decode_wide.cu"],
+}
+
+
+def decode_kernel_for(rows_per_kv_head: int) -> str:
+    return "decode_mma16_kernel" if rows_per_kv_head <= 16 else "decode_wide_kernel"
 
 
 # ----------------------------------------------------------------------------------------
@@ -115,24 +125,24 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "paged_mla_decode_11_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, kernel: str):
     """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
-    the current kernel sources; None otherwise."""
+    the current sources of that decode kernel; None otherwise."""
     path = os.path.join(ROOT, "profiles", f"decode_{workload}_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_t = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     m_h = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
-    if not m_t or not m_h or m_h.group(1) != kernel_source_hash():
+    if not m_t or not m_h or m_h.group(1) != kernel_source_hash(kernel):
         return None
     return float(m_t.group(1))
 
@@ -446,7 +456,8 @@ def run_ours(args):
         peak = peaks["bf16_tflops"]
         nominal = NOMINAL_PEAKS["bf16_tflops"]
         r_unit = "TFLOP/s"
-    traffic = recorded_traffic(args.workload)
+    # the summaries were taken with the library's own kernel choice
+    traffic = recorded_traffic(args.workload, decode_kernel_for(R)) if args.kernel == "auto" else None
 
     # end to end through the public API from pinned host buffers (the latent page pool is
     # resident device state; each step sends q, block_table and cache_seqlens and reads

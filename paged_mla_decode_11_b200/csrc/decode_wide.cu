@@ -209,10 +209,12 @@ __global__ void __launch_bounds__(Wide64::kThreads, 1)
     // pages are read once, unless another 64-row block of the same latent head reads them
     // too (from L2, shortly after)
     const uint64_t policy = gridDim.y == 1 ? l2_evict_first_policy() : l2_evict_normal_policy();
-    // With one latent head a page's 64 token rows are one contiguous 72 KB range: the first
-    // 64-row block of the part also asks L2 for the page kPrefetchAhead pages ahead, so that
-    // the ring's copies, which can start only when a slot frees, mostly hit L2.
-    const bool prefetch = p.h_kv == 1 && mb == 0;
+    // With one latent head a page's 64 token rows are one contiguous 72 KB range.  When two
+    // or more 64-row blocks read the same pages, the first also asks L2 for the page
+    // kPrefetchAhead pages ahead, so that the ring's copies, which can start only when a slot
+    // frees, mostly hit L2.  A single row block streams from HBM, where the extra requests
+    // only compete with the ring's own copies.
+    const bool prefetch = p.h_kv == 1 && mb == 0 && gridDim.y > 1;
     int it = 0;
     int last_page[T::NS];
 #pragma unroll
