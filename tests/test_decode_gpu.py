@@ -134,6 +134,32 @@ def test_parity_tcgen05_several_latent_heads(s_q, h_q, h_kv):
     full_parity(x)
 
 
+@pytest.mark.parametrize("h_q", [64, 128], ids=["one-row-block", "two-row-blocks"])
+def test_parity_tcgen05_one_part_walks_every_slot_phase(h_q):
+    # One part per row block walks 40 sequences of 1 to 5 pages in order, so sequence pieces
+    # start in every slot of the three-page ring: page pairs in slots 0-1 and 1-2, pairs back
+    # to back on one score buffer, runs of single pages, ragged last pages.
+    rng = np.random.default_rng(11)
+    lens = (rng.integers(1, 6, size=40) * 64 - rng.integers(0, 64, size=40)).tolist()
+    x = W.make_inputs(W.custom(40, 1, h_q, 1, lens, causal=True), seed=12)
+    full_parity(x, kernel="tcgen05", num_parts=1)
+
+
+@pytest.mark.parametrize("h_q", [16, 64, 128])
+def test_parity_running_max_grows_every_page(h_q):
+    # The p-th page of every sequence is scaled by 1 + 3p, so the row maximum of the scores
+    # grows by more than 8 in log2 units from page to page: the output accumulator is
+    # rescaled in most score groups (in the 64-row kernel, each time after the previous
+    # group's PV has completed).  Both sides read the same scaled bf16 pages.
+    x = W.make_inputs(W.custom(3, 1, h_q, 1, [1000, 640, 129], causal=False), seed=31)
+    kc, bt = x["k_cache"], x["block_table"]
+    for b, L in enumerate(x["cache_seqlens"].tolist()):
+        for p in range((L + 63) // 64):
+            page = int(bt[b, p])
+            kc[page] = (kc[page].float() * (1 + 3 * p)).to(torch.bfloat16)
+    full_parity(x)
+
+
 @pytest.mark.parametrize("kernel", ["auto", "tcgen05"])
 @pytest.mark.parametrize("h_q,s_q", [(16, 1), (8, 2), (4, 1), (24, 1), (32, 1), (12, 3), (48, 1), (64, 1), (16, 4)])
 def test_parity_row_paddings(h_q, s_q, kernel):
