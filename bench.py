@@ -125,11 +125,19 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def _code_only(src: str) -> str:
+    """CUDA source without comments and with whitespace collapsed: what the compiler sees."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def kernel_source_hash(kernel: str) -> str:
+    """Hash of the code (not the comments) of the sources a decode kernel is built from."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "paged_mla_decode_11_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "paged_mla_decode_11_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

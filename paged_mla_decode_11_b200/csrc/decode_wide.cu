@@ -28,7 +28,8 @@
 //                        keys, V = the page's first 512 columns read in place as an
 //                        MN-major operand
 // Warp roles:
-//   warp 0      TMA producer: pages gathered through block_table into the ring
+//   warp 0      TMA producer: pages gathered through block_table into the ring (and, when
+//               two or more row blocks share the pages, an L2 prefetch three pages ahead)
 //   warp 1      TMEM owner and MMA issuer (one thread): scores run up to two groups ahead
 //               of PV and each step issues whichever group is ready, so the softmax of one
 //               group overlaps tensor-core work on the next
