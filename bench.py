@@ -470,9 +470,10 @@ def run_ours(args):
     # end to end through the public API from pinned host buffers (the latent page pool is
     # resident device state; each step sends q, block_table and cache_seqlens and reads
     # back out and lse).  Two steps are in flight, as a serving loop would run them: step
-    # i+1's inputs go up on a copy stream and step i-1's result comes back while step i's
-    # kernels run; every step's copies and its result's arrival on the host are inside the
-    # timed region.
+    # i+1's inputs go up on an upload stream and step i-1's result comes back on a download
+    # stream while step i's kernels run (one stream for both directions would queue each
+    # upload behind the previous step's download, which waits for that step's kernels);
+    # every step's copies and its result's arrival on the host are inside the timed region.
     e2e_steps = min(args.steps, 50)
     hq = x["q"].pin_memory()
     hbt = x["block_table"].pin_memory()
@@ -480,12 +481,15 @@ def run_ours(args):
     d0 = reps[0]
     ws_e2e = d0["ws"]
     kstream = torch.cuda.current_stream(dev)  # the API launches on the current stream
-    cstream = torch.cuda.Stream(device=dev)
+    up_stream = torch.cuda.Stream(device=dev)
+    down_stream = torch.cuda.Stream(device=dev)
     slots = []
     for _ in range(2):
         slots.append({
             "q": torch.empty_like(d0["q"]), "bt": torch.empty_like(d0["block_table"]),
             "sl": torch.empty_like(d0["cache_seqlens"]),
+            "tile": torch.empty(nparts, ops.TILE_FIELDS, dtype=torch.int32, device=dev),
+            "splits": torch.empty(w.batch + 1, dtype=torch.int32, device=dev),
             "out": torch.empty(w.batch, w.s_q, w.h_q, 512, dtype=torch.bfloat16, device=dev),
             "lse": torch.empty(w.batch, w.h_q, w.s_q, dtype=torch.float32, device=dev),
             "hout": torch.empty(w.batch, w.s_q, w.h_q, 512, dtype=torch.bfloat16).pin_memory(),
@@ -494,37 +498,40 @@ def run_ours(args):
 
     def e2e_issue(i):
         sl_ = slots[i % 2]
-        with torch.cuda.stream(cstream):
+        with torch.cuda.stream(up_stream):
             if i >= 2:
-                cstream.wait_event(sl_["done"])  # step i-2's kernels have read this slot
+                up_stream.wait_event(sl_["done"])  # step i-2's kernels have read this slot
             sl_["q"].copy_(hq, non_blocking=True)
             sl_["bt"].copy_(hbt, non_blocking=True)
             sl_["sl"].copy_(hsl, non_blocking=True)
-            sl_["up"].record(cstream)
+            sl_["up"].record(up_stream)
         kstream.wait_event(sl_["up"])
         if i >= 2:
             kstream.wait_event(sl_["back"])      # step i-2's result has left this slot
-        tile, splits = ops.get_mla_metadata(sl_["sl"], R, w.h_kv)
+        # the plan goes into this slot's buffers: the previous user of the slot (step i-2)
+        # ran earlier on the same stream
+        tile, splits = ops.get_mla_metadata(sl_["sl"], R, w.h_kv, tile_metadata=sl_["tile"],
+                                            num_splits=sl_["splits"])
         ops.flash_mla_with_kvcache(sl_["q"], d0["k_cache"], sl_["bt"], sl_["sl"], 512, tile, splits,
                                    softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
                                    out=sl_["out"], lse=sl_["lse"], kernel=args.kernel)
         sl_["done"].record(kstream)
-        with torch.cuda.stream(cstream):
-            cstream.wait_event(sl_["done"])
+        with torch.cuda.stream(down_stream):
+            down_stream.wait_event(sl_["done"])
             sl_["hout"].copy_(sl_["out"], non_blocking=True)
             sl_["hlse"].copy_(sl_["lse"], non_blocking=True)
-            sl_["back"].record(cstream)
+            sl_["back"].record(down_stream)
 
     def e2e_run(n, e_start=None, e_end=None):
         if e_start is not None:
-            e_start.record(cstream)
+            e_start.record(up_stream)
         for i in range(n):
             e2e_issue(i)
             if i >= 1:
                 slots[(i - 1) % 2]["back"].synchronize()  # the host has step i-1's result
         slots[(n - 1) % 2]["back"].synchronize()
         if e_end is not None:
-            e_end.record(cstream)
+            e_end.record(down_stream)
             e_end.synchronize()
 
     e2e_run(3)

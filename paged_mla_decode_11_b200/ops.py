@@ -44,6 +44,7 @@ EXPORTED = (
 
 _lib = None
 _lib_lock = threading.Lock()
+_I64x3 = ctypes.c_int64 * 3
 
 
 class MlaError(RuntimeError):
@@ -55,6 +56,9 @@ class MlaError(RuntimeError):
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     """Load libpagedmla.so and declare its C signatures (raises if it is not built)."""
     global _lib
+    lib = _lib
+    if lib is not None:  # loaded: no lock on the per-call path
+        return lib
     with _lib_lock:
         if _lib is not None:
             return _lib
@@ -104,12 +108,17 @@ _sm_count: dict = {}
 
 
 def device_sm_count(device: Optional[torch.device] = None) -> int:
+    n = _sm_count.get(device)  # keyed by what the caller passed, then by device index
+    if n is not None:
+        return n
     dev = torch.cuda.current_device() if device is None else torch.device(device).index
     if dev not in _sm_count:
         lib = load_library()
-        n = ctypes.c_int(0)
-        _check(lib.mla_device_sm_count(dev, ctypes.byref(n)))
-        _sm_count[dev] = n.value
+        c = ctypes.c_int(0)
+        _check(lib.mla_device_sm_count(dev, ctypes.byref(c)))
+        _sm_count[dev] = c.value
+    if device is not None:
+        _sm_count[device] = _sm_count[dev]
     return _sm_count[dev]
 
 
@@ -127,20 +136,35 @@ def num_parts_for(num_sms: int, rows_per_kv_head: int, h_kv: int) -> int:
 
 
 def get_mla_metadata(cache_seqlens: torch.Tensor, rows_per_kv_head: int, h_kv: int,
-                     num_parts: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Split-KV plan for one decode step: (tile_metadata [num_parts, 8], num_splits [b+1])."""
+                     num_parts: Optional[int] = None, tile_metadata: Optional[torch.Tensor] = None,
+                     num_splits: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split-KV plan for one decode step: (tile_metadata [num_parts, 8], num_splits [b+1]).
+
+    ``tile_metadata`` and ``num_splits`` may be passed to reuse buffers (contiguous int32 of
+    those shapes on the same device); otherwise they are allocated."""
     _require_cuda(cache_seqlens, "cache_seqlens", torch.int32)
-    if cache_seqlens.dim() != 1 or not cache_seqlens.is_contiguous():
+    shape = cache_seqlens.shape
+    if len(shape) != 1 or not cache_seqlens.is_contiguous():
         raise ValueError("cache_seqlens must be a contiguous 1-D int32 tensor")
     dev = cache_seqlens.device
     if num_parts is None:
         num_parts = num_parts_for(device_sm_count(dev), rows_per_kv_head, h_kv)
-    batch = cache_seqlens.shape[0]
-    tile = torch.empty(num_parts, TILE_FIELDS, dtype=torch.int32, device=dev)
-    splits = torch.empty(batch + 1, dtype=torch.int32, device=dev)
+    batch = shape[0]
+    if tile_metadata is None:
+        tile_metadata = torch.empty(num_parts, TILE_FIELDS, dtype=torch.int32, device=dev)
+    else:
+        _require_cuda(tile_metadata, "tile_metadata", torch.int32)
+        if tile_metadata.shape != (num_parts, TILE_FIELDS) or not tile_metadata.is_contiguous():
+            raise ValueError(f"tile_metadata must be a contiguous [{num_parts}, {TILE_FIELDS}] tensor")
+    if num_splits is None:
+        num_splits = torch.empty(batch + 1, dtype=torch.int32, device=dev)
+    else:
+        _require_cuda(num_splits, "num_splits", torch.int32)
+        if num_splits.shape != (batch + 1,) or not num_splits.is_contiguous():
+            raise ValueError("num_splits must be a contiguous [batch + 1] tensor")
     _check(load_library().mla_get_metadata(cache_seqlens.data_ptr(), batch, rows_per_kv_head, num_parts,
-                                           tile.data_ptr(), splits.data_ptr(), _stream_ptr(dev)))
-    return tile, splits
+                                           tile_metadata.data_ptr(), num_splits.data_ptr(), _stream_ptr(dev)))
+    return tile_metadata, num_splits
 
 
 _ws_size_cache: dict = {}
@@ -192,48 +216,51 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
     _require_cuda(cache_seqlens, "cache_seqlens", torch.int32)
     _require_cuda(tile_metadata, "tile_metadata", torch.int32)
     _require_cuda(num_splits, "num_splits", torch.int32)
-    if q.dim() != 4 or k_cache.dim() != 4 or block_table.dim() != 2:
+    qshape, kshape, btshape = q.shape, k_cache.shape, block_table.shape
+    if len(qshape) != 4 or len(kshape) != 4 or len(btshape) != 2:
         raise ValueError("q and k_cache must be 4-D, block_table 2-D")
-    b, s_q, h_q, d = q.shape
-    num_pages, page, h_kv, d2 = k_cache.shape
+    b, s_q, h_q, d = qshape
+    num_pages, page, h_kv, d2 = kshape
     if d2 != d:
         raise ValueError("q and k_cache disagree on the latent width")
-    if q.stride(3) != 1:
+    qst = q.stride()
+    if qst[3] != 1:
         raise ValueError("q's last dimension must be contiguous")
     if not k_cache.is_contiguous():
         raise ValueError("k_cache must be contiguous")
-    if block_table.stride(1) != 1 or block_table.shape[0] != b:
+    btst = block_table.stride()
+    if btst[1] != 1 or btshape[0] != b:
         raise ValueError("block_table must be [batch, max_pages] with contiguous rows")
     if cache_seqlens.shape != (b,) or not cache_seqlens.is_contiguous():
         raise ValueError("cache_seqlens must be a contiguous [batch] tensor")
-    if tile_metadata.dim() != 2 or tile_metadata.shape[1] != TILE_FIELDS or not tile_metadata.is_contiguous():
+    tshape = tile_metadata.shape
+    if len(tshape) != 2 or tshape[1] != TILE_FIELDS or not tile_metadata.is_contiguous():
         raise ValueError("tile_metadata must be a contiguous [num_parts, 8] tensor")
     if num_splits.shape != (b + 1,):
         raise ValueError("num_splits must be [batch + 1]")
+    flags = KERNELS.get(kernel)
+    if flags is None:
+        raise ValueError(f"kernel must be one of {sorted(KERNELS)}")
+    if skip_combine:
+        flags |= MLA_FLAG_SKIP_COMBINE
     dev = q.device
-    num_parts = tile_metadata.shape[0]
+    num_parts = tshape[0]
     scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
     if out is None:
         out = torch.empty(b, s_q, h_q, dv, dtype=torch.bfloat16, device=dev)
+    elif out.shape != (b, s_q, h_q, dv) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [b, s_q, h_q, dv] tensor")
     if lse is None:
         lse = torch.empty(b, h_q, s_q, dtype=torch.float32, device=dev)
-    if out.shape != (b, s_q, h_q, dv) or out.dtype != torch.bfloat16 or not out.is_contiguous():
-        raise ValueError("out must be a contiguous bf16 [b, s_q, h_q, dv] tensor")
-    if lse.shape != (b, h_q, s_q) or lse.dtype != torch.float32 or not lse.is_contiguous():
+    elif lse.shape != (b, h_q, s_q) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [b, h_q, s_q] tensor")
-    need = workspace_size(b, s_q, h_q, h_kv, num_parts)
     if workspace is None:
-        workspace = _default_workspace(need, dev)
-    strides = (ctypes.c_int64 * 3)(q.stride(0), q.stride(1), q.stride(2))
-    if kernel not in KERNELS:
-        raise ValueError(f"kernel must be one of {sorted(KERNELS)}")
-    flags = (MLA_FLAG_SKIP_COMBINE if skip_combine else 0) | KERNELS[kernel]
+        workspace = _default_workspace(workspace_size(b, s_q, h_q, h_kv, num_parts), dev)
     _check(load_library().mla_decode_paged(
-        q.data_ptr(), strides, b, s_q, h_q, d, k_cache.data_ptr(), num_pages, page, h_kv,
-        block_table.data_ptr(), block_table.stride(0), cache_seqlens.data_ptr(), dv,
-        tile_metadata.data_ptr(), num_parts, num_splits.data_ptr(), scale, int(bool(causal)),
-        out.data_ptr(), lse.data_ptr(), workspace.data_ptr(), workspace.numel(), flags,
-        _stream_ptr(dev)))
+        q.data_ptr(), _I64x3(qst[0], qst[1], qst[2]), b, s_q, h_q, d, k_cache.data_ptr(), num_pages, page,
+        h_kv, block_table.data_ptr(), btst[0], cache_seqlens.data_ptr(), dv, tile_metadata.data_ptr(),
+        num_parts, num_splits.data_ptr(), scale, int(bool(causal)), out.data_ptr(), lse.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), flags, _stream_ptr(dev)))
     return out, lse
 
 
