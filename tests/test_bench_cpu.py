@@ -1,0 +1,95 @@
+"""bench.py bookkeeping that needs no GPU: which ncu traffic figure a bench line may carry,
+and the whole-job aggregate."""
+
+import importlib.util
+import os
+import re
+import shutil
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    argv = sys.argv
+    sys.argv = ["bench.py"]
+    try:
+        spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+    finally:
+        sys.argv = argv
+    return mod
+
+
+def test_code_hash_ignores_comments_and_layout(bench):
+    a = "int f(int x) {  // doubles x\n  return 2 * x; /* a block\n comment */ }\n"
+    b = "/* header */\nint f(int x) {\n  return 2 * x;\n}  // trailing\n"
+    c = "int f(int x) { return 3 * x; }"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    # PTX inside asm strings is code and survives
+    assert "tcgen05.commit" in bench._code_only('asm volatile("tcgen05.commit.b64 [%0];" ::"r"(b)); // x')
+
+
+def _copy_tree(tmp_path):
+    for d in ("profiles", os.path.join("paged_mla_decode_11_b200", "csrc")):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d)
+    return tmp_path
+
+
+@pytest.mark.parametrize("workload,kernel,source", [
+    ("memory_bound", "decode_mma16_kernel", "decode_mma.cu"),
+    ("compute_bound", "decode_wide_kernel", "decode_wide.cu"),
+])
+def test_traffic_follows_the_kernel_code(bench, monkeypatch, tmp_path, workload, kernel, source):
+    root = _copy_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    path = root / "profiles" / f"decode_{workload}_ncu.md"
+    text = path.read_text()
+    recorded = float(re.search(r"traffic_bytes_per_launch:\s*(\S+)", text).group(1))
+    # stamp the summary with the copied sources' hash: the figure is reported
+    stamped = re.sub(r"kernel_source_hash: \S+", "kernel_source_hash: " + bench.kernel_source_hash(kernel), text)
+    path.write_text(stamped)
+    assert bench.recorded_traffic(workload, kernel) == recorded
+    # a comment-only edit keeps it
+    src = root / "paged_mla_decode_11_b200" / "csrc" / source
+    src.write_text(src.read_text() + "\n// a note\n")
+    assert bench.recorded_traffic(workload, kernel) == recorded
+    # a code edit drops it
+    src.write_text(src.read_text() + "\nstatic int unused_marker_for_the_test;\n")
+    assert bench.recorded_traffic(workload, kernel) is None
+    # no summary, no figure
+    path.unlink()
+    assert bench.recorded_traffic(workload, kernel) is None
+
+
+@pytest.mark.parametrize("workload,lo,hi", [("memory_bound", 0.99, 1.05), ("compute_bound", 0.99, 1.10)])
+def test_committed_traffic_is_close_to_the_algorithmic_bytes(bench, workload, lo, hi):
+    # whatever kernel version it was taken on, a committed figure far from the algorithmic
+    # bytes of its workload would mean a wrong capture (another workload, re-reads)
+    import torch
+
+    from paged_mla_decode_11_b200 import workloads as W
+    text = open(os.path.join(ROOT, "profiles", f"decode_{workload}_ncu.md")).read()
+    traffic = float(re.search(r"traffic_bytes_per_launch:\s*(\S+)", text).group(1))
+    w = W.WORKLOADS[workload]
+    # the lengths are the generator's first draw for seed 0 (the bench's inputs)
+    lens = W._draw_seqlens(w, torch.Generator().manual_seed(0)).tolist()
+    nbytes, _ = W.algorithmic_work(lens, w.s_q, w.h_q, w.h_kv, w.causal)
+    assert lo <= traffic / nbytes <= hi
+
+
+def test_decode_kernel_choice_follows_rows(bench):
+    assert bench.decode_kernel_for(16) == "decode_mma16_kernel"
+    assert bench.decode_kernel_for(17) == "decode_wide_kernel"
+    assert bench.decode_kernel_for(256) == "decode_wide_kernel"
+
+
+def test_whole_job_aggregate_is_weak_scaling(bench):
+    # each rank decodes its own batch: N ranks do N times the units in the slowest rank's time
+    assert bench.aggregate_throughput(100.0, 1, 2.0) == 50.0
+    assert bench.aggregate_throughput(100.0, 8, 2.0) == 400.0
