@@ -87,6 +87,15 @@ MLA_API int mla_device_sm_count(int device, int *num_sms);
 MLA_API int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_parts);
 
 /*
+ * mla_metadata_size -- the part count mla_get_metadata needs on the calling thread's current
+ * CUDA device: mla_num_parts with that device's SM count.  tile_metadata then takes
+ * num_parts * 8 int32 and num_splits batch + 1.  Host only (no kernel, no allocation).
+ * Errors: MLA_ERR_ARG (null out pointer, batch < 1 or > MLA_MAX_BATCH, rows_per_kv_head or
+ * h_kv < 1), MLA_ERR_CUDA (no current device).
+ */
+MLA_API int mla_metadata_size(int batch, int rows_per_kv_head, int h_kv, int *num_parts);
+
+/*
  * mla_get_metadata -- the split-KV tile scheduler ("OpenSourceWeek Day 1 - FlashMLA",
  * section V.2: get_mla_metadata(cache_seqlens, s_q*h_q//h_kv, h_kv) -> tile_metadata,
  * num_splits; the pages print its call only, the plan is this library's specification).

@@ -11,6 +11,7 @@ from .ops import (  # noqa: F401
     flash_mla_with_kvcache,
     get_mla_metadata,
     load_library,
+    metadata_size,
     mla_combine,
     mla_decode_paged,
     new_workspace,

@@ -173,6 +173,20 @@ int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_parts) {
   return MLA_OK;
 }
 
+int mla_metadata_size(int batch, int rows_per_kv_head, int h_kv, int *num_parts) {
+  if (!num_parts) return fail(MLA_ERR_ARG, "num_parts is null");
+  if (batch < 1 || batch > MLA_MAX_BATCH)
+    return fail(MLA_ERR_ARG, "batch must be in [1, %d] (got %d)", MLA_MAX_BATCH, batch);
+  if (rows_per_kv_head < 1 || h_kv < 1) return fail(MLA_ERR_ARG, "rows_per_kv_head and h_kv must be >= 1");
+  int device = 0;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int sms = 0;
+  const int rc = mla_device_sm_count(device, &sms);
+  if (rc != MLA_OK) return rc;
+  return mla_num_parts(sms, rows_per_kv_head, h_kv, num_parts);
+}
+
 int mla_get_metadata(const int32_t *cache_seqlens, int batch, int rows_per_kv_head, int num_parts,
                      int32_t *tile_metadata, int32_t *num_splits, mla_stream_t stream) {
   if (!cache_seqlens || !tile_metadata || !num_splits)

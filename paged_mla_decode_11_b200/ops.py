@@ -37,7 +37,7 @@ D_V = 512
 TILE_FIELDS = 8
 
 EXPORTED = (
-    "mla_device_sm_count", "mla_num_parts", "mla_get_metadata", "mla_workspace_size",
+    "mla_device_sm_count", "mla_num_parts", "mla_metadata_size", "mla_get_metadata", "mla_workspace_size",
     "mla_decode_paged", "mla_combine", "mla_query_status", "mla_watchdog_selftest",
     "mla_last_error_string", "mla_decode_paged_static",
 )
@@ -69,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         sig = {
             "mla_device_sm_count": [I, P],
             "mla_num_parts": [I, I, I, P],
+            "mla_metadata_size": [I, I, I, P],
             "mla_get_metadata": [P, I, I, I, P, P, P],
             "mla_workspace_size": [I, I, I, I, I, P],
             "mla_decode_paged": [P, P, I, I, I, I, P, I64, I, I, P, I64, P, I, P, I, P,
@@ -133,6 +134,13 @@ def num_parts_for(num_sms: int, rows_per_kv_head: int, h_kv: int) -> int:
         _check(lib.mla_num_parts(num_sms, rows_per_kv_head, h_kv, ctypes.byref(n)))
         _parts_cache[key] = n.value
     return _parts_cache[key]
+
+
+def metadata_size(batch: int, rows_per_kv_head: int, h_kv: int) -> int:
+    """Part count get_mla_metadata plans on the current CUDA device (tile_metadata rows)."""
+    n = ctypes.c_int(0)
+    _check(load_library().mla_metadata_size(batch, rows_per_kv_head, h_kv, ctypes.byref(n)))
+    return n.value
 
 
 def get_mla_metadata(cache_seqlens: torch.Tensor, rows_per_kv_head: int, h_kv: int,

@@ -72,3 +72,16 @@ def test_host_side_rejections(lib):
     rc = lib.mla_decode_paged(16, strides, 1, 1, 16, 576, 16, 1, 64, 1, 16, 1, 16, 512, 16, 1, 16,
                               ctypes.c_float(-1.0), 1, 16, 16, 256, 1 << 20, 0, None)
     assert rc == -1 and b"softmax_scale" in lib.mla_last_error_string()
+
+
+def test_metadata_size_host_checks(lib):
+    n = ctypes.c_int(0)
+    assert lib.mla_metadata_size(4, 16, 1, None) == -1
+    assert lib.mla_metadata_size(0, 16, 1, ctypes.byref(n)) == -1
+    assert b"batch" in lib.mla_last_error_string()
+    assert lib.mla_metadata_size(4, 0, 1, ctypes.byref(n)) == -1
+    # without a device it reports a CUDA error; with one, the part count of that device
+    rc = lib.mla_metadata_size(4, 16, 1, ctypes.byref(n))
+    assert rc in (0, -5)
+    if rc == 0:
+        assert n.value >= 1

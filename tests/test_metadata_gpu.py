@@ -35,3 +35,12 @@ def test_plan_matches_specification(batch, rows):
         want_tiles, want_splits = spec.schedule(lens.tolist(), num_parts, rows)
         assert tile.cpu().tolist() == want_tiles
         assert splits.cpu().tolist() == want_splits
+
+
+@pytest.mark.parametrize("rows,h_kv", [(16, 1), (64, 1), (128, 1), (256, 1), (64, 2)])
+def test_metadata_size_is_the_default_part_count(rows, h_kv):
+    # the host-side sizing call and the scheduler's default agree on the current device
+    lens = torch.from_numpy(lengths(40, seed=rows + h_kv)).cuda()
+    tile, splits = ops.get_mla_metadata(lens, rows, h_kv)
+    assert ops.metadata_size(40, rows, h_kv) == tile.shape[0]
+    assert tile.shape[0] == ops.num_parts_for(ops.device_sm_count(), rows, h_kv)
