@@ -66,9 +66,9 @@ extern "C" {
 
 #define MLA_FLAG_SKIP_COMBINE 1u  /* mla_decode_paged: leave split partials unmerged */
 #define MLA_FLAG_WARP_MMA 2u      /* mla_decode_paged: force the warp-MMA (mma.sync) kernels */
-#define MLA_FLAG_TCGEN05 4u       /* mla_decode_paged: force the tcgen05 kernels (above 16
-                                     rows per latent head h_q / h_kv must be a multiple or a
-                                     divisor of 64) */
+#define MLA_FLAG_TCGEN05 4u       /* mla_decode_paged: force the tcgen05 kernels (up to 16
+                                     rows per latent head the 16-row tcgen05 kernel; above 16
+                                     rows the default is the tcgen05 kernel already) */
 
 typedef struct CUstream_st *mla_stream_t; /* identical to cudaStream_t */
 
@@ -90,8 +90,8 @@ MLA_API int mla_num_parts(int num_sms, int rows_per_kv_head, int h_kv, int *num_
  * mla_metadata_size -- the part count mla_get_metadata needs on the calling thread's current
  * CUDA device: mla_num_parts with that device's SM count.  tile_metadata then takes
  * num_parts * 8 int32 and num_splits batch + 1.  Host only (no kernel, no allocation).
- * Errors: MLA_ERR_ARG (null out pointer, batch < 1 or > MLA_MAX_BATCH, rows_per_kv_head or
- * h_kv < 1), MLA_ERR_CUDA (no current device).
+ * Errors: MLA_ERR_ARG (null out pointer, batch < 1 or > MLA_MAX_BATCH, rows_per_kv_head
+ * outside [1, 2^20] as in mla_get_metadata, h_kv < 1), MLA_ERR_CUDA (no current device).
  */
 MLA_API int mla_metadata_size(int batch, int rows_per_kv_head, int h_kv, int *num_parts);
 
@@ -167,8 +167,10 @@ MLA_API int mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int num_pa
  *                  the workspace for a later mla_combine) and at most one kernel choice:
  *                  MLA_FLAG_WARP_MMA or MLA_FLAG_TCGEN05.  By default the kernel follows
  *                  the measured costs on B200: up to 16 rows per latent head the 16-row
- *                  warp-MMA kernel; above that the 64-row tcgen05 kernel when h_q / h_kv
- *                  is a multiple or a divisor of 64, else the 64-row warp-MMA kernel.
+ *                  warp-MMA kernel; above 16 rows (any h_q / h_kv) the 64-row tcgen05
+ *                  kernel.  MLA_FLAG_WARP_MMA selects the 64-row warp-MMA kernel above 16
+ *                  rows, MLA_FLAG_TCGEN05 the 16-row tcgen05 kernel up to 16 rows; both are
+ *                  kept as measured alternatives and parity-tested like the defaults.
  * Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.  A device
  * wait that times out (never in correct use) sets the workspace status word; read it
  * with mla_query_status.
@@ -221,13 +223,18 @@ MLA_API int mla_watchdog_selftest(void *workspace, uint64_t timeout_ns, mla_stre
  * for deployment only.
  *   - A shape whose split scratch (mla_workspace_size) exceeds 8 MiB is rejected with
  *     MLA_ERR_WORKSPACE before anything is enqueued.
- *   - The first call made while a device is current looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - MLA_FLAG_SKIP_COMBINE is rejected with MLA_ERR_ARG: the split partials stay in the
+ *     library's own array, which cannot be passed to mla_combine, so the combine always
+ *     runs.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, host only); the first call on a device may load the library's
+ *     device code there, so make it before any stream capture.
  *   - Each call clears the array's 256-byte status block on `stream`, then runs the
  *     decode; the partial results in the array are overwritten by every call.
  *   - All calls share the one array: calls that can overlap on the GPU (different
  *     streams without ordering between them) race and corrupt each other's results.
- *   - A device-side time-out is recorded in the array's status block and not reported.
+ *   - A device-side wait that times out is recorded in the array's status block; read it
+ *     with mla_query_status_static before the next static call clears it.
  */
 #define MLA_STATIC_SCRATCH_BYTES (8u << 20)
 MLA_API int mla_decode_paged_static(const void *q, const int64_t q_strides[3], int batch, int s_q,
@@ -237,6 +244,14 @@ MLA_API int mla_decode_paged_static(const void *q, const int64_t q_strides[3], i
                                     int dv, const int32_t *tile_metadata, int num_parts,
                                     const int32_t *num_splits, float softmax_scale, int causal,
                                     void *out, float *lse, unsigned flags, mla_stream_t stream);
+
+/*
+ * mla_query_status_static -- mla_query_status for the static array of
+ * mla_decode_paged_static on the current device: synchronise `stream`, read and clear its
+ * status block.  Returns MLA_OK, MLA_ERR_TIMEOUT (the last static call's device waits gave
+ * up; its out/lse are invalid) or MLA_ERR_CUDA.  Allocates nothing.
+ */
+MLA_API int mla_query_status_static(mla_stream_t stream);
 
 /* Thread-local description of this thread's last error ("" when none). */
 MLA_API const char *mla_last_error_string(void);

@@ -177,7 +177,9 @@ int mla_metadata_size(int batch, int rows_per_kv_head, int h_kv, int *num_parts)
   if (!num_parts) return fail(MLA_ERR_ARG, "num_parts is null");
   if (batch < 1 || batch > MLA_MAX_BATCH)
     return fail(MLA_ERR_ARG, "batch must be in [1, %d] (got %d)", MLA_MAX_BATCH, batch);
-  if (rows_per_kv_head < 1 || h_kv < 1) return fail(MLA_ERR_ARG, "rows_per_kv_head and h_kv must be >= 1");
+  if (rows_per_kv_head < 1 || rows_per_kv_head > (1 << 20))
+    return fail(MLA_ERR_ARG, "rows_per_kv_head must be in [1, 2^20]");
+  if (h_kv < 1) return fail(MLA_ERR_ARG, "h_kv must be >= 1");
   int device = 0;
   cudaError_t e = cudaGetDevice(&device);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");

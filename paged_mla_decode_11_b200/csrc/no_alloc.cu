@@ -8,14 +8,14 @@
 // statically sized device array that the library module itself carries, instead of a
 // caller-provided workspace.  The caller still provides every input and output buffer.
 //
-// The array is a host-side symbol only; its device address is looked up once per device
-// with cudaGetSymbolAddress (on the first call made while that device is current).
+// In host code the array's name is only a host-side stand-in, never a device address: its
+// device address is looked up with cudaGetSymbolAddress on every call, with the caller's
+// device current (a cached address could outlive a reset or re-created primary context,
+// which reloads the module and may move the array).  mla_query_status_static reads the
+// array's status block, so a static call whose device-side waits gave up is reported.
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
-#include <utility>
-#include <vector>
 
 #include "launch.h"
 #include "pagedmla.h"
@@ -26,24 +26,12 @@ constexpr size_t kStaticScratchBytes = MLA_STATIC_SCRATCH_BYTES;  // held on eve
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::mutex g_scratch_mu;
-std::vector<std::pair<int, void *>> g_scratch_ptr;  // (device, device address of g_static_scratch)
-
+// Device address of g_static_scratch on the current device (host-only lookup).
 int static_scratch(void **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return pagedmla::record_error(MLA_ERR_CUDA, "cudaGetDevice failed");
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  for (auto &d : g_scratch_ptr)
-    if (d.first == dev) {
-      *out = d.second;
-      return MLA_OK;
-    }
   void *ptr = nullptr;
-  e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+  cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
   if (e != cudaSuccess || ptr == nullptr)
     return pagedmla::record_error(MLA_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
-  g_scratch_ptr.emplace_back(dev, ptr);
   *out = ptr;
   return MLA_OK;
 }
@@ -56,6 +44,12 @@ extern "C" MLA_API int mla_decode_paged_static(
     const int32_t *cache_seqlens, int dv, const int32_t *tile_metadata, int num_parts,
     const int32_t *num_splits, float softmax_scale, int causal, void *out, float *lse, unsigned flags,
     mla_stream_t stream) {
+  // The split partials stay in the library's private array, which the caller cannot name,
+  // so leaving them unmerged for a later mla_combine is refused.
+  if (flags & MLA_FLAG_SKIP_COMBINE)
+    return pagedmla::record_error(MLA_ERR_ARG,
+                                  "MLA_FLAG_SKIP_COMBINE is not accepted by mla_decode_paged_static: its split "
+                                  "partials live in the library's static array, which mla_combine cannot be given");
   size_t need = 0;
   int rc = mla_workspace_size(batch, s_q, h_q, h_kv, num_parts, &need);
   if (rc) return rc;
@@ -77,4 +71,11 @@ extern "C" MLA_API int mla_decode_paged_static(
   return mla_decode_paged(q, q_strides, batch, s_q, h_q, d, k_cache, num_pages, page_size, h_kv, block_table,
                           block_table_stride, cache_seqlens, dv, tile_metadata, num_parts, num_splits,
                           softmax_scale, causal, out, lse, ws, kStaticScratchBytes, flags, stream);
+}
+
+extern "C" MLA_API int mla_query_status_static(mla_stream_t stream) {
+  void *ws = nullptr;
+  const int rc = static_scratch(&ws);
+  if (rc) return rc;
+  return mla_query_status(ws, stream);
 }

@@ -39,7 +39,7 @@ TILE_FIELDS = 8
 EXPORTED = (
     "mla_device_sm_count", "mla_num_parts", "mla_metadata_size", "mla_get_metadata", "mla_workspace_size",
     "mla_decode_paged", "mla_combine", "mla_query_status", "mla_watchdog_selftest",
-    "mla_last_error_string", "mla_decode_paged_static",
+    "mla_last_error_string", "mla_decode_paged_static", "mla_query_status_static",
 )
 
 _lib = None
@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "mla_combine": [P, I, I, I, I, I, I, P, ctypes.c_size_t, P, P, P],
             "mla_query_status": [P, P],
             "mla_watchdog_selftest": [P, U64, P],
+            "mla_query_status_static": [P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)

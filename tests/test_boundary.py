@@ -80,8 +80,38 @@ def test_metadata_size_host_checks(lib):
     assert lib.mla_metadata_size(0, 16, 1, ctypes.byref(n)) == -1
     assert b"batch" in lib.mla_last_error_string()
     assert lib.mla_metadata_size(4, 0, 1, ctypes.byref(n)) == -1
+    # the same row bound as mla_get_metadata, so no part count is given for a shape the
+    # scheduler call would refuse
+    assert lib.mla_metadata_size(4, (1 << 20) + 1, 1, ctypes.byref(n)) == -1
+    assert b"2^20" in lib.mla_last_error_string()
     # without a device it reports a CUDA error; with one, the part count of that device
     rc = lib.mla_metadata_size(4, 16, 1, ctypes.byref(n))
     assert rc in (0, -5)
     if rc == 0:
         assert n.value >= 1
+
+
+def static_entry(lib):
+    fn = lib.mla_decode_paged_static
+    P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    fn.argtypes = [P, P, I, I, I, I, P, I64, I, I, P, I64, P, I, P, I, P, ctypes.c_float, I, P, P,
+                   ctypes.c_uint, P]
+    fn.restype = I
+    return fn
+
+
+def test_static_entry_host_rejections(lib):
+    # Both refusals happen before the library touches a device.
+    fn = static_entry(lib)
+    strides = (ctypes.c_int64 * 3)(576 * 128, 576 * 128, 576)
+    # leaving split partials unmerged is refused: they would stay in the library's own
+    # array, which the caller cannot pass to mla_combine
+    rc = fn(None, strides, 4, 1, 16, 576, None, 1, 64, 1, None, 1, None, 512, None, 148, None,
+            ctypes.c_float(0.04), 1, None, None, ops.MLA_FLAG_SKIP_COMBINE, None)
+    assert rc == -1
+    assert b"MLA_FLAG_SKIP_COMBINE" in lib.mla_last_error_string()
+    # 2048 sequences x 128 rows of fp32 partials need far more than the static array holds
+    rc = fn(None, strides, 2048, 1, 128, 576, None, 1, 64, 1, None, 1, None, 512, None, 148, None,
+            ctypes.c_float(0.04), 1, None, None, 0, None)
+    assert rc == -3
+    assert b"static scratch holds" in lib.mla_last_error_string()

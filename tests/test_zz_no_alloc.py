@@ -64,12 +64,13 @@ def test_static_scratch_matches_workspace_entry_point(kernel_rows):
     assert int(splits[1] - splits[0]) > 1          # the long sequence is split: scratch is used
     ref_out, ref_lse = ops.mla_decode_paged(d["q"], d["k_cache"], d["block_table"], d["cache_seqlens"], 512,
                                             tile, splits, softmax_scale=w.scale, causal=True)
-    _, fn = static_entry()
+    lib, fn = static_entry()
     for _ in range(2):
         out = torch.full_like(ref_out, float("nan"))
         lse = torch.full_like(ref_lse, float("nan"))
         assert call_static(fn, d, tile, splits, w, out, lse) == 0
-        torch.cuda.synchronize()
+        # the array's status block: no device-side wait of this call gave up
+        assert lib.mla_query_status_static(torch.cuda.current_stream().cuda_stream) == 0
         close(out, lse, ref_out, ref_lse)
 
 
