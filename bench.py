@@ -15,10 +15,15 @@ Timing: W warm-up steps, then exactly K steps replayed from one CUDA graph, brac
 a barrier and a device synchronisation on both sides and timed with CUDA events on the
 launching stream; the maximum over ranks is reported.  Steps rotate over enough copies
 of the inputs that everything a step reads was last touched more than one L2 (126 MB)
-ago.  The roofline duration of the decode kernel comes from a second graph of K decode
-launches alone, back to back over the same rotating inputs and their precomputed plans,
-timed with one pair of CUDA events around the whole replay (events around every launch
-would add their own overhead to each kernel's time).
+ago.  The decode kernel is timed two ways: a second graph of K decode launches alone,
+back to back over the same rotating inputs and their precomputed plans, timed with one
+pair of CUDA events around the whole replay (events around every launch would add their
+own overhead to each kernel's time; each launch's prologue overlaps its predecessor),
+and the median of at least 20 individually event-timed decode + combine runs, each after
+a 256 MB write that evicts L2 (the scheduler is timed the same way, separately).
+
+On one GPU the line also carries `per_workload`: the same measurements (without the
+end-to-end leg, with a ~2 s oracle sample) for every workload of the specification.
 
 N > 1 (torchrun, one process per GPU): sequences are independent, so every rank decodes
 its own batch with no data-path collective (weak scaling); only the timing is reduced.
@@ -332,21 +337,23 @@ def run_reference(args):
 # ----------------------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------------------
-def run_ours(args):
-    from paged_mla_decode_11_b200 import ops
-    rank, local_rank, world = dist_env()
-    if args.gpus != world:
-        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} processes (launch with torchrun)")
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    group = RankGroup("nccl", dev)
-    barrier, max_over_ranks = group.barrier, group.max
+FLUSH_BYTES = 256 * 1024 * 1024  # L2-flush write between individually timed runs (> 126 MB L2)
+ISOLATED_RUNS = 20
 
-    w = W.WORKLOADS[args.workload]
+
+def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
+    """Times one workload: the whole step (scheduler, decode, combine) from a CUDA graph of
+    K steps, the decode kernel from a graph of K back-to-back decode launches, and the
+    median of individually event-timed decode + combine runs (and scheduler runs) with an
+    L2-flush write before each.  Optionally the end-to-end leg through the public API and
+    the CPU oracle's throughput on a bounded sample.  Returns a dict of results."""
+    from paged_mla_decode_11_b200 import ops
+    barrier, max_over_ranks = group.barrier, group.max
+    w = W.WORKLOADS[name]
     R = w.rows_per_kv_head
     x = W.make_inputs(w, seed=args.seed + rank)
     nbytes, flops = workload_work(x, w)
-    unit, bound = metric_of(args.workload)
+    unit, bound = metric_of(name)
     per_rep = x["k_cache"].numel() * 2
     n_rep = max(2, math.ceil(1.5 * L2_BYTES / per_rep) + 1)
 
@@ -382,7 +389,7 @@ def run_ours(args):
             step(reps[i % n_rep])
     # the timed graph: K whole steps back to back (no events between kernels, so each
     # kernel's launch overlaps its predecessor); a second graph of K decode launches alone,
-    # on plans computed beforehand, gives the decode kernel's duration
+    # on plans computed beforehand, gives the decode kernel's back-to-back duration
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for i in range(args.steps):
@@ -414,7 +421,7 @@ def run_ours(args):
     cgraph.replay()
     torch.cuda.synchronize(dev)
 
-    sampler = ClockSampler(local_rank)
+    sampler = ClockSampler(dev.index)
     # keep the GPU loaded for ~1 s before timing so the sampled clocks describe the load
     t_end = time.perf_counter() + 1.0
     while time.perf_counter() < t_end:
@@ -429,6 +436,7 @@ def run_ours(args):
         end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
+
     def graph_time(g):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
@@ -442,11 +450,36 @@ def run_ours(args):
     kernel_s = max_over_ranks(graph_time(kgraph))
     sched_s = max_over_ranks(graph_time(mgraph))
     combine_s = max_over_ranks(graph_time(cgraph))
+
+    # Individually timed runs: before each, a 256 MB write evicts L2; then one event pair
+    # around the decode kernel and its combine (on precomputed plans), and, separately, one
+    # around the scheduler.  Median over the runs.
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    n_iso = max(ISOLATED_RUNS, args.steps)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2 * n_iso)]
+    with torch.cuda.stream(stream):
+        for i in range(n_iso):
+            d = reps[i % n_rep]
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            decode(d, *d["plan"])
+            ev[i][1].record(stream)
+        for i in range(n_iso):
+            d = reps[i % n_rep]
+            flush.fill_(float(i))
+            ev[n_iso + i][0].record(stream)
+            ops.get_mla_metadata(d["cache_seqlens"], R, w.h_kv)
+            ev[n_iso + i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    iso_s = max_over_ranks(statistics.median(ev[i][0].elapsed_time(ev[i][1]) for i in range(n_iso)) * 1e-3)
+    iso_sched_s = max_over_ranks(
+        statistics.median(ev[n_iso + i][0].elapsed_time(ev[n_iso + i][1]) for i in range(n_iso)) * 1e-3)
+    del flush
     clocks = sampler.stop()
     # a device-side wait that gave up invalidates the run: its kernels returned early
     for d in reps:
         if ops.query_status(d["ws"]) != ops.MLA_OK:
-            raise RuntimeError("a device-side wait timed out during the timed region")
+            raise RuntimeError(f"{name}: a device-side wait timed out during the timed region")
     elapsed = max_over_ranks(start.elapsed_time(end) * 1e-3)
     per_step = elapsed / args.steps
     total_bytes = aggregate_throughput(nbytes, world, 1.0)
@@ -454,31 +487,60 @@ def run_ours(args):
     value = (total_bytes / per_step / 1e9) if unit == "GB/s" else (total_flops / per_step / 1e12)
 
     peaks, peak_kind = load_peaks()
+    work = nbytes / 1e9 if bound == "hbm" else flops / 1e12
     if bound == "hbm":
-        achieved = nbytes / kernel_s / 1e9
-        peak = peaks["hbm_gbs"]
-        nominal = NOMINAL_PEAKS["hbm_gbs"]
-        r_unit = "GB/s"
+        peak, nominal, r_unit = peaks["hbm_gbs"], NOMINAL_PEAKS["hbm_gbs"], "GB/s"
     else:
-        achieved = flops / kernel_s / 1e12
-        peak = peaks["bf16_tflops"]
-        nominal = NOMINAL_PEAKS["bf16_tflops"]
-        r_unit = "TFLOP/s"
+        peak, nominal, r_unit = peaks["bf16_tflops"], NOMINAL_PEAKS["bf16_tflops"], "TFLOP/s"
+    achieved = work / kernel_s
+    iso_achieved = work / iso_s
     # the summaries were taken with the library's own kernel choice
-    traffic = recorded_traffic(args.workload, decode_kernel_for(R)) if args.kernel == "auto" else None
+    traffic = recorded_traffic(name, decode_kernel_for(R)) if args.kernel == "auto" else None
+    res = {
+        "workload": name, "config": workload_config(w), "unit": unit, "value": value,
+        "ms_per_step": per_step * 1e3, "n_rep": n_rep, "per_rep_bytes": per_rep,
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+                     "kernel": "decode", "kernel_ms": kernel_s * 1e3,
+                     "kernel_timing": f"average over a graph of {args.steps} back-to-back decode launches",
+                     "isolated_ms": iso_s * 1e3, "isolated_achieved": iso_achieved,
+                     "isolated_frac": iso_achieved / peak,
+                     "isolated_timing": (f"median of {n_iso} individually event-timed decode + combine runs, "
+                                         f"each after a {FLUSH_BYTES >> 20} MB L2-flush write"),
+                     "frac_of_nominal": achieved / nominal, "nominal_peak": nominal,
+                     "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
+                     "whole_page_bytes_per_launch": W.whole_page_bytes(x["cache_seqlens"].tolist(), w.h_kv),
+                     "scheduler_ms": sched_s * 1e3, "scheduler_isolated_ms": iso_sched_s * 1e3,
+                     "combine_ms": combine_s * 1e3},
+        "clocks": clocks,
+    }
 
-    # end to end through the public API from pinned host buffers (the latent page pool is
-    # resident device state; each step sends q, block_table and cache_seqlens and reads
-    # back out and lse).  Two steps are in flight, as a serving loop would run them: step
-    # i+1's inputs go up on an upload stream and step i-1's result comes back on a download
-    # stream while step i's kernels run (one stream for both directions would queue each
-    # upload behind the previous step's download, which waits for that step's kernels);
-    # every step's copies and its result's arrival on the host are inside the timed region.
+    if with_e2e:
+        res["e2e"] = e2e_leg(args, w, x, reps[0], dev, nparts, R, unit, total_bytes, total_flops,
+                             barrier, max_over_ranks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and cpu_seconds > 0:
+        res["cpu_baseline"] = cpu_baseline(x, w, unit, seconds=cpu_seconds)
+    for g in (warm_graph, graph, kgraph, mgraph, cgraph):
+        g.reset()
+    del reps, warm_graph, graph, kgraph, mgraph, cgraph
+    torch.cuda.empty_cache()
+    return res
+
+
+def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barrier, max_over_ranks):
+    """End to end through the public API from pinned host buffers (the latent page pool is
+    resident device state; each step sends q, block_table and cache_seqlens and reads back
+    out and lse).  Two steps are in flight, as a serving loop would run them: step i+1's
+    inputs go up on an upload stream and step i-1's result comes back on a download stream
+    while step i's kernels run (one stream for both directions would queue each upload
+    behind the previous step's download, which waits for that step's kernels); every
+    step's copies and its result's arrival on the host are inside the timed region."""
+    from paged_mla_decode_11_b200 import ops
     e2e_steps = min(args.steps, 50)
     hq = x["q"].pin_memory()
     hbt = x["block_table"].pin_memory()
     hsl = x["cache_seqlens"].pin_memory()
-    d0 = reps[0]
     ws_e2e = d0["ws"]
     kstream = torch.cuda.current_stream(dev)  # the API launches on the current stream
     up_stream = torch.cuda.Stream(device=dev)
@@ -545,40 +607,52 @@ def run_ours(args):
     hout, hlse = slots[0]["hout"], slots[0]["hlse"]
     h2d = hq.numel() * 2 + hbt.numel() * 4 + hsl.numel() * 4
     d2h = hout.numel() * 2 + hlse.numel() * 4
+    return {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": e2e_s * 1e3, "steps_in_flight": 2}
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(x, w, unit)
 
+def run_ours(args):
+    rank, local_rank, world = dist_env()
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} needs {args.gpus} processes (launch with torchrun)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    group = RankGroup("nccl", dev)
+
+    head = measure(args.workload, args, dev, group, rank, world, with_e2e=True, cpu_seconds=10.0)
+    # every workload of the specification on the same line (one GPU only: at N > 1 the
+    # per-rank work is the headline workload alone)
+    per_workload = None
+    if world == 1 and not args.no_per_workload:
+        per_workload = {}
+        for name in W.WORKLOADS:
+            r = head if name == args.workload else measure(name, args, dev, group, rank, world,
+                                                            with_e2e=False, cpu_seconds=2.0)
+            per_workload[name] = {k: r[k] for k in ("config", "unit", "value", "ms_per_step", "roofline",
+                                                    "clocks") if k in r}
+            per_workload[name]["cpu_baseline"] = r.get("cpu_baseline")
     group.close()
     if rank != 0:
         return
-    cfg = workload_config(w)
-    cfg["l2"] = (f"inputs larger than L2: steps rotate over {n_rep} copies of the inputs "
-                 f"({per_rep / 1e6:.0f} MB latent pool each)")
+    cfg = dict(head["config"])
+    cfg["l2"] = (f"inputs larger than L2: steps rotate over {head['n_rep']} copies of the inputs "
+                 f"({head['per_rep_bytes'] / 1e6:.0f} MB latent pool each); isolated runs flush L2 "
+                 f"with a {FLUSH_BYTES >> 20} MB write")
     cfg["parallelism"] = f"dp{world} (independent batches per GPU)"
     cfg["timing"] = (f"{args.steps} steps replayed from one CUDA graph; decode-kernel time from a graph "
-                     f"of {args.steps} back-to-back decode launches on the same rotating inputs")
+                     f"of {args.steps} back-to-back decode launches on the same rotating inputs, and the "
+                     f"median of individually timed decode + combine runs after an L2 flush")
     cfg["kernel"] = args.kernel
     line = {
-        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": cfg,
-        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
-                     "kernel": "decode", "kernel_ms": kernel_s * 1e3,
-                     "frac_of_nominal": achieved / nominal, "nominal_peak": nominal,
-                     "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
-                     "whole_page_bytes_per_launch": W.whole_page_bytes(x["cache_seqlens"].tolist(), w.h_kv),
-                     "scheduler_ms": sched_s * 1e3, "combine_ms": combine_s * 1e3},
-        "cpu_baseline": cpu,
-        "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_s * 1e3, "steps_in_flight": 2},
-        "gpu_launches": 3 * args.steps,
-        "clocks": clocks,
+        "metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": cfg, "roofline": head["roofline"],
+        "cpu_baseline": head.get("cpu_baseline"), "e2e": head["e2e"],
+        "gpu_launches": 3 * args.steps, "clocks": head["clocks"],
     }
+    if per_workload is not None:
+        line["per_workload"] = per_workload
     print(json.dumps(line), flush=True)
 
 
@@ -591,6 +665,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="measure only --workload (by default one GPU also measures every workload)")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "warp_mma"],
                     help="decode kernel choice (auto = the library's choice by shape)")
     args = ap.parse_args()

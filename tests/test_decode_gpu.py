@@ -54,6 +54,9 @@ def check_metadata(x, tile, splits):
 
 
 def assert_parity(out, lse, ref_out, ref_lse):
+    """Element-wise check of every output and LSE entry; returns the error figures (max abs
+    output error over max |ref|, LSE error against max(|ref|, 1), and the plain relative
+    LSE error |lse - ref| / |ref|, which is reported, not bounded)."""
     out = out.double().cpu().numpy()
     lse = lse.double().cpu().numpy()
     ref_inf = np.isneginf(ref_lse)
@@ -62,9 +65,16 @@ def assert_parity(out, lse, ref_out, ref_lse):
     err = np.abs(out - ref_out).max()
     assert err <= OUT_TOL * scale, f"max abs err {err:.3e} > {OUT_TOL} * {scale:.3e}"
     fin = ~ref_inf
+    stats = {"out_err_over_max_ref": err / scale, "lse_rel": 0.0, "lse_plain_rel": 0.0}
     if fin.any():
-        rel = np.abs(lse[fin] - ref_lse[fin]) / np.maximum(np.abs(ref_lse[fin]), 1.0)
+        d = np.abs(lse[fin] - ref_lse[fin])
+        rel = d / np.maximum(np.abs(ref_lse[fin]), 1.0)
         assert rel.max() <= LSE_RTOL, f"lse rel err {rel.max():.3e}"
+        stats["lse_rel"] = float(rel.max())
+        nz = np.abs(ref_lse[fin]) > 0
+        if nz.any():
+            stats["lse_plain_rel"] = float((d[nz] / np.abs(ref_lse[fin][nz])).max())
+    return stats
 
 
 def full_parity(x, **kw):
@@ -249,8 +259,8 @@ def test_watchdog_times_out_and_context_survives():
 
 
 # ---------------------------------------------------------------------------------------
-# Full-size workloads, in the launch configuration the benchmark times: bit-exact plan,
-# finite outputs everywhere, and sampled rows against the oracle computed one by one.
+# Full-size workloads, in the launch configuration the benchmark times: bit-exact plan and
+# every output and LSE entry against the oracle.
 # ---------------------------------------------------------------------------------------
 def sample_rows(x, per_seq=2, seed=0):
     rng = np.random.default_rng(seed)
@@ -268,13 +278,7 @@ def test_full_size_workloads(name):
     x = W.make_inputs(W.WORKLOADS[name], seed=0)
     out, lse, tile, splits = run_gpu(x)
     check_metadata(x, tile, splits)
-    assert torch.isfinite(out).all()
-    assert torch.isfinite(lse).all()
-    rows = sample_rows(x)
-    ro, rl = oracle.mla_decode_rows(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], rows,
-                                    dv=512, softmax_scale=x["softmax_scale"], causal=x["causal"])
-    o = out.double().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
-    l = lse.double().cpu().numpy()[rows[:, 0], rows[:, 2], rows[:, 1]]
-    err = np.abs(o - ro).max()
-    assert err <= OUT_TOL * np.abs(ro).max(), err
-    assert (np.abs(l - rl) / np.maximum(np.abs(rl), 1.0)).max() <= LSE_RTOL
+    ref_out, ref_lse = oracle.mla_decode(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"],
+                                         dv=512, softmax_scale=x["softmax_scale"], causal=x["causal"])
+    stats = assert_parity(out, lse, ref_out, ref_lse)
+    print(f"{name}: " + ", ".join(f"{k} {v:.3e}" for k, v in stats.items()))
