@@ -68,7 +68,9 @@ extern "C" {
 #define MLA_FLAG_WARP_MMA 2u      /* mla_decode_paged: force the warp-MMA (mma.sync) kernels */
 #define MLA_FLAG_TCGEN05 4u       /* mla_decode_paged: force the tcgen05 kernels (up to 16
                                      rows per latent head the 16-row tcgen05 kernel; above 16
-                                     rows the default is the tcgen05 kernel already) */
+                                     rows the default is a tcgen05 kernel already) */
+#define MLA_FLAG_ONE_SM 8u        /* mla_decode_paged: above 16 rows, the 1-SM 64-row tcgen05
+                                     kernel even where the CTA-pair kernel applies */
 
 typedef struct CUstream_st *mla_stream_t; /* identical to cudaStream_t */
 
@@ -165,11 +167,15 @@ MLA_API int mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int num_pa
  *   workspace      device scratch of mla_workspace_size bytes (see there)
  *   flags          0, or an OR of MLA_FLAG_SKIP_COMBINE (leave the split partials in
  *                  the workspace for a later mla_combine) and at most one kernel choice:
- *                  MLA_FLAG_WARP_MMA or MLA_FLAG_TCGEN05.  By default the kernel follows
- *                  the measured costs on B200: up to 16 rows per latent head the 16-row
- *                  warp-MMA kernel; above 16 rows (any h_q / h_kv) the 64-row tcgen05
- *                  kernel.  MLA_FLAG_WARP_MMA selects the 64-row warp-MMA kernel above 16
- *                  rows, MLA_FLAG_TCGEN05 the 16-row tcgen05 kernel up to 16 rows; both are
+ *                  MLA_FLAG_WARP_MMA, MLA_FLAG_TCGEN05 or MLA_FLAG_ONE_SM.  By default
+ *                  the kernel follows the measured costs on B200: up to 16 rows per latent
+ *                  head the 16-row warp-MMA kernel; for whole 128-row blocks with
+ *                  h_q / h_kv a multiple or a divisor of 64 the CTA-pair tcgen05 kernel
+ *                  (two SMs share each MMA, 64 rows each, at the full tensor rate); other
+ *                  shapes above 16 rows the 1-SM 64-row tcgen05 kernel.
+ *                  MLA_FLAG_WARP_MMA selects the 64-row warp-MMA kernel above 16 rows,
+ *                  MLA_FLAG_TCGEN05 the 16-row tcgen05 kernel up to 16 rows and
+ *                  MLA_FLAG_ONE_SM the 1-SM 64-row tcgen05 kernel above 16 rows; all are
  *                  kept as measured alternatives and parity-tested like the defaults.
  * Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE, MLA_ERR_CUDA.  A device
  * wait that times out (never in correct use) sets the workspace status word; read it

@@ -234,10 +234,10 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
     return fail(MLA_ERR_ARG, "softmax_scale must be positive and finite");
-  if (flags & ~(MLA_FLAG_SKIP_COMBINE | MLA_FLAG_WARP_MMA | MLA_FLAG_TCGEN05))
+  if (flags & ~(MLA_FLAG_SKIP_COMBINE | MLA_FLAG_WARP_MMA | MLA_FLAG_TCGEN05 | MLA_FLAG_ONE_SM))
     return fail(MLA_ERR_ARG, "unknown flags 0x%x", flags);
-  if ((flags & MLA_FLAG_WARP_MMA) && (flags & MLA_FLAG_TCGEN05))
-    return fail(MLA_ERR_ARG, "MLA_FLAG_WARP_MMA and MLA_FLAG_TCGEN05 are exclusive");
+  if (__builtin_popcount(flags & (MLA_FLAG_WARP_MMA | MLA_FLAG_TCGEN05 | MLA_FLAG_ONE_SM)) > 1)
+    return fail(MLA_ERR_ARG, "MLA_FLAG_WARP_MMA, MLA_FLAG_TCGEN05 and MLA_FLAG_ONE_SM are exclusive");
   for (int i = 0; i < 3; ++i)
     if (q_strides[i] < 0 || q_strides[i] % 8 != 0)
       return fail(MLA_ERR_ARG, "q strides must be non-negative multiples of 8 elements");
@@ -253,19 +253,24 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
   if (workspace_bytes < wl.total)
     return fail(MLA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, wl.total);
 
-  // Kernel choice.  Measured on B200: a tcgen05 MMA costs at least a 128x128x16 tile (an
-  // M = 64 one as much as M = 128), so up to 16 query rows the 16-row warp-MMA tiles do the
-  // same work in fewer tensor cycles; above that the 64-row tcgen05 kernel.
-  enum { kMma16, kMma64, kTc, kWide } kind;
+  // Kernel choice.  Measured on B200: a 1-SM tcgen05 MMA costs at least a 128x128x16 tile
+  // (an M = 64 one as much as M = 128), so up to 16 query rows the 16-row warp-MMA tiles do
+  // the same work in fewer tensor cycles; a CTA-pair MMA with 64 rows per SM and N = 256
+  // runs at the full rate, so whole 128-row blocks go to the pair kernel; other shapes
+  // above 16 rows to the 1-SM 64-row tcgen05 kernel.
+  enum { kMma16, kMma64, kTc, kWide, kPair } kind;
+  const bool pair_ok = pair_supported(R, g);
   if (flags & MLA_FLAG_WARP_MMA) {
     kind = R <= 16 ? kMma16 : kMma64;
   } else if (flags & MLA_FLAG_TCGEN05) {
-    kind = R <= 16 ? kTc : kWide;
+    kind = R <= 16 ? kTc : (pair_ok ? kPair : kWide);
+  } else if (flags & MLA_FLAG_ONE_SM) {
+    kind = R <= 16 ? kMma16 : kWide;
   } else {
-    kind = R <= 16 ? kMma16 : (wide_supported(R, g) ? kWide : kMma64);
+    kind = R <= 16 ? kMma16 : (pair_ok ? kPair : (wide_supported(R, g) ? kWide : kMma64));
   }
   CUtensorMap map;
-  rc = encode_kv_map(&map, k_cache, num_pages, h_kv, kind == kMma64 || kind == kWide ? kPage : 32);
+  rc = encode_kv_map(&map, k_cache, num_pages, h_kv, kind == kMma64 || kind == kWide || kind == kPair ? kPage : 32);
   if (rc) return rc;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -303,6 +308,14 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
     e = launch_decode_mma(map, p, st);
   } else if (kind == kWide) {
     e = launch_decode_wide(map, p, st);  // reads the query rows itself (any g)
+  } else if (kind == kPair) {
+    // each CTA's 64 query rows as one TMA box: 64 heads of one position (g a multiple of
+    // 64), or all g heads of 64 / g positions (g a divisor of 64)
+    const int box_heads = g % 64 == 0 ? 64 : g, box_s = g % 64 == 0 ? 1 : 64 / g;
+    CUtensorMap qmap;
+    rc = encode_q_map(&qmap, q, batch, s_q, h_q, box_heads, box_s, q_strides);
+    if (rc) return rc;
+    e = launch_decode_pair(map, qmap, p, box_heads, st);
   } else {
     CUtensorMap qmap;
     rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, s_q, q_strides);

@@ -24,6 +24,11 @@ cudaError_t launch_decode_mma16(const CUtensorMap &kv_map, const CUtensorMap &q_
 // The 64-row tcgen05 kernel takes more than 16 rows per latent head.
 bool wide_supported(int R, int g);
 cudaError_t launch_decode_wide(const CUtensorMap &kv_map, const DecodeParams &p, cudaStream_t stream);
+// The CTA-pair tcgen05 kernel takes whole 128-row blocks whose 64-row halves are (position,
+// head) rectangles: g a multiple or a divisor of 64.
+bool pair_supported(int R, int g);
+cudaError_t launch_decode_pair(const CUtensorMap &kv_map, const CUtensorMap &q_map, const DecodeParams &p,
+                               int q_box_heads, cudaStream_t stream);
 cudaError_t launch_decode_tc_narrow(const CUtensorMap &kv_map, const CUtensorMap &q_map,
                                     const DecodeParams &p, cudaStream_t stream);
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,

@@ -30,7 +30,8 @@ MLA_ERR_TIMEOUT = -4
 MLA_FLAG_SKIP_COMBINE = 1
 MLA_FLAG_WARP_MMA = 2
 MLA_FLAG_TCGEN05 = 4
-KERNELS = {"auto": 0, "warp_mma": MLA_FLAG_WARP_MMA, "tcgen05": MLA_FLAG_TCGEN05}
+MLA_FLAG_ONE_SM = 8
+KERNELS = {"auto": 0, "warp_mma": MLA_FLAG_WARP_MMA, "tcgen05": MLA_FLAG_TCGEN05, "one_sm": MLA_FLAG_ONE_SM}
 PAGE = 64
 D_QK = 576
 D_V = 512
@@ -217,8 +218,8 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
 
     Without ``workspace`` a per-(device, stream) scratch buffer is reused; calls that may
     run concurrently on one stream's buffer must pass their own.  ``kernel`` is "auto"
-    (the library's choice by shape), "warp_mma" or "tcgen05" (up to 64 rows per latent
-    head)."""
+    (the library's choice by shape), "warp_mma", "tcgen05" or "one_sm" (the 1-SM 64-row
+    tcgen05 kernel where the CTA-pair kernel would apply)."""
     _require_cuda(q, "q", torch.bfloat16)
     _require_cuda(k_cache, "k_cache", torch.bfloat16)
     _require_cuda(block_table, "block_table", torch.int32)

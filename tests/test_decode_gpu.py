@@ -137,6 +137,37 @@ def test_parity_tcgen05_64_row_tiles(case, num_parts):
     full_parity(x, kernel="tcgen05", num_parts=num_parts)
 
 
+PAIR_CASES = [
+    # (batch, s_q, h_q, h_kv, seqlens, causal): the CTA-pair kernel (whole 128-row blocks)
+    (2, 1, 128, 1, [5000, 33], True),          # one pair, a long split sequence, a one-page piece
+    (3, 1, 128, 1, [64, 65, 191], False),      # exact pages, a lone last page, an odd page count
+    (2, 2, 128, 1, [700, 2], True),            # 256 rows: two pairs; their halves see different key ends
+    (2, 2, 64, 1, [333, 1000], True),          # g = 64: CTA 0 holds position 0, CTA 1 position 1
+    (2, 4, 32, 1, [129, 900], True),           # g = 32: each CTA's rows are 32 heads x 2 positions
+    (2, 8, 16, 1, [77, 640], True),            # g = 16: 16 heads x 4 positions per CTA
+    (3, 1, 128, 2, [700, 65, 3000], True),     # two latent heads
+    (3, 1, 256, 1, [640, 100, 1], False),      # g = 256: two pairs on one position
+    (3, 1, 128, 1, [0, 4000, 0], True),        # empty sequences around a long one
+    (1, 2, 128, 1, [1], True),                 # a causal row with no visible key
+]
+
+
+@pytest.mark.parametrize("case", PAIR_CASES, ids=lambda c: f"b{c[0]}sq{c[1]}h{c[2]}kv{c[3]}")
+@pytest.mark.parametrize("num_parts", [None, 1, 3, 200])
+def test_parity_cta_pair_kernel(case, num_parts):
+    b, s_q, h_q, h_kv, lens, causal = case
+    x = W.make_inputs(W.custom(b, s_q, h_q, h_kv, lens, causal=causal), seed=len(lens) * 7 + h_q + s_q)
+    full_parity(x, num_parts=num_parts)
+
+
+@pytest.mark.parametrize("case", PAIR_CASES[:4], ids=lambda c: f"b{c[0]}sq{c[1]}h{c[2]}kv{c[3]}")
+def test_parity_one_sm_kernel_on_pair_shapes(case):
+    # the 1-SM 64-row kernel stays available (MLA_FLAG_ONE_SM) on the shapes the pair kernel takes
+    b, s_q, h_q, h_kv, lens, causal = case
+    x = W.make_inputs(W.custom(b, s_q, h_q, h_kv, lens, causal=causal), seed=len(lens) * 5 + h_q)
+    full_parity(x, kernel="one_sm")
+
+
 @pytest.mark.parametrize("s_q,h_q,h_kv", [(1, 128, 2), (2, 64, 2), (1, 96, 3)], ids=["R64x2", "R64x2-mtp", "R32x3"])
 def test_parity_tcgen05_several_latent_heads(s_q, h_q, h_kv):
     # the 64-row kernel with more than one latent head: grid z, page rows of head kvh
