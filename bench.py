@@ -57,16 +57,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # nominal B200 figures, reported beside the measured-peak fractions
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 # sources of the decode kernel the library picks for a workload (16 rows or fewer per latent
-# head: the warp-MMA kernel; more: the 64-row tcgen05 kernel); a committed ncu summary stays
-# valid while these are unchanged
+# head: the warp-MMA kernel; whole 128-row blocks with g a multiple or divisor of 64: the
+# CTA-pair tcgen05 kernel; other shapes: the 64-row tcgen05 kernel); a committed ncu summary
+# stays valid while these are unchanged
 KERNEL_SOURCES = {
     "decode_mma16_kernel": ["common.cuh", "decode_mma.cu"],
     "decode_wide_kernel": ["common.cuh", "decode_wide.cu"],
+    "decode_pair_kernel": ["common.cuh", "decode_pair.cu"],
 }
 
 
-def decode_kernel_for(rows_per_kv_head: int) -> str:
-    return "decode_mma16_kernel" if rows_per_kv_head <= 16 else "decode_wide_kernel"
+def decode_kernel_for(rows_per_kv_head: int, g: int = 0) -> str:
+    if rows_per_kv_head <= 16:
+        return "decode_mma16_kernel"
+    if rows_per_kv_head % 128 == 0 and g > 0 and (g % 64 == 0 or 64 % g == 0):
+        return "decode_pair_kernel"
+    return "decode_wide_kernel"
 
 
 # ----------------------------------------------------------------------------------------
@@ -495,7 +501,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     achieved = work / kernel_s
     iso_achieved = work / iso_s
     # the summaries were taken with the library's own kernel choice
-    traffic = recorded_traffic(name, decode_kernel_for(R)) if args.kernel == "auto" else None
+    traffic = recorded_traffic(name, decode_kernel_for(R, w.h_q // w.h_kv)) if args.kernel == "auto" else None
     res = {
         "workload": name, "config": workload_config(w), "unit": unit, "value": value,
         "ms_per_step": per_step * 1e3, "n_rep": n_rep, "per_rep_bytes": per_rep,

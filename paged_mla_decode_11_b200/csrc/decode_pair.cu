@@ -39,15 +39,14 @@
 //
 // Warp roles (both CTAs):
 //   warp 0      producer: own pages into the ring, the partner page's value half after
-//               each score, L2 prefetch two groups ahead; copies complete on the CTA's own
-//               barriers
-//   warp 1      TMEM owner; in CTA 0 the MMA issuer (one thread), in CTA 1 a relay that
-//               forwards its copies' completion to CTA 0's barriers
+//               each score, L2 prefetch two groups ahead; both CTAs' copies complete on CTA
+//               0's barriers (.cta_group::2 loads)
+//   warp 1      TMEM owner; in CTA 0 the MMA issuer (one thread)
 //   warps 2-5   softmax, O rescale and epilogue: thread (lane l of sub-partition q) owns row
 //               l mod 64 and the l / 64 half (keys of the second page; value columns 256-511)
 //   warps 6-9   query loaders: column block 0 into tensor memory, blocks 1-8 by TMA
-// Cross-CTA signals: the MMA issuer's commits are multicast to both CTAs; CTA 1's threads
-// arrive on CTA 0's barriers through their cluster addresses.  Every wait is bounded.
+// Cross-CTA signals: the MMA issuer's commits are multicast to both CTAs; CTA 1's copies and
+// threads arrive on CTA 0's barriers through their cluster addresses.  Every wait is bounded.
 #include "common.cuh"
 #include "launch.h"
 
@@ -109,6 +108,17 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 }
 
 __device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity) { return mbar_test_wait(bar, parity); }
+
+// TMA 3-D load into this CTA's shared memory whose completion (bytes) is counted on an
+// mbarrier of CTA 0, given by its cluster address (.cta_group::2 form).
+__device__ __forceinline__ void tma_load_3d_to_cta0(uint32_t dst, const CUtensorMap *map, uint32_t bar_cluster, int c0,
+                                                    int c1, int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
 
 __device__ __forceinline__ void umma2_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -236,13 +246,6 @@ __device__ __forceinline__ void walker_next(const DecodeParams &p, const PartCur
   if (++w.j == w.ngroups) walker_seek(p, pc, prow0, w, w.seq + 1);
 }
 
-// Number of groups of the part (all pieces).
-__device__ __forceinline__ int part_groups(const DecodeParams &p, const PartCursor &pc, int prow0) {
-  int n = 0;
-  for (int seq = pc.bi; part_has(pc, seq); ++seq) n += pair_piece(p, pc, seq, prow0).ngroups;
-  return n;
-}
-
 // The pair is the cluster's x dimension (grid x = the CTAs of the 128-row blocks, y = parts,
 // z = latent heads): a pair along y was refused at launch ("cluster misconfiguration").
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1)
@@ -271,8 +274,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(T::FULL + i), leader ? 2 : 1);
-      mbar_init(bar(T::VFULL + i), leader ? 2 : 1);
+      mbar_init(bar(T::FULL + i), 1);
+      mbar_init(bar(T::VFULL + i), 1);
       mbar_init(bar(T::EMPTY + i), 1);
       mbar_init(bar(T::SFULL + i), 1);
       mbar_init(bar(T::SFREE + i), 8);
@@ -329,11 +332,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1
           const int phys = walker_page(p, wb, rank == 0 ? pB : pA, lane);
           if (lane == 0) {
             const int st = gb & 1;
-            mbar_arrive_expect_tx(bar(T::VFULL + st), T::kHalfVBytes);
+            if (leader) mbar_arrive_expect_tx(bar(T::VFULL + st), 2 * T::kHalfVBytes);
             // CTA 0 takes the partner's value blocks 0-3 into slots 4-7, CTA 1 blocks 4-7 into slots 0-3
             for (int c = 0; c < 4; ++c)
-              tma_load_3d_hint(slot(st, rank == 0 ? 4 + c : c), &kv_map, bar(T::VFULL + st),
-                               (rank == 0 ? c : 4 + c) * 64, kvh, phys * kPage, policy);
+              tma_load_3d_to_cta0(slot(st, rank == 0 ? 4 + c : c), &kv_map, bar_cta0(T::VFULL + st),
+                                  (rank == 0 ? c : 4 + c) * 64, kvh, phys * kPage, policy);
             last_b[st] = gb;
           }
           walker_next(p, pc, prow0, wb);
@@ -355,10 +358,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1
           }
           if (lane == 0) {
             const int st = ga & 1;
-            mbar_arrive_expect_tx(bar(T::FULL + st), T::kOwnBytes);
+            if (leader) mbar_arrive_expect_tx(bar(T::FULL + st), 2 * T::kOwnBytes);
+            const uint32_t fb = bar_cta0(T::FULL + st);
 #pragma unroll
-            for (int c = 0; c < kColBlocks; ++c)
-              tma_load_3d_hint(slot(st, c), &kv_map, bar(T::FULL + st), c * 64, kvh, phys * kPage, policy);
+            for (int c = 0; c < kColBlocks; ++c) tma_load_3d_to_cta0(slot(st, c), &kv_map, fb, c * 64, kvh, phys * kPage, policy);
             if (pf >= 0) prefetch_l2_bulk(p.kv_base + (int64_t)pf * kPage * p.kv_token_bytes, kPageBytes);
             last_a[st] = ga;
           }
@@ -373,7 +376,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1
       } else {
         // nothing ready: sleep briefly so the polling warp leaves its issue slots to the
         // softmax warp on the same sub-partition
-        __nanosleep(64);
+        __nanosleep(32);
       }
       if (!progressed && (++spins & 15u) == 0) {
         int stop = 0;
@@ -392,9 +395,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1
         ok = __shfl_sync(0xffffffffu, stop, 0) == 0;
       }
     }
-    // every copy issued must land before the CTA exits (its own barriers: in CTA 0 they also
-    // count CTA 1's relayed arrival, which a stalled partner may never send: bounded)
-    if (lane == 0) {
+    // every copy issued must land before the CTAs exit: CTA 0's barriers count both CTAs'
+    // bytes, and CTA 1 leaves only after CTA 0 (final cluster barrier), so CTA 0 waits for all
+    if (lane == 0 && leader) {
       int never = 0;
       for (int st = 0; st < 2; ++st) {
         if (last_a[st] >= 0) mbar_wait(bar(T::FULL + st), (last_a[st] >> 1) & 1, &never, p.status, lim_ns);
@@ -495,42 +498,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1
         }
       }
       umma2_commit_both(bar(T::FINAL));
-    } else if (!leader && lane == 0) {
-      // ------------------------- relay (CTA 1) -------------------------
-      // This CTA's copies complete on its own barriers; forward each completion to CTA 0,
-      // whose MMA thread waits for both CTAs' data.
-      const int total = part_groups(p, pc, prow0);
-      int fg = 0, vgr = 0;
-      bool ok = true;
-      unsigned long long idle_since = 0;
-      uint32_t spins = 0;
-      while (ok && (fg < total || vgr < total)) {
-        bool progressed = false;
-        if (fg < total && mbar_test_wait(bar(T::FULL + (fg & 1)), (fg >> 1) & 1)) {
-          mbar_arrive_cluster(bar_cta0(T::FULL + (fg & 1)));
-          ++fg;
-          progressed = true;
-        }
-        if (vgr < fg && mbar_test_wait(bar(T::VFULL + (vgr & 1)), (vgr >> 1) & 1)) {
-          mbar_arrive_cluster(bar_cta0(T::VFULL + (vgr & 1)));
-          ++vgr;
-          progressed = true;
-        }
-        if (progressed) {
-          idle_since = 0;
-        } else if (__nanosleep(32), (++spins & 15u) == 0) {
-          const unsigned long long now = global_ns();
-          if (*abort) {
-            ok = false;
-          } else if (idle_since == 0) {
-            idle_since = now;
-          } else if (now - idle_since > lim_ns) {
-            *abort = 1;
-            report_timeout(p.status);
-            ok = false;
-          }
-        }
-      }
     }
     __syncwarp();
     // all tensor-core work (issued by CTA 0, writing both CTAs' tensor memory) is complete
@@ -595,13 +562,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(sfree + 8u * b);
         const int key0 = w.t0 + 128 * j + 64 * hf;
-        float mx = -INFINITY;
+        // keys at or past this row's limit get -inf (only partial groups need the test)
+        if (key0 + 64 > lim) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float v = key0 + i < lim ? sv[i] * p.scale_log2 : -INFINITY;
-          sv[i] = v;
-          mx = fmaxf(mx, v);
+          for (int i = 0; i < 64; ++i)
+            if (key0 + i >= lim) sv[i] = -INFINITY;
         }
+        // maximum of the raw scores (scale > 0), four independent chains
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < 64; ++i) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
+        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
         // the row's other half lives on the partner warp: exchange maxima
         xmax[(b * 2 + hf) * 64 + lrow] = mx;
         named_bar_sync(xbar, 64);
@@ -613,14 +584,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Pair128::kThreads, 1
           alpha = fast_exp2(m_used - m_new);
           m_used = m_new;
         }
-        const float base = m_used == -INFINITY ? 0.f : m_used;
-        float sum = 0.f;
+        const float nbase = m_used == -INFINITY ? 0.f : -m_used;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          sv[i] = fast_exp2(sv[i] - base);
-          sum += sv[i];
+          sv[i] = fast_exp2(fmaf(sv[i], p.scale_log2, nbase));
+          s4[i & 3] += sv[i];
         }
-        l = l * alpha + sum;
+        l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
         const bool rescale = __any_sync(0xffffffffu, need && j > 0);
         // O may be rescaled once the previous group's PV has completed (its commit arrives
         // on EMPTY of that group's stage; that barrier is at most one phase behind)

@@ -86,7 +86,13 @@ def test_committed_traffic_is_close_to_the_algorithmic_bytes(bench, workload, lo
 def test_decode_kernel_choice_follows_rows(bench):
     assert bench.decode_kernel_for(16) == "decode_mma16_kernel"
     assert bench.decode_kernel_for(17) == "decode_wide_kernel"
-    assert bench.decode_kernel_for(256) == "decode_wide_kernel"
+    assert bench.decode_kernel_for(256) == "decode_wide_kernel"          # g unknown
+    # whole 128-row blocks whose g is a multiple or divisor of 64: the CTA-pair kernel
+    assert bench.decode_kernel_for(128, 128) == "decode_pair_kernel"
+    assert bench.decode_kernel_for(256, 128) == "decode_pair_kernel"
+    assert bench.decode_kernel_for(128, 32) == "decode_pair_kernel"
+    assert bench.decode_kernel_for(64, 64) == "decode_wide_kernel"      # skewed: one 64-row block
+    assert bench.decode_kernel_for(192, 96) == "decode_wide_kernel"
 
 
 def test_whole_job_aggregate_is_weak_scaling(bench):
