@@ -7,6 +7,9 @@ does, and shares no code with it.
 Contents
   mla_decode / mla_decode_rows   fp64 decode of every (b, s, h), or of listed rows
                                  (plain C, ``mla_oracle.c``; two-pass softmax)
+  mla_decode_fp8 / ..._rows_fp8  the same over an FP8 latent cache (E4M3 codes and one fp32
+                                 scale per token and latent head, dequantised exactly)
+  e4m3_to_float64                OCP E4M3 decoding (the C oracle's, exposed for its pins)
   combine                        log-sum-exp merge of split partials (numpy fp64)
   metadata                       split-KV scheduler specification (``metadata.py``)
 
@@ -56,6 +59,15 @@ def _load():
             i32, f64, i32,
             P, i64, P, P]
         lib.oracle_mla_decode_rows.restype = i32
+        lib.oracle_mla_decode_rows_fp8.argtypes = [
+            P, i64, i64, i64, i32, i32, i32, i32,
+            P, P, i64, i32, i32,
+            P, i64, P, P, P,
+            i32, f64, i32,
+            P, i64, P, P]
+        lib.oracle_mla_decode_rows_fp8.restype = i32
+        lib.oracle_e4m3_to_double.argtypes = [P, i64, P]
+        lib.oracle_e4m3_to_double.restype = i32
         lib.oracle_num_threads.restype = i32
         _lib = lib
     return _lib
@@ -109,6 +121,79 @@ def mla_decode_rows(q, k_cache, block_table, cache_seqlens, rows, dv: int = 512,
         ptr(rows), n, ptr(out), ptr(lse))
     if rc != 0:
         raise ValueError(f"oracle rejected its inputs (status {rc})")
+    return out, lse
+
+
+def e4m3_to_float64(codes) -> np.ndarray:
+    """OCP E4M3 codes (uint8 array) -> float64 values (NaN for 0x7F / 0xFF)."""
+    c = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    out = np.empty(c.shape, dtype=np.float64)
+    if _load().oracle_e4m3_to_double(c.ctypes.data, c.size, out.ctypes.data) != 0:
+        raise ValueError("bad arguments")
+    return out
+
+
+def _u8(t) -> np.ndarray:
+    import torch
+    if isinstance(t, torch.Tensor):
+        t = t.detach().cpu().contiguous()
+        if t.dtype != torch.uint8:
+            t = t.view(torch.uint8)
+        return t.numpy()
+    return np.ascontiguousarray(np.asarray(t, dtype=np.uint8))
+
+
+def mla_decode_rows_fp8(q, k8, k_scale, block_table, cache_seqlens, rows, dv: int = 512,
+                        softmax_scale: Optional[float] = None, causal: bool = True,
+                        kv_begin=None, kv_end=None):
+    """fp64 decode of the listed rows over an FP8 latent cache.
+
+    k8 [num_pages, page, h_kv, d] uint8 E4M3 codes (or a float8_e4m3fn tensor), k_scale
+    [h_kv, num_pages, page] fp32; the latent row of a token is scale * e4m3(code).  Other
+    arguments and the result as in mla_decode_rows.
+    """
+    lib = _load()
+    b, s_q, h_q, d = (int(x) for x in q.shape)
+    num_pages, page, h_kv, d2 = (int(x) for x in k8.shape)
+    if d2 != d:
+        raise ValueError("q and k8 disagree on the latent width")
+    qn = _bf16_bits(q)
+    kn = _u8(k8)
+    import torch
+    ks = k_scale.detach().cpu().contiguous().numpy() if isinstance(k_scale, torch.Tensor) else np.asarray(k_scale)
+    ks = np.ascontiguousarray(ks, dtype=np.float32)
+    if ks.shape != (h_kv, num_pages, page):
+        raise ValueError("k_scale must be [h_kv, num_pages, page]")
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(cache_seqlens, dtype=np.int32))
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    kb = None if kv_begin is None else np.ascontiguousarray(np.asarray(kv_begin, dtype=np.int32))
+    ke = None if kv_end is None else np.ascontiguousarray(np.asarray(kv_end, dtype=np.int32))
+    n = rows.shape[0]
+    out = np.zeros((n, dv), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    scale = d ** -0.5 if softmax_scale is None else float(softmax_scale)
+    ptr = lambda a: None if a is None else a.ctypes.data
+    rc = lib.oracle_mla_decode_rows_fp8(
+        ptr(qn), s_q * h_q * d, h_q * d, d, b, s_q, h_q, d,
+        ptr(kn), ptr(ks), num_pages, page, h_kv,
+        ptr(bt), bt.shape[1], ptr(sl), ptr(kb), ptr(ke),
+        dv, scale, int(bool(causal)),
+        ptr(rows), n, ptr(out), ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its inputs (status {rc})")
+    return out, lse
+
+
+def mla_decode_fp8(q, k8, k_scale, block_table, cache_seqlens, dv: int = 512,
+                   softmax_scale: Optional[float] = None, causal: bool = True,
+                   kv_begin=None, kv_end=None):
+    """fp64 decode of the whole batch over an FP8 latent cache (see mla_decode_rows_fp8)."""
+    b, s_q, h_q, _ = (int(x) for x in q.shape)
+    out, lse = mla_decode_rows_fp8(q, k8, k_scale, block_table, cache_seqlens, all_rows(b, s_q, h_q),
+                                   dv, softmax_scale, causal, kv_begin, kv_end)
+    out = out.reshape(b, s_q, h_q, dv)
+    lse = lse.reshape(b, s_q, h_q).transpose(0, 2, 1).copy()
     return out, lse
 
 

@@ -28,6 +28,15 @@
  *   no keys: out = 0, lse = -inf
  *
  * bf16 inputs are decoded exactly to double.  Build: gcc -O2 -fopenmp -shared -fPIC.
+ *
+ * FP8 latent cache (oracle_mla_decode_rows_fp8).  The Baidu page on Flash MLA ("Flash MLA：
+ * 面向可变长度序列的高效MLA解码内核库解析", section 三.2 and the flow of section 四, step 3)
+ * names FP8 storage of the cache as the precision lever but gives no format.  Reading taken
+ * here: every token's latent row is stored as 576 OCP E4M3 ("e4m3fn") codes with one fp32
+ * scale per token and latent head, and the row the decode uses is the dequantised
+ *   c_j[t] = scale_j * e4m3(code_j[t]);
+ * the decode itself is the definition above applied to these rows.  k8 is [num_pages, page,
+ * h_kv, d] uint8, k_scale is [h_kv, num_pages, page] fp32.
  */
 #include <math.h>
 #include <stdint.h>
@@ -44,6 +53,24 @@ static double bf16_bits_to_double(uint16_t h) {
     return (double)f;
 }
 
+/* OCP 8-bit floating point E4M3 ("e4m3fn"): sign bit 7, exponent bits 6..3 (bias 7),
+ * mantissa bits 2..0; exponent 0 holds subnormals (m / 8) * 2^-6; exponent 15 with
+ * mantissa 7 is NaN; there is no infinity (the largest finite value is 448). */
+static double e4m3_to_double(uint8_t v) {
+    const int sgn = v >> 7, e = (v >> 3) & 15, m = v & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m / 8.0, -6);
+    else mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sgn ? -mag : mag;
+}
+
+int oracle_e4m3_to_double(const uint8_t *codes, int64_t n, double *out) {
+    if (!codes || !out || n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_double(codes[i]);
+    return 0;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
@@ -52,25 +79,52 @@ int oracle_num_threads(void) {
 #endif
 }
 
-/*
- * rows: n_rows triples (b, s, h).  out_rows: [n_rows, dv] doubles, lse_rows: [n_rows].
- * q strides are in elements (innermost stride 1).  k_cache is [num_pages, page, h_kv, d]
- * contiguous.  block_table row stride is bt_stride elements.
- * Returns 0, or -1 on an argument error, -2 on allocation failure, -3 when a block-table
- * entry addressed by a key is out of range.
- */
-int oracle_mla_decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs_h,
-                           int batch, int s_q, int h_q, int d,
-                           const uint16_t *k_cache, int64_t num_pages, int page, int h_kv,
-                           const int32_t *block_table, int64_t bt_stride,
-                           const int32_t *cache_seqlens,
-                           const int32_t *kv_begin, const int32_t *kv_end,
-                           int dv, double scale, int causal,
-                           const int32_t *rows, int64_t n_rows,
-                           double *out_rows, double *lse_rows) {
-    if (!q || !k_cache || !block_table || !cache_seqlens || !rows || !out_rows || !lse_rows)
-        return -1;
-    if (h_kv <= 0 || h_q % h_kv != 0 || dv > d || page <= 0 || batch <= 0 || s_q <= 0)
+/* The latent row of (page phys, slot, latent head kvh) as doubles: bf16 codes, or E4M3 codes
+ * times the token's scale. */
+typedef struct {
+    const uint16_t *bf16;  /* [num_pages, page, h_kv, d] or NULL */
+    const uint8_t *e4m3;   /* [num_pages, page, h_kv, d] or NULL */
+    const float *scale;    /* [h_kv, num_pages, page] with e4m3 */
+    int64_t num_pages;
+    int page, h_kv, d;
+} cache_t;
+
+/* q_row . c over all d columns of the latent row of (page phys, slot, latent head kvh). */
+static double row_dot(const cache_t *c, int64_t phys, int slot, int kvh, const uint16_t *q_row) {
+    const int64_t row = ((phys * c->page + slot) * c->h_kv + kvh) * (int64_t)c->d;
+    double acc = 0.0;
+    if (c->bf16) {
+        for (int t = 0; t < c->d; ++t) acc += bf16_bits_to_double(q_row[t]) * bf16_bits_to_double(c->bf16[row + t]);
+    } else {
+        const double sc = (double)c->scale[((int64_t)kvh * c->num_pages + phys) * c->page + slot];
+        for (int t = 0; t < c->d; ++t) acc += bf16_bits_to_double(q_row[t]) * (sc * e4m3_to_double(c->e4m3[row + t]));
+    }
+    return acc;
+}
+
+/* o[0:dv] += p * c[0:dv] for the same latent row. */
+static void row_axpy(const cache_t *c, int64_t phys, int slot, int kvh, double p, double *o, int dv) {
+    const int64_t row = ((phys * c->page + slot) * c->h_kv + kvh) * (int64_t)c->d;
+    if (c->bf16) {
+        for (int t = 0; t < dv; ++t) o[t] += p * bf16_bits_to_double(c->bf16[row + t]);
+    } else {
+        const double sc = (double)c->scale[((int64_t)kvh * c->num_pages + phys) * c->page + slot];
+        for (int t = 0; t < dv; ++t) o[t] += p * (sc * e4m3_to_double(c->e4m3[row + t]));
+    }
+}
+
+static int decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs_h,
+                       int batch, int s_q, int h_q, int d, const cache_t *cache,
+                       const int32_t *block_table, int64_t bt_stride,
+                       const int32_t *cache_seqlens,
+                       const int32_t *kv_begin, const int32_t *kv_end,
+                       int dv, double scale, int causal,
+                       const int32_t *rows, int64_t n_rows,
+                       double *out_rows, double *lse_rows) {
+    const int64_t num_pages = cache->num_pages;
+    const int page = cache->page, h_kv = cache->h_kv;
+    if (!q || !block_table || !cache_seqlens || !rows || !out_rows || !lse_rows) return -1;
+    if (cache->d != d || h_kv <= 0 || h_q % h_kv != 0 || dv > d || page <= 0 || batch <= 0 || s_q <= 0)
         return -1;
     const int g = h_q / h_kv;
     int status = 0;
@@ -119,9 +173,7 @@ int oracle_mla_decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_
             for (int64_t j = lo; j < hi; ++j) {
                 const int64_t phys = block_table[b * bt_stride + j / page];
                 if (phys < 0 || phys >= num_pages) { bad = 1; break; }
-                const uint16_t *c = k_cache + ((phys * page + j % page) * h_kv + kvh) * (int64_t)d;
-                double acc = 0.0;
-                for (int t = 0; t < d; ++t) acc += bf16_bits_to_double(qrow[t]) * bf16_bits_to_double(c[t]);
+                const double acc = row_dot(cache, phys, (int)(j % page), kvh, qrow);
                 x[j - lo] = scale * acc;
                 if (x[j - lo] > M) M = x[j - lo];
             }
@@ -136,13 +188,50 @@ int oracle_mla_decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_
             for (int64_t j = lo; j < hi; ++j) Z += exp(x[j - lo] - M);
             for (int64_t j = lo; j < hi; ++j) {
                 const int64_t phys = block_table[b * bt_stride + j / page];
-                const uint16_t *c = k_cache + ((phys * page + j % page) * h_kv + kvh) * (int64_t)d;
                 const double p = exp(x[j - lo] - M) / Z;
-                for (int t = 0; t < dv; ++t) o[t] += p * bf16_bits_to_double(c[t]);
+                row_axpy(cache, phys, (int)(j % page), kvh, p, o, dv);
             }
             lse_rows[r] = M + log(Z);
         }
         free(x);
     }
     return status;
+}
+
+/*
+ * rows: n_rows triples (b, s, h).  out_rows: [n_rows, dv] doubles, lse_rows: [n_rows].
+ * q strides are in elements (innermost stride 1).  k_cache is [num_pages, page, h_kv, d]
+ * contiguous.  block_table row stride is bt_stride elements.
+ * Returns 0, or -1 on an argument error, -2 on allocation failure, -3 when a block-table
+ * entry addressed by a key is out of range.
+ */
+int oracle_mla_decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs_h,
+                           int batch, int s_q, int h_q, int d,
+                           const uint16_t *k_cache, int64_t num_pages, int page, int h_kv,
+                           const int32_t *block_table, int64_t bt_stride,
+                           const int32_t *cache_seqlens,
+                           const int32_t *kv_begin, const int32_t *kv_end,
+                           int dv, double scale, int causal,
+                           const int32_t *rows, int64_t n_rows,
+                           double *out_rows, double *lse_rows) {
+    if (!k_cache) return -1;
+    cache_t c = {k_cache, NULL, NULL, num_pages, page, h_kv, d};
+    return decode_rows(q, qs_b, qs_s, qs_h, batch, s_q, h_q, d, &c, block_table, bt_stride, cache_seqlens,
+                       kv_begin, kv_end, dv, scale, causal, rows, n_rows, out_rows, lse_rows);
+}
+
+/* The same decode over an FP8 (E4M3 + per-token fp32 scale) latent cache. */
+int oracle_mla_decode_rows_fp8(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs_h,
+                               int batch, int s_q, int h_q, int d,
+                               const uint8_t *k8, const float *k_scale, int64_t num_pages, int page, int h_kv,
+                               const int32_t *block_table, int64_t bt_stride,
+                               const int32_t *cache_seqlens,
+                               const int32_t *kv_begin, const int32_t *kv_end,
+                               int dv, double scale, int causal,
+                               const int32_t *rows, int64_t n_rows,
+                               double *out_rows, double *lse_rows) {
+    if (!k8 || !k_scale) return -1;
+    cache_t c = {NULL, k8, k_scale, num_pages, page, h_kv, d};
+    return decode_rows(q, qs_b, qs_s, qs_h, batch, s_q, h_q, d, &c, block_table, bt_stride, cache_seqlens,
+                       kv_begin, kv_end, dv, scale, causal, rows, n_rows, out_rows, lse_rows);
 }

@@ -160,6 +160,31 @@ def make_inputs(w: Workload, seed: int = 0, max_pages: Optional[int] = None) -> 
                 causal=w.causal, softmax_scale=w.scale, dv=D_V)
 
 
+E4M3_MAX = 448.0  # largest finite OCP E4M3 value
+
+
+def to_fp8_cache(k_cache: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """Store a bf16 latent cache in the FP8 format (the cache writer's side, not the decode
+    path): one fp32 scale per token and latent head, amax(|row|) / 448 (1 for an all-zero
+    row), and the row divided by it rounded to OCP E4M3 by torch's float8_e4m3fn conversion.
+
+    Returns (k8 [num_pages, page, h_kv, d] uint8 codes, k_scale [h_kv, num_pages, page] fp32).
+    """
+    rows = k_cache.float()
+    amax = rows.abs().amax(dim=-1)                                    # [pages, page, h_kv]
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    k8 = (rows / scale[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return k8.contiguous(), scale.permute(2, 0, 1).contiguous()
+
+
+def make_inputs_fp8(w: Workload, seed: int = 0, max_pages: Optional[int] = None) -> dict:
+    """make_inputs, with the latent cache stored in the FP8 format (to_fp8_cache): adds
+    k8 and k_scale; k_cache stays the bf16 source the codes were made from."""
+    x = make_inputs(w, seed, max_pages)
+    x["k8"], x["k_scale"] = to_fp8_cache(x["k_cache"])
+    return x
+
+
 def custom(batch: int, s_q: int, h_q: int, h_kv: int, seqlens: Sequence[int],
            causal: bool = True, scale: Optional[float] = None, outlier_frac: float = 0.0,
            name: str = "custom") -> Workload:
@@ -169,18 +194,21 @@ def custom(batch: int, s_q: int, h_q: int, h_kv: int, seqlens: Sequence[int],
 
 
 def algorithmic_work(seqlens: Sequence[int], s_q: int, h_q: int, h_kv: int, causal: bool,
-                     d: int = D_QK, dv: int = D_V, batch_meta: bool = True) -> tuple[int, int]:
+                     d: int = D_QK, dv: int = D_V, batch_meta: bool = True,
+                     token_bytes: Optional[int] = None) -> tuple[int, int]:
     """Algorithmic (bytes, flops) of one decode call.
 
-    Bytes: every valid token's latent row (h_kv heads x d bf16) read once, q read once,
-    out (bf16) and lse (fp32) written once, plus cache_seqlens and the block-table rows
-    actually addressed.  Flops: 2 * (d + dv) per (query row, unmasked key).
+    Bytes: every valid token's latent row (h_kv heads x d bf16, or token_bytes per token
+    and latent head for another cache format) read once, q read once, out (bf16) and lse
+    (fp32) written once, plus cache_seqlens and the block-table rows actually addressed.
+    Flops: 2 * (d + dv) per (query row, unmasked key).
     """
+    per_token = d * 2 if token_bytes is None else int(token_bytes)
     nbytes = 0
     flops = 0
     for L in seqlens:
         L = int(L)
-        nbytes += L * h_kv * d * 2
+        nbytes += L * h_kv * per_token
         nbytes += s_q * h_q * d * 2 + s_q * h_q * dv * 2 + s_q * h_q * 4
         if batch_meta:
             nbytes += 4 + ((L + PAGE - 1) // PAGE) * 4
