@@ -190,6 +190,30 @@ MLA_API int mla_decode_paged(const void *q, const int64_t q_strides[3], int batc
                      size_t workspace_bytes, unsigned flags, mla_stream_t stream);
 
 /*
+ * mla_decode_paged_fp8 -- mla_decode_paged over an FP8 latent cache, for up to 16 query rows
+ * per latent head (s_q * h_q / h_kv <= 16: the memory-bound decode shape; the cache bytes
+ * halve).  The Baidu page on Flash MLA ("Flash MLA：面向可变长度序列的高效MLA解码内核库解析",
+ * section 三.2 and section 四, step 3) names FP8 storage of the cache without a format; this
+ * library's format:
+ *   k8        device uint8 [num_pages][page_size][h_kv][d]: every token's latent row as OCP
+ *             E4M3 ("e4m3fn") codes, contiguous, 16-byte aligned
+ *   k_scale   device fp32 [h_kv][num_pages][page_size]: one scale per token and latent head,
+ *             contiguous, 16-byte aligned
+ * and the latent row a token contributes (to the score and, first dv columns, to the
+ * value) is k_scale * e4m3(k8).  Codes are widened to bf16 exactly in the kernel; all other
+ * arguments, layouts, results and errors as in mla_decode_paged (flags: 0 or
+ * MLA_FLAG_SKIP_COMBINE; the same workspace size and the same mla_combine).  Errors also:
+ * MLA_ERR_UNSUPPORTED for more than 16 rows per latent head.
+ */
+MLA_API int mla_decode_paged_fp8(const void *q, const int64_t q_strides[3], int batch, int s_q, int h_q,
+                                 int d, const void *k8, const float *k_scale, int64_t num_pages,
+                                 int page_size, int h_kv, const int32_t *block_table,
+                                 int64_t block_table_stride, const int32_t *cache_seqlens, int dv,
+                                 const int32_t *tile_metadata, int num_parts, const int32_t *num_splits,
+                                 float softmax_scale, int causal, void *out, float *lse, void *workspace,
+                                 size_t workspace_bytes, unsigned flags, mla_stream_t stream);
+
+/*
  * mla_combine -- log-sum-exp merge of split-KV partials: for every sequence with more
  * than one split and every query row, lse = ln sum_k exp(lse_k) and
  * out = sum_k exp(lse_k - lse) * o_k (partials with lse_k = -inf weigh nothing).

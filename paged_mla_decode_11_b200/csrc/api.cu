@@ -120,6 +120,39 @@ int encode_q_map(CUtensorMap *map, const void *q, int batch, int s_q, int h_q, i
   return MLA_OK;
 }
 
+// FP8 latent cache codes [num_pages * 64 tokens][h_kv][576] bytes as a 3-D map (columns, latent
+// head, token); one box = 128 columns (128 bytes, 128-byte swizzle) x 1 head x 32 tokens.  A box
+// at column 512 reaches past column 575; TMA fills those columns with zeros.
+int encode_k8_map(CUtensorMap *map, const void *k8, int64_t num_pages, int h_kv) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(h_kv), cuuint64_t(num_pages) * kPage};
+  cuuint64_t strides[2] = {cuuint64_t(kD), cuuint64_t(h_kv) * kD};
+  cuuint32_t box[3] = {128, 1, 32};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(k8), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled (fp8 cache) failed (%d)", int(r));
+  return MLA_OK;
+}
+
+// Token scales [h_kv][num_pages][64] fp32 as a 3-D map (slot, page, latent head); one box =
+// the 32 scales of a 32-token chunk.
+int encode_scale_map(CUtensorMap *map, const float *k_scale, int64_t num_pages, int h_kv) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+  cuuint64_t dims[3] = {cuuint64_t(kPage), cuuint64_t(num_pages), cuuint64_t(h_kv)};
+  cuuint64_t strides[2] = {cuuint64_t(kPage) * 4, cuuint64_t(num_pages) * kPage * 4};
+  cuuint32_t box[3] = {32, 1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(k_scale), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled (fp8 scales) failed (%d)", int(r));
+  return MLA_OK;
+}
+
 int check_common(int batch, int s_q, int h_q, int h_kv, int dv) {
   if (batch < 1 || s_q < 1 || h_q < 1 || h_kv < 1)
     return fail(MLA_ERR_ARG, "batch, s_q, h_q and h_kv must be >= 1");
@@ -323,6 +356,88 @@ int mla_decode_paged(const void *q, const int64_t q_strides[3], int batch, int s
     e = kind == kTc ? launch_decode_tc_narrow(map, qmap, p, st) : launch_decode_mma16(map, qmap, p, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  if (!(flags & MLA_FLAG_SKIP_COMBINE)) {
+    e = launch_combine(num_splits, batch, s_q, h_q, h_kv, p.lse_accum, p.o_accum, p.out, lse, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+  }
+  return MLA_OK;
+}
+
+int mla_decode_paged_fp8(const void *q, const int64_t q_strides[3], int batch, int s_q, int h_q, int d,
+                         const void *k8, const float *k_scale, int64_t num_pages, int page_size, int h_kv,
+                         const int32_t *block_table, int64_t block_table_stride, const int32_t *cache_seqlens,
+                         int dv, const int32_t *tile_metadata, int num_parts, const int32_t *num_splits,
+                         float softmax_scale, int causal, void *out, float *lse, void *workspace,
+                         size_t workspace_bytes, unsigned flags, mla_stream_t stream) {
+  if (!q || !q_strides || !k8 || !k_scale || !block_table || !cache_seqlens || !tile_metadata || !num_splits ||
+      !out || !lse)
+    return fail(MLA_ERR_ARG, "null pointer argument");
+  int rc = check_common(batch, s_q, h_q, h_kv, dv);
+  if (rc) return rc;
+  if (d != kD) return fail(MLA_ERR_UNSUPPORTED, "d must be %d (got %d)", kD, d);
+  if (page_size != kPage) return fail(MLA_ERR_UNSUPPORTED, "page_size must be %d (got %d)", kPage, page_size);
+  const int g = h_q / h_kv, R = s_q * g;
+  if (R > 16)
+    return fail(MLA_ERR_UNSUPPORTED,
+                "the FP8 cache is decoded by the 16-row kernel: s_q * h_q / h_kv must be <= 16 (got %d)", R);
+  if (num_pages < 1 || num_pages > (int64_t(1) << 25))
+    return fail(MLA_ERR_ARG, "num_pages must be in [1, 2^25]");
+  if (block_table_stride < 1) return fail(MLA_ERR_ARG, "block_table_stride must be >= 1");
+  if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(MLA_ERR_ARG, "softmax_scale must be positive and finite");
+  if (flags & ~MLA_FLAG_SKIP_COMBINE) return fail(MLA_ERR_ARG, "unknown flags 0x%x", flags);
+  for (int i = 0; i < 3; ++i)
+    if (q_strides[i] < 0 || q_strides[i] % 8 != 0)
+      return fail(MLA_ERR_ARG, "q strides must be non-negative multiples of 8 elements");
+  if (!aligned(q, 16) || !aligned(k8, 16) || !aligned(k_scale, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return fail(MLA_ERR_ARG, "q, k8, k_scale and out must be 16-byte aligned, lse 4-byte aligned");
+  rc = check_device();
+  if (rc) return rc;
+  const WorkspaceLayout wl = workspace_layout(batch, R, h_kv, num_parts);
+  if (!workspace) return fail(MLA_ERR_WORKSPACE, "workspace is null");
+  if (!aligned(workspace, 256)) return fail(MLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (workspace_bytes < wl.total)
+    return fail(MLA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, wl.total);
+
+  CUtensorMap k8_map, scale_map, qmap;
+  rc = encode_k8_map(&k8_map, k8, num_pages, h_kv);
+  if (rc) return rc;
+  rc = encode_scale_map(&scale_map, k_scale, num_pages, h_kv);
+  if (rc) return rc;
+  rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, s_q, q_strides);
+  if (rc) return rc;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.q_sb = q_strides[0];
+  p.q_ss = q_strides[1];
+  p.q_sh = q_strides[2];
+  p.batch = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.g = g;
+  p.R = R;
+  p.block_table = block_table;
+  p.bt_stride = block_table_stride;
+  p.kv_base = static_cast<const uint8_t *>(k8);
+  p.kv_token_bytes = int64_t(h_kv) * kD;
+  p.seqlens = cache_seqlens;
+  p.tile_md = tile_metadata;
+  p.num_parts = num_parts;
+  p.num_splits = num_splits;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.lse_accum = reinterpret_cast<float *>(ws + wl.lse_off);
+  p.o_accum = reinterpret_cast<float *>(ws + wl.o_off);
+  p.status = reinterpret_cast<int *>(ws);
+  p.watchdog_ns = kWatchdogNs;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_decode_fp8(k8_map, scale_map, qmap, p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "fp8 decode kernel launch");
   if (!(flags & MLA_FLAG_SKIP_COMBINE)) {
     e = launch_combine(num_splits, batch, s_q, h_q, h_kv, p.lse_accum, p.o_accum, p.out, lse, st);
     if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");

@@ -31,6 +31,8 @@ cudaError_t launch_decode_pair(const CUtensorMap &kv_map, const CUtensorMap &q_m
                                int q_box_heads, cudaStream_t stream);
 cudaError_t launch_decode_tc_narrow(const CUtensorMap &kv_map, const CUtensorMap &q_map,
                                     const DecodeParams &p, cudaStream_t stream);
+cudaError_t launch_decode_fp8(const CUtensorMap &k8_map, const CUtensorMap &scale_map, const CUtensorMap &q_map,
+                              const DecodeParams &p, cudaStream_t stream);
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,
                            const float *lse_accum, const float *o_accum, __nv_bfloat16 *out,
                            float *lse, cudaStream_t stream);

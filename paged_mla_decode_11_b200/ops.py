@@ -40,7 +40,7 @@ TILE_FIELDS = 8
 EXPORTED = (
     "mla_device_sm_count", "mla_num_parts", "mla_metadata_size", "mla_get_metadata", "mla_workspace_size",
     "mla_decode_paged", "mla_combine", "mla_query_status", "mla_watchdog_selftest",
-    "mla_last_error_string", "mla_decode_paged_static", "mla_query_status_static",
+    "mla_last_error_string", "mla_decode_paged_static", "mla_query_status_static", "mla_decode_paged_fp8",
 )
 
 _lib = None
@@ -79,6 +79,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "mla_query_status": [P, P],
             "mla_watchdog_selftest": [P, U64, P],
             "mla_query_status_static": [P],
+            "mla_decode_paged_fp8": [P, P, I, I, I, I, P, P, I64, I, I, P, I64, P, I, P, I, P,
+                                     ctypes.c_float, I, P, P, P, ctypes.c_size_t, ctypes.c_uint, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -276,6 +278,68 @@ def mla_decode_paged(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.
 
 # The pages' name for the decode call.
 flash_mla_with_kvcache = mla_decode_paged
+
+
+def mla_decode_paged_fp8(q: torch.Tensor, k8: torch.Tensor, k_scale: torch.Tensor, block_table: torch.Tensor,
+                         cache_seqlens: torch.Tensor, dv: int, tile_metadata: torch.Tensor,
+                         num_splits: torch.Tensor, softmax_scale: Optional[float] = None,
+                         causal: bool = False, workspace: Optional[torch.Tensor] = None,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                         skip_combine: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Paged MLA decode over an FP8 latent cache: k8 [pages, 64, h_kv, 576] uint8 E4M3 codes
+    (or float8_e4m3fn), k_scale [h_kv, pages, 64] fp32, one scale per token and latent head;
+    up to 16 query rows per latent head.  Other arguments and results as mla_decode_paged."""
+    _require_cuda(q, "q", torch.bfloat16)
+    if k8.dtype == torch.float8_e4m3fn:
+        k8 = k8.view(torch.uint8)
+    _require_cuda(k8, "k8", torch.uint8)
+    _require_cuda(k_scale, "k_scale", torch.float32)
+    _require_cuda(block_table, "block_table", torch.int32)
+    _require_cuda(cache_seqlens, "cache_seqlens", torch.int32)
+    _require_cuda(tile_metadata, "tile_metadata", torch.int32)
+    _require_cuda(num_splits, "num_splits", torch.int32)
+    if q.dim() != 4 or k8.dim() != 4 or block_table.dim() != 2:
+        raise ValueError("q and k8 must be 4-D, block_table 2-D")
+    b, s_q, h_q, d = q.shape
+    num_pages, page, h_kv, d2 = k8.shape
+    if d2 != d:
+        raise ValueError("q and k8 disagree on the latent width")
+    if q.stride(3) != 1:
+        raise ValueError("q's last dimension must be contiguous")
+    if not k8.is_contiguous():
+        raise ValueError("k8 must be contiguous")
+    if k_scale.shape != (h_kv, num_pages, page) or not k_scale.is_contiguous():
+        raise ValueError("k_scale must be a contiguous [h_kv, num_pages, page] tensor")
+    if block_table.stride(1) != 1 or block_table.shape[0] != b:
+        raise ValueError("block_table must be [batch, max_pages] with contiguous rows")
+    if cache_seqlens.shape != (b,) or not cache_seqlens.is_contiguous():
+        raise ValueError("cache_seqlens must be a contiguous [batch] tensor")
+    tshape = tile_metadata.shape
+    if len(tshape) != 2 or tshape[1] != TILE_FIELDS or not tile_metadata.is_contiguous():
+        raise ValueError("tile_metadata must be a contiguous [num_parts, 8] tensor")
+    if num_splits.shape != (b + 1,):
+        raise ValueError("num_splits must be [batch + 1]")
+    dev = q.device
+    num_parts = tshape[0]
+    scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty(b, s_q, h_q, dv, dtype=torch.bfloat16, device=dev)
+    elif out.shape != (b, s_q, h_q, dv) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [b, s_q, h_q, dv] tensor")
+    if lse is None:
+        lse = torch.empty(b, h_q, s_q, dtype=torch.float32, device=dev)
+    elif lse.shape != (b, h_q, s_q) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [b, h_q, s_q] tensor")
+    if workspace is None:
+        workspace = _default_workspace(workspace_size(b, s_q, h_q, h_kv, num_parts), dev)
+    qst = q.stride()
+    _check(load_library().mla_decode_paged_fp8(
+        q.data_ptr(), _I64x3(qst[0], qst[1], qst[2]), b, s_q, h_q, d, k8.data_ptr(), k_scale.data_ptr(),
+        num_pages, page, h_kv, block_table.data_ptr(), block_table.stride(0), cache_seqlens.data_ptr(), dv,
+        tile_metadata.data_ptr(), num_parts, num_splits.data_ptr(), scale, int(bool(causal)), out.data_ptr(),
+        lse.data_ptr(), workspace.data_ptr(), workspace.numel(), MLA_FLAG_SKIP_COMBINE if skip_combine else 0,
+        _stream_ptr(dev)))
+    return out, lse
 
 
 def mla_combine(num_splits: torch.Tensor, s_q: int, h_q: int, h_kv: int, num_parts: int,
