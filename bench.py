@@ -213,13 +213,28 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def workload_work(x, w):
+# Workloads with the latent cache in the FP8 format (E4M3 codes + one fp32 scale per token and
+# latent head), decoded by mla_decode_paged_fp8; the name maps to the bf16 workload it stores.
+FP8_WORKLOADS = {"memory_bound_fp8": "memory_bound"}
+FP8_TOKEN_BYTES = 576 + 4
+
+
+def workload_spec(name):
+    """(Workload, is_fp8) of a bench workload name."""
+    if name in FP8_WORKLOADS:
+        return W.WORKLOADS[FP8_WORKLOADS[name]], True
+    return W.WORKLOADS[name], False
+
+
+def workload_work(x, w, fp8=False):
     lens = x["cache_seqlens"].tolist()
-    nbytes, flops = W.algorithmic_work(lens, w.s_q, w.h_q, w.h_kv, w.causal)
+    nbytes, flops = W.algorithmic_work(lens, w.s_q, w.h_q, w.h_kv, w.causal,
+                                       token_bytes=FP8_TOKEN_BYTES if fp8 else None)
     return nbytes, flops
 
 
 def metric_of(w_name):
+    w_name = FP8_WORKLOADS.get(w_name, w_name)
     if w_name in ("compute_bound", "causal_mtp"):
         return "TFLOP/s", "tensor"
     return "GB/s", "hbm"
@@ -228,12 +243,13 @@ def metric_of(w_name):
 METRIC = "paged MLA decode on 1 B200: HBM GB/s (mem-bound), TFLOPS (compute-bound)"
 
 
-def workload_config(w):
+def workload_config(w, fp8=False):
     lens = w.seqlens
-    return {"workload": f"{w.name}: batch={w.batch}, s_q={w.s_q}, h_q={w.h_q}, h_kv={w.h_kv}, "
-                        f"d=576, dv=512, page 64, seqlens {lens}, causal={w.causal}, "
-                        f"scale={w.scale:.6g}, bf16 q/cache ~N(0,1), random block_table over one pool, "
-                        "seed 0"}
+    cache = ("FP8 cache (E4M3 codes of the bf16 ~N(0,1) pool, one fp32 scale per token)" if fp8
+             else "bf16 q/cache ~N(0,1)")
+    return {"workload": f"{w.name}{' fp8' if fp8 else ''}: batch={w.batch}, s_q={w.s_q}, h_q={w.h_q}, "
+                        f"h_kv={w.h_kv}, d=576, dv=512, page 64, seqlens {lens}, causal={w.causal}, "
+                        f"scale={w.scale:.6g}, {cache}, random block_table over one pool, seed 0"}
 
 
 # ----------------------------------------------------------------------------------------
@@ -244,12 +260,17 @@ def oracle_sample(x, w, seqs):
     import oracle
     rows = [(b, s, h) for b in seqs for s in range(w.s_q) for h in range(w.h_q)]
     rows = np.array(rows, dtype=np.int32)
+    fp8 = "k8" in x
     t0 = time.perf_counter()
-    oracle.mla_decode_rows(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], rows, dv=512,
-                           softmax_scale=w.scale, causal=w.causal)
+    if fp8:
+        oracle.mla_decode_rows_fp8(x["q"], x["k8"], x["k_scale"], x["block_table"], x["cache_seqlens"], rows,
+                                   dv=512, softmax_scale=w.scale, causal=w.causal)
+    else:
+        oracle.mla_decode_rows(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], rows, dv=512,
+                               softmax_scale=w.scale, causal=w.causal)
     dt = time.perf_counter() - t0
     lens = [int(x["cache_seqlens"][b]) for b in seqs]
-    nb, fl = W.algorithmic_work(lens, w.s_q, w.h_q, w.h_kv, w.causal)
+    nb, fl = W.algorithmic_work(lens, w.s_q, w.h_q, w.h_kv, w.causal, token_bytes=FP8_TOKEN_BYTES if fp8 else None)
     return dt, nb, fl
 
 
@@ -290,8 +311,8 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle
-    w = W.WORKLOADS[args.workload]
-    x = W.make_inputs(w, seed=0)
+    w, fp8 = workload_spec(args.workload)
+    x = W.make_inputs_fp8(w, seed=0) if fp8 else W.make_inputs(w, seed=0)
     unit, _ = metric_of(args.workload)
     budget = 90.0 / max(args.steps + args.warmup, 1)
     per_step = min(2.0, max(0.05, budget))
@@ -331,7 +352,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w),
+        "data": "synthetic", "config": workload_config(w, fp8),
         "cpu_baseline": {"value": val, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -355,12 +376,17 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     the CPU oracle's throughput on a bounded sample.  Returns a dict of results."""
     from paged_mla_decode_11_b200 import ops
     barrier, max_over_ranks = group.barrier, group.max
-    w = W.WORKLOADS[name]
+    w, fp8 = workload_spec(name)
     R = w.rows_per_kv_head
-    x = W.make_inputs(w, seed=args.seed + rank)
-    nbytes, flops = workload_work(x, w)
+    if fp8:
+        x = W.make_inputs_fp8(w, seed=args.seed + rank)
+        del x["k_cache"]  # the bf16 source of the codes stays on the host
+        per_rep = x["k8"].numel() + x["k_scale"].numel() * 4
+    else:
+        x = W.make_inputs(w, seed=args.seed + rank)
+        per_rep = x["k_cache"].numel() * 2
+    nbytes, flops = workload_work(x, w, fp8)
     unit, bound = metric_of(name)
-    per_rep = x["k_cache"].numel() * 2
     n_rep = max(2, math.ceil(1.5 * L2_BYTES / per_rep) + 1)
 
     reps = []
@@ -375,6 +401,11 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
         reps.append(d)
 
     def decode(d, tile, splits, kernel_only=False):
+        if fp8:
+            ops.mla_decode_paged_fp8(d["q"], d["k8"], d["k_scale"], d["block_table"], d["cache_seqlens"], 512, tile,
+                                     splits, softmax_scale=w.scale, causal=w.causal, workspace=d["ws"],
+                                     out=d["out"], lse=d["lse"], skip_combine=kernel_only)
+            return
         ops.mla_decode_paged(d["q"], d["k_cache"], d["block_table"], d["cache_seqlens"], 512, tile,
                              splits, softmax_scale=w.scale, causal=w.causal, workspace=d["ws"],
                              out=d["out"], lse=d["lse"], skip_combine=kernel_only, kernel=args.kernel)
@@ -503,7 +534,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     # the summaries were taken with the library's own kernel choice
     traffic = recorded_traffic(name, decode_kernel_for(R, w.h_q // w.h_kv)) if args.kernel == "auto" else None
     res = {
-        "workload": name, "config": workload_config(w), "unit": unit, "value": value,
+        "workload": name, "config": workload_config(w, fp8), "unit": unit, "value": value,
         "ms_per_step": per_step * 1e3, "n_rep": n_rep, "per_rep_bytes": per_rep,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
                      "frac": achieved / peak, "traffic": traffic,
@@ -516,7 +547,9 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
                                          f"each after a {FLUSH_BYTES >> 20} MB L2-flush write"),
                      "frac_of_nominal": achieved / nominal, "nominal_peak": nominal,
                      "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
-                     "whole_page_bytes_per_launch": W.whole_page_bytes(x["cache_seqlens"].tolist(), w.h_kv),
+                     "whole_page_bytes_per_launch": (W.whole_page_bytes(x["cache_seqlens"].tolist(), w.h_kv) *
+                                                     FP8_TOKEN_BYTES // (2 * 576) if fp8 else
+                                                     W.whole_page_bytes(x["cache_seqlens"].tolist(), w.h_kv)),
                      "scheduler_ms": sched_s * 1e3, "scheduler_isolated_ms": iso_sched_s * 1e3,
                      "combine_ms": combine_s * 1e3},
         "clocks": clocks,
@@ -524,7 +557,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
 
     if with_e2e:
         res["e2e"] = e2e_leg(args, w, x, reps[0], dev, nparts, R, unit, total_bytes, total_flops,
-                             barrier, max_over_ranks)
+                             barrier, max_over_ranks, fp8)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and cpu_seconds > 0:
         res["cpu_baseline"] = cpu_baseline(x, w, unit, seconds=cpu_seconds)
     for g in (warm_graph, graph, kgraph, mgraph, cgraph):
@@ -534,7 +567,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     return res
 
 
-def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barrier, max_over_ranks):
+def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barrier, max_over_ranks, fp8=False):
     """End to end through the public API from pinned host buffers (the latent page pool is
     resident device state; each step sends q, block_table and cache_seqlens and reads back
     out and lse).  Two steps are in flight, as a serving loop would run them: step i+1's
@@ -580,9 +613,14 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
         # ran earlier on the same stream
         tile, splits = ops.get_mla_metadata(sl_["sl"], R, w.h_kv, tile_metadata=sl_["tile"],
                                             num_splits=sl_["splits"])
-        ops.flash_mla_with_kvcache(sl_["q"], d0["k_cache"], sl_["bt"], sl_["sl"], 512, tile, splits,
-                                   softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
-                                   out=sl_["out"], lse=sl_["lse"], kernel=args.kernel)
+        if fp8:
+            ops.mla_decode_paged_fp8(sl_["q"], d0["k8"], d0["k_scale"], sl_["bt"], sl_["sl"], 512, tile, splits,
+                                     softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
+                                     out=sl_["out"], lse=sl_["lse"])
+        else:
+            ops.flash_mla_with_kvcache(sl_["q"], d0["k_cache"], sl_["bt"], sl_["sl"], 512, tile, splits,
+                                       softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
+                                       out=sl_["out"], lse=sl_["lse"], kernel=args.kernel)
         sl_["done"].record(kstream)
         with torch.cuda.stream(down_stream):
             down_stream.wait_event(sl_["done"])
@@ -631,7 +669,7 @@ def run_ours(args):
     per_workload = None
     if world == 1 and not args.no_per_workload:
         per_workload = {}
-        for name in W.WORKLOADS:
+        for name in list(W.WORKLOADS) + list(FP8_WORKLOADS):
             r = head if name == args.workload else measure(name, args, dev, group, rank, world,
                                                             with_e2e=False, cpu_seconds=2.0)
             per_workload[name] = {k: r[k] for k in ("config", "unit", "value", "ms_per_step", "roofline",
@@ -667,7 +705,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="memory_bound", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="memory_bound", choices=sorted(list(W.WORKLOADS) + list(FP8_WORKLOADS)))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
