@@ -226,6 +226,52 @@ MLA_API int mla_combine(const int32_t *num_splits, int batch, int s_q, int h_q, 
                 float *lse, mla_stream_t stream);
 
 /*
+ * mla_merge_partials -- log-sum-exp merge of n_parts partial decodes of the same query rows,
+ * each over a disjoint part of the keys (a sequence sharded over GPUs: every GPU decodes its
+ * shard of the pages with mla_decode_paged, the (out, lse) of all shards are gathered, then
+ * merged here).  The merge is the combine's (north_star: "split-KV partials are merged by a
+ * log-sum-exp combine"): lse = ln sum_k exp(lse_k), out = sum_k exp(lse_k - lse) out_k;
+ * partials with lse_k = -inf weigh nothing; rows with no key in any part get out = 0 and
+ * lse = -inf.
+ *   o_parts    device bf16 [n_parts][batch][s_q][h_q][dv], contiguous, 16-byte aligned
+ *   lse_parts  device fp32 [n_parts][batch][h_q][s_q] (natural log), contiguous
+ *   out, lse   device bf16 [batch][s_q][h_q][dv] and fp32 [batch][h_q][s_q], written
+ * dv must be 512.  One kernel on `stream`.  Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED,
+ * MLA_ERR_CUDA.
+ */
+MLA_API int mla_merge_partials(const void *o_parts, const float *lse_parts, int n_parts, int batch, int s_q,
+                               int h_q, int dv, void *out, float *lse, mla_stream_t stream);
+
+/*
+ * mla_absorb_query / mla_absorb_output -- the dense GEMMs either side of the latent decode
+ * ("DeepSeek FlashMLA ... practitioner notes", dpshk.com, section 2.1: with the per-head key
+ * k_h = W^UK_h c of latent row c, the score q_h . k_h = (W^UK_h^T q_h) . c, so the query is
+ * carried into latent space once instead of expanding the cache per head; the value
+ * W^UV_h c likewise leaves latent space after the weighted sum).  Head sizes are fixed to
+ * those of the call shape: 128 non-positional query columns per head, 64 positional (rope)
+ * columns, latent width 512, 128 output columns per head.  tokens = batch * s_q.
+ *
+ * mla_absorb_query:  q_out[t][h][0:512] = sum_d q_nope[t][h][d] * w_uk[h][d][0:512];
+ *                    q_out[t][h][512:576] = q_rope[t][h][0:64]
+ *   q_nope   device bf16, element (t, h, d) at t * nope_strides[0] + h * nope_strides[1] + d
+ *   q_rope   device bf16, element (t, h, c) at t * rope_strides[0] + h * rope_strides[1] + c
+ *   w_uk     device bf16 [heads][128][512], contiguous
+ *   q_out    device bf16 [tokens][heads][576], contiguous (the decode's q)
+ * mla_absorb_output: out[t][h][d] = sum_c o_latent[t][h][c] * w_uv[h][d][c]
+ *   o_latent device bf16, element (t, h, c) at t * latent_strides[0] + h * latent_strides[1]
+ *            + c (the decode's out)
+ *   w_uv     device bf16 [heads][128][512], contiguous
+ *   out      device bf16 [tokens][heads][128], contiguous
+ * bf16 inputs, fp32 accumulation (warp MMA), bf16 results; strides in elements, multiples of
+ * 8.  Errors: MLA_ERR_ARG, MLA_ERR_CUDA.
+ */
+MLA_API int mla_absorb_query(const void *q_nope, const int64_t nope_strides[2], const void *q_rope,
+                             const int64_t rope_strides[2], const void *w_uk, int tokens, int heads, void *q_out,
+                             mla_stream_t stream);
+MLA_API int mla_absorb_output(const void *o_latent, const int64_t latent_strides[2], const void *w_uv, int tokens,
+                              int heads, void *out, mla_stream_t stream);
+
+/*
  * mla_query_status -- synchronise `stream`, read and clear the workspace status block.
  * Returns MLA_OK, MLA_ERR_TIMEOUT (a device wait gave up; its results are invalid) or
  * MLA_ERR_CUDA (the stream reported an error).

@@ -11,6 +11,8 @@ Contents
                                  scale per token and latent head, dequantised exactly)
   e4m3_to_float64                OCP E4M3 decoding (the C oracle's, exposed for its pins)
   combine                        log-sum-exp merge of split partials (numpy fp64)
+  absorb_query / absorb_output   the weight-absorption products either side of the latent
+                                 decode (numpy fp64 einsum)
   metadata                       split-KV scheduler specification (``metadata.py``)
 
 Where each formula comes from is stated in ``mla_oracle.c`` and ``metadata.py``.
@@ -236,3 +238,30 @@ def combine(lse_parts, o_parts):
     scale = np.where(finite, np.exp(lse_parts - np.where(finite, lse, 0.0)), 0.0)
     out = np.sum(scale[..., None] * o_parts, axis=0)
     return out, lse
+
+
+def absorb_query(q_nope, q_rope, w_uk):
+    """Query carried into latent space ("DeepSeek FlashMLA ... practitioner notes", dpshk.com,
+    section 2.1: the per-head key is the up-projection W^UK_h of the latent row c, so the
+    score q_h . (W^UK_h c) is (W^UK_h^T q_h) . c and the projection moves onto the query).
+
+    q_nope [T, H, 128], q_rope [T, H, 64], w_uk [H, 128, 512] (head h's key up-projection,
+    rows = key column d, columns = latent column); any float dtype, computed in fp64.
+    Returns q' [T, H, 576]: q'[t, h, c] = sum_d q_nope[t, h, d] w_uk[h, d, c] for c < 512,
+    then the rope columns unchanged (the positional key part is stored as is in the cache).
+    """
+    qn = np.asarray(q_nope, dtype=np.float64)
+    qr = np.asarray(q_rope, dtype=np.float64)
+    w = np.asarray(w_uk, dtype=np.float64)
+    return np.concatenate([np.einsum("thd,hdc->thc", qn, w), qr], axis=-1)
+
+
+def absorb_output(o_latent, w_uv):
+    """Attention output taken out of latent space (same notes, section 2.1: the value is
+    W^UV_h c, and the weighted sum commutes with the projection, so it is applied once to
+    the latent output).  o_latent [T, H, 512], w_uv [H, 128, 512] (head h's value
+    up-projection, rows = output column d).  Returns o [T, H, 128] in fp64:
+    o[t, h, d] = sum_c w_uv[h, d, c] o_latent[t, h, c]."""
+    o = np.asarray(o_latent, dtype=np.float64)
+    w = np.asarray(w_uv, dtype=np.float64)
+    return np.einsum("thc,hdc->thd", o, w)

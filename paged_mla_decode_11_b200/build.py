@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libpagedmla.so")
 
-SOURCES = ["api.cu", "metadata.cu", "decode_mma.cu", "decode_tc.cu", "decode_wide.cu", "decode_pair.cu", "decode_fp8.cu", "combine.cu", "no_alloc.cu"]
+SOURCES = ["api.cu", "metadata.cu", "decode_mma.cu", "decode_tc.cu", "decode_wide.cu", "decode_pair.cu", "decode_fp8.cu", "combine.cu", "merge.cu", "absorb.cu", "no_alloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

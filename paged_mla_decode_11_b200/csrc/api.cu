@@ -467,6 +467,57 @@ int mla_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv
   return MLA_OK;
 }
 
+int mla_merge_partials(const void *o_parts, const float *lse_parts, int n_parts, int batch, int s_q, int h_q,
+                       int dv, void *out, float *lse, mla_stream_t stream) {
+  if (!o_parts || !lse_parts || !out || !lse) return fail(MLA_ERR_ARG, "null pointer argument");
+  if (n_parts < 1 || batch < 1 || s_q < 1 || h_q < 1)
+    return fail(MLA_ERR_ARG, "n_parts, batch, s_q and h_q must be >= 1");
+  if (dv != kDV) return fail(MLA_ERR_UNSUPPORTED, "dv must be %d (got %d)", kDV, dv);
+  if (!aligned(o_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) || !aligned(lse, 4))
+    return fail(MLA_ERR_ARG, "o_parts and out must be 16-byte aligned, lse_parts and lse 4-byte aligned");
+  cudaError_t e = launch_merge(static_cast<const __nv_bfloat16 *>(o_parts), lse_parts, n_parts, batch, s_q, h_q,
+                               static_cast<__nv_bfloat16 *>(out), lse, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge kernel launch");
+  return MLA_OK;
+}
+
+int mla_absorb_query(const void *q_nope, const int64_t nope_strides[2], const void *q_rope,
+                     const int64_t rope_strides[2], const void *w_uk, int tokens, int heads, void *q_out,
+                     mla_stream_t stream) {
+  if (!q_nope || !nope_strides || !q_rope || !rope_strides || !w_uk || !q_out)
+    return fail(MLA_ERR_ARG, "null pointer argument");
+  if (tokens < 1 || heads < 1) return fail(MLA_ERR_ARG, "tokens and heads must be >= 1");
+  if (int64_t(tokens + 63) / 64 > 65535 || heads > 65535) return fail(MLA_ERR_ARG, "too many tokens or heads");
+  for (int i = 0; i < 2; ++i)
+    if (nope_strides[i] < 0 || nope_strides[i] % 8 || rope_strides[i] < 0 || rope_strides[i] % 8)
+      return fail(MLA_ERR_ARG, "strides must be non-negative multiples of 8 elements");
+  if (!aligned(q_nope, 16) || !aligned(q_rope, 16) || !aligned(w_uk, 4) || !aligned(q_out, 16))
+    return fail(MLA_ERR_ARG, "q_nope, q_rope and q_out must be 16-byte aligned, w_uk 4-byte aligned");
+  cudaError_t e = launch_absorb_q(static_cast<const __nv_bfloat16 *>(q_nope), nope_strides[0], nope_strides[1],
+                                  static_cast<const __nv_bfloat16 *>(q_rope), rope_strides[0], rope_strides[1],
+                                  static_cast<const __nv_bfloat16 *>(w_uk), static_cast<__nv_bfloat16 *>(q_out), tokens,
+                                  heads, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "query absorption launch");
+  return MLA_OK;
+}
+
+int mla_absorb_output(const void *o_latent, const int64_t latent_strides[2], const void *w_uv, int tokens, int heads,
+                      void *out, mla_stream_t stream) {
+  if (!o_latent || !latent_strides || !w_uv || !out) return fail(MLA_ERR_ARG, "null pointer argument");
+  if (tokens < 1 || heads < 1) return fail(MLA_ERR_ARG, "tokens and heads must be >= 1");
+  if (int64_t(tokens + 63) / 64 > 65535 || heads > 65535) return fail(MLA_ERR_ARG, "too many tokens or heads");
+  for (int i = 0; i < 2; ++i)
+    if (latent_strides[i] < 0 || latent_strides[i] % 8)
+      return fail(MLA_ERR_ARG, "strides must be non-negative multiples of 8 elements");
+  if (!aligned(o_latent, 16) || !aligned(w_uv, 4) || !aligned(out, 4))
+    return fail(MLA_ERR_ARG, "o_latent must be 16-byte aligned, w_uv and out 4-byte aligned");
+  cudaError_t e = launch_absorb_out(static_cast<const __nv_bfloat16 *>(o_latent), latent_strides[0], latent_strides[1],
+                                    static_cast<const __nv_bfloat16 *>(w_uv), static_cast<__nv_bfloat16 *>(out), tokens,
+                                    heads, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "output absorption launch");
+  return MLA_OK;
+}
+
 int mla_query_status(void *workspace, mla_stream_t stream) {
   if (!workspace) return fail(MLA_ERR_ARG, "workspace is null");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

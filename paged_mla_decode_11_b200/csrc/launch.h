@@ -36,6 +36,13 @@ cudaError_t launch_decode_fp8(const CUtensorMap &k8_map, const CUtensorMap &scal
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,
                            const float *lse_accum, const float *o_accum, __nv_bfloat16 *out,
                            float *lse, cudaStream_t stream);
+cudaError_t launch_merge(const __nv_bfloat16 *o_parts, const float *lse_parts, int n_parts, int batch, int s_q,
+                         int h_q, __nv_bfloat16 *out, float *lse, cudaStream_t stream);
+cudaError_t launch_absorb_q(const __nv_bfloat16 *q_nope, int64_t n_row, int64_t n_head, const __nv_bfloat16 *q_rope,
+                            int64_t r_row, int64_t r_head, const __nv_bfloat16 *w_uk, __nv_bfloat16 *q_out, int T,
+                            int H, cudaStream_t stream);
+cudaError_t launch_absorb_out(const __nv_bfloat16 *o_lat, int64_t l_row, int64_t l_head, const __nv_bfloat16 *w_uv,
+                              __nv_bfloat16 *out, int T, int H, cudaStream_t stream);
 cudaError_t launch_watchdog_selftest(int *status, unsigned long long timeout_ns,
                                      cudaStream_t stream);
 

@@ -41,6 +41,7 @@ EXPORTED = (
     "mla_device_sm_count", "mla_num_parts", "mla_metadata_size", "mla_get_metadata", "mla_workspace_size",
     "mla_decode_paged", "mla_combine", "mla_query_status", "mla_watchdog_selftest",
     "mla_last_error_string", "mla_decode_paged_static", "mla_query_status_static", "mla_decode_paged_fp8",
+    "mla_merge_partials", "mla_absorb_query", "mla_absorb_output",
 )
 
 _lib = None
@@ -79,6 +80,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "mla_query_status": [P, P],
             "mla_watchdog_selftest": [P, U64, P],
             "mla_query_status_static": [P],
+            "mla_merge_partials": [P, P, I, I, I, I, I, P, P, P],
+            "mla_absorb_query": [P, P, P, P, P, I, I, P, P],
+            "mla_absorb_output": [P, P, P, I, I, P, P],
             "mla_decode_paged_fp8": [P, P, I, I, I, I, P, P, I64, I, I, P, I64, P, I, P, I, P,
                                      ctypes.c_float, I, P, P, P, ctypes.c_size_t, ctypes.c_uint, P],
         }
@@ -350,6 +354,68 @@ def mla_combine(num_splits: torch.Tensor, s_q: int, h_q: int, h_kv: int, num_par
     _check(load_library().mla_combine(num_splits.data_ptr(), b, s_q, h_q, h_kv, dv, num_parts,
                                       workspace.data_ptr(), workspace.numel(), out.data_ptr(),
                                       lse.data_ptr(), _stream_ptr(out.device)))
+
+
+def mla_merge_partials(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Log-sum-exp merge of partial decodes over disjoint keys: o_parts [n, b, s_q, h_q, 512]
+    bf16, lse_parts [n, b, h_q, s_q] fp32 -> (out [b, s_q, h_q, 512], lse [b, h_q, s_q])."""
+    _require_cuda(o_parts, "o_parts", torch.bfloat16)
+    _require_cuda(lse_parts, "lse_parts", torch.float32)
+    if o_parts.dim() != 5 or lse_parts.dim() != 4:
+        raise ValueError("o_parts must be [n, b, s_q, h_q, dv] and lse_parts [n, b, h_q, s_q]")
+    n, b, s_q, h_q, dv = o_parts.shape
+    if lse_parts.shape != (n, b, h_q, s_q):
+        raise ValueError("lse_parts must be [n, b, h_q, s_q] matching o_parts")
+    if not o_parts.is_contiguous() or not lse_parts.is_contiguous():
+        raise ValueError("o_parts and lse_parts must be contiguous")
+    dev = o_parts.device
+    if out is None:
+        out = torch.empty(b, s_q, h_q, dv, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(b, h_q, s_q, dtype=torch.float32, device=dev)
+    _check(load_library().mla_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), n, b, s_q, h_q, dv,
+                                             out.data_ptr(), lse.data_ptr(), _stream_ptr(dev)))
+    return out, lse
+
+
+_I64x2 = ctypes.c_int64 * 2
+
+
+def absorb_query(q_nope: torch.Tensor, q_rope: torch.Tensor, w_uk: torch.Tensor,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """q' = [W^UK^T q_nope ; q_rope] per token and head: q_nope [T, H, 128], q_rope [T, H, 64]
+    (bf16, last dim contiguous), w_uk [H, 128, 512] -> q' [T, H, 576] bf16."""
+    for t, n in ((q_nope, "q_nope"), (q_rope, "q_rope"), (w_uk, "w_uk")):
+        _require_cuda(t, n, torch.bfloat16)
+    T, H, dn = q_nope.shape
+    if dn != 128 or q_rope.shape != (T, H, 64) or w_uk.shape != (H, 128, 512):
+        raise ValueError("q_nope [T, H, 128], q_rope [T, H, 64], w_uk [H, 128, 512]")
+    if q_nope.stride(2) != 1 or q_rope.stride(2) != 1 or not w_uk.is_contiguous():
+        raise ValueError("innermost dimensions must be contiguous, w_uk contiguous")
+    if out is None:
+        out = torch.empty(T, H, 576, dtype=torch.bfloat16, device=q_nope.device)
+    _check(load_library().mla_absorb_query(q_nope.data_ptr(), _I64x2(q_nope.stride(0), q_nope.stride(1)),
+                                           q_rope.data_ptr(), _I64x2(q_rope.stride(0), q_rope.stride(1)),
+                                           w_uk.data_ptr(), T, H, out.data_ptr(), _stream_ptr(q_nope.device)))
+    return out
+
+
+def absorb_output(o_latent: torch.Tensor, w_uv: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """o = W^UV o_latent per token and head: o_latent [T, H, 512] bf16 (last dim contiguous),
+    w_uv [H, 128, 512] -> o [T, H, 128] bf16."""
+    _require_cuda(o_latent, "o_latent", torch.bfloat16)
+    _require_cuda(w_uv, "w_uv", torch.bfloat16)
+    T, H, dc = o_latent.shape
+    if dc != 512 or w_uv.shape != (H, 128, 512):
+        raise ValueError("o_latent [T, H, 512], w_uv [H, 128, 512]")
+    if o_latent.stride(2) != 1 or not w_uv.is_contiguous():
+        raise ValueError("o_latent's last dimension and w_uv must be contiguous")
+    if out is None:
+        out = torch.empty(T, H, 128, dtype=torch.bfloat16, device=o_latent.device)
+    _check(load_library().mla_absorb_output(o_latent.data_ptr(), _I64x2(o_latent.stride(0), o_latent.stride(1)),
+                                            w_uv.data_ptr(), T, H, out.data_ptr(), _stream_ptr(o_latent.device)))
+    return out
 
 
 def query_status(workspace: torch.Tensor) -> int:

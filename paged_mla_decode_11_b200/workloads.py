@@ -185,6 +185,27 @@ def make_inputs_fp8(w: Workload, seed: int = 0, max_pages: Optional[int] = None)
     return x
 
 
+D_NOPE = 128   # non-positional query / key columns per head
+D_ROPE = 64    # positional (rope) columns, stored in the cache as they are
+D_HEAD_V = 128  # value columns per head after the output up-projection
+
+
+def make_absorb_inputs(tokens: int, heads: int, seed: int = 0) -> dict:
+    """Per-head query halves and random-init up-projections for the absorption products.
+
+    Draw order from one CPU generator: q_nope ~ N(0, 1) [T, H, 128], q_rope ~ N(0, 1)
+    [T, H, 64], w_uk ~ N(0, 1/128) [H, 128, 512], w_uv ~ N(0, 1/512) [H, 128, 512] (variance
+    1 / fan-in), o_latent ~ N(0, 1) [T, H, 512]; all rounded to bf16.  q_nope and q_rope are
+    the two column ranges of one [T, H, 192] projection output, as a model produces them.
+    """
+    g = torch.Generator().manual_seed(seed)
+    qkv = torch.randn(tokens, heads, D_NOPE + D_ROPE, generator=g).to(torch.bfloat16)
+    w_uk = (torch.randn(heads, D_NOPE, D_V, generator=g) * D_NOPE ** -0.5).to(torch.bfloat16)
+    w_uv = (torch.randn(heads, D_HEAD_V, D_V, generator=g) * D_V ** -0.5).to(torch.bfloat16)
+    o_lat = torch.randn(tokens, heads, D_V, generator=g).to(torch.bfloat16)
+    return dict(q_nope=qkv[..., :D_NOPE], q_rope=qkv[..., D_NOPE:], w_uk=w_uk, w_uv=w_uv, o_latent=o_lat)
+
+
 def custom(batch: int, s_q: int, h_q: int, h_kv: int, seqlens: Sequence[int],
            causal: bool = True, scale: Optional[float] = None, outlier_frac: float = 0.0,
            name: str = "custom") -> Workload:
