@@ -10,6 +10,9 @@ Contents
   mla_decode_fp8 / ..._rows_fp8  the same over an FP8 latent cache (E4M3 codes and one fp32
                                  scale per token and latent head, dequantised exactly)
   e4m3_to_float64                OCP E4M3 decoding (the C oracle's, exposed for its pins)
+  mla_decode_sparse / ..._rows_sparse
+                                 token-level sparse decode: each query token attends to the
+                                 key positions of its CSR list (row_ptr, col_idx)
   combine                        log-sum-exp merge of split partials (numpy fp64)
   absorb_query / absorb_output   the weight-absorption products either side of the latent
                                  decode (numpy fp64 einsum)
@@ -68,6 +71,13 @@ def _load():
             i32, f64, i32,
             P, i64, P, P]
         lib.oracle_mla_decode_rows_fp8.restype = i32
+        lib.oracle_mla_decode_rows_sparse.argtypes = [
+            P, i64, i64, i64, i32, i32, i32, i32,
+            P, i64, i32, i32,
+            P, i64, P, P, P, P, P,
+            i32, f64, i32,
+            P, i64, P, P]
+        lib.oracle_mla_decode_rows_sparse.restype = i32
         lib.oracle_e4m3_to_double.argtypes = [P, i64, P]
         lib.oracle_e4m3_to_double.restype = i32
         lib.oracle_num_threads.restype = i32
@@ -184,6 +194,65 @@ def mla_decode_rows_fp8(q, k8, k_scale, block_table, cache_seqlens, rows, dv: in
         ptr(rows), n, ptr(out), ptr(lse))
     if rc != 0:
         raise ValueError(f"oracle rejected its inputs (status {rc})")
+    return out, lse
+
+
+def mla_decode_rows_sparse(q, k_cache, block_table, cache_seqlens, row_ptr, col_idx, rows, dv: int = 512,
+                           softmax_scale: Optional[float] = None, causal: bool = True,
+                           kv_begin=None, kv_end=None):
+    """fp64 token-level sparse decode of the listed rows.
+
+    row_ptr [batch * s_q + 1] int32 (non-decreasing), col_idx [nnz] int32: query token
+    (b, s) attends to the positions col_idx[row_ptr[b * s_q + s] : row_ptr[b * s_q + s + 1]]
+    that lie in [0, n) with n the row's visible length (causal rule as in the dense
+    decode); other entries are pruned, repeated entries count once per listing.  kv_begin /
+    kv_end (optional [b]) select list entries by their index in the list.  Other arguments
+    and the result as in mla_decode_rows.
+    """
+    lib = _load()
+    b, s_q, h_q, d = (int(x) for x in q.shape)
+    num_pages, page, h_kv, d2 = (int(x) for x in k_cache.shape)
+    if d2 != d:
+        raise ValueError("q and k_cache disagree on the latent width")
+    qn = _bf16_bits(q)
+    kn = _bf16_bits(k_cache)
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    sl = np.ascontiguousarray(np.asarray(cache_seqlens, dtype=np.int32))
+    rp = np.ascontiguousarray(np.asarray(row_ptr, dtype=np.int32).reshape(-1))
+    ci = np.ascontiguousarray(np.asarray(col_idx, dtype=np.int32).reshape(-1))
+    if rp.shape[0] != b * s_q + 1 or int(rp[-1]) > ci.shape[0]:
+        raise ValueError("row_ptr must have batch * s_q + 1 entries within col_idx")
+    if ci.shape[0] == 0:
+        ci = np.zeros(1, dtype=np.int32)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    kb = None if kv_begin is None else np.ascontiguousarray(np.asarray(kv_begin, dtype=np.int32))
+    ke = None if kv_end is None else np.ascontiguousarray(np.asarray(kv_end, dtype=np.int32))
+    n = rows.shape[0]
+    out = np.zeros((n, dv), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    scale = d ** -0.5 if softmax_scale is None else float(softmax_scale)
+    ptr = lambda a: None if a is None else a.ctypes.data
+    rc = lib.oracle_mla_decode_rows_sparse(
+        ptr(qn), s_q * h_q * d, h_q * d, d, b, s_q, h_q, d,
+        ptr(kn), num_pages, page, h_kv,
+        ptr(bt), bt.shape[1], ptr(sl), ptr(rp), ptr(ci), ptr(kb), ptr(ke),
+        dv, scale, int(bool(causal)),
+        ptr(rows), n, ptr(out), ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its inputs (status {rc})")
+    return out, lse
+
+
+def mla_decode_sparse(q, k_cache, block_table, cache_seqlens, row_ptr, col_idx, dv: int = 512,
+                      softmax_scale: Optional[float] = None, causal: bool = True,
+                      kv_begin=None, kv_end=None):
+    """fp64 token-level sparse decode of the whole batch (see mla_decode_rows_sparse):
+    out [b, s_q, h_q, dv], lse [b, h_q, s_q]."""
+    b, s_q, h_q, _ = (int(x) for x in q.shape)
+    out, lse = mla_decode_rows_sparse(q, k_cache, block_table, cache_seqlens, row_ptr, col_idx,
+                                      all_rows(b, s_q, h_q), dv, softmax_scale, causal, kv_begin, kv_end)
+    out = out.reshape(b, s_q, h_q, dv)
+    lse = lse.reshape(b, s_q, h_q).transpose(0, 2, 1).copy()
     return out, lse
 
 

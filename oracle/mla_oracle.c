@@ -37,6 +37,18 @@
  *   c_j[t] = scale_j * e4m3(code_j[t]);
  * the decode itself is the definition above applied to these rows.  k8 is [num_pages, page,
  * h_kv, d] uint8, k_scale is [h_kv, num_pages, page] fp32.
+ *
+ * Token-level sparse decode (oracle_mla_decode_rows_sparse).  The same Baidu page, section
+ * 三.3 (the token-level sparse attention kernel), keeps only the Top-K key connections of a
+ * query and stores the sparse attention pattern in CSR form; the scoring that picks them is
+ * outside the decode.  Reading taken here: query token (b, s) comes with a list of key
+ * positions col_idx[row_ptr[b * s_q + s] .. row_ptr[b * s_q + s + 1]) in CSR form, shared by
+ * all h_q heads of that token (the cache has one latent row per token and latent head).  The
+ * decode is the definition above with the keys j in [lo, hi) replaced by the list entries
+ * whose position lies in [0, n) (n as above, so the causal rule still holds); other entries
+ * (padding such as -1, or positions the row may not see) are pruned.  Entries are taken as
+ * listed: a position listed twice counts twice.  kv_begin / kv_end, when given, select list
+ * entries by their index in the list (a split of the list).
  */
 #include <math.h>
 #include <stdint.h>
@@ -118,6 +130,7 @@ static int decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs
                        const int32_t *block_table, int64_t bt_stride,
                        const int32_t *cache_seqlens,
                        const int32_t *kv_begin, const int32_t *kv_end,
+                       const int32_t *row_ptr, const int32_t *col_idx,
                        int dv, double scale, int causal,
                        const int32_t *rows, int64_t n_rows,
                        double *out_rows, double *lse_rows) {
@@ -133,6 +146,7 @@ static int decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs
     {
         int64_t cap = 0;
         double *x = NULL;
+        int64_t *pos = NULL;
 #pragma omp for schedule(dynamic, 1)
         for (int64_t r = 0; r < n_rows; ++r) {
             const int b = rows[3 * r + 0], s = rows[3 * r + 1], h = rows[3 * r + 2];
@@ -146,36 +160,47 @@ static int decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs
             const int64_t L = cache_seqlens[b];
             int64_t n = causal ? L - (s_q - 1 - s) : L;
             if (n < 0) n = 0;
+            /* the candidate keys: positions [0, n), or the token's list entries */
+            const int64_t e0 = row_ptr ? row_ptr[(int64_t)b * s_q + s] : 0;
+            const int64_t cnt = row_ptr ? row_ptr[(int64_t)b * s_q + s + 1] - e0 : n;
             int64_t lo = kv_begin ? kv_begin[b] : 0;
-            int64_t hi = kv_end ? kv_end[b] : n;
-            if (hi > n) hi = n;
+            int64_t hi = kv_end ? kv_end[b] : cnt;
+            if (hi > cnt) hi = cnt;
             if (lo < 0) lo = 0;
             for (int t = 0; t < dv; ++t) o[t] = 0.0;
-            if (hi <= lo) {
-                lse_rows[r] = -INFINITY;
-                continue;
-            }
             if (hi - lo > cap) {
                 free(x);
+                free(pos);
                 cap = hi - lo;
                 x = (double *)malloc((size_t)cap * sizeof(double));
-                if (!x) {
+                pos = (int64_t *)malloc((size_t)cap * sizeof(int64_t));
+                if (!x || !pos) {
 #pragma omp atomic write
                     status = -2;
                     cap = 0;
                     continue;
                 }
             }
+            /* the key positions this row attends to */
+            int64_t nk = 0;
+            for (int64_t e = lo; e < hi; ++e) {
+                const int64_t j = row_ptr ? col_idx[e0 + e] : e;
+                if (j >= 0 && j < n) pos[nk++] = j;
+            }
+            if (nk == 0) {
+                lse_rows[r] = -INFINITY;
+                continue;
+            }
             const uint16_t *qrow = q + b * qs_b + s * qs_s + h * qs_h;
             /* pass 1: scores and their maximum */
             double M = -INFINITY;
             int bad = 0;
-            for (int64_t j = lo; j < hi; ++j) {
+            for (int64_t k = 0; k < nk; ++k) {
+                const int64_t j = pos[k];
                 const int64_t phys = block_table[b * bt_stride + j / page];
                 if (phys < 0 || phys >= num_pages) { bad = 1; break; }
-                const double acc = row_dot(cache, phys, (int)(j % page), kvh, qrow);
-                x[j - lo] = scale * acc;
-                if (x[j - lo] > M) M = x[j - lo];
+                x[k] = scale * row_dot(cache, phys, (int)(j % page), kvh, qrow);
+                if (x[k] > M) M = x[k];
             }
             if (bad) {
 #pragma omp atomic write
@@ -185,15 +210,16 @@ static int decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs
             }
             /* pass 2: normaliser and weighted sum of the first dv columns */
             double Z = 0.0;
-            for (int64_t j = lo; j < hi; ++j) Z += exp(x[j - lo] - M);
-            for (int64_t j = lo; j < hi; ++j) {
+            for (int64_t k = 0; k < nk; ++k) Z += exp(x[k] - M);
+            for (int64_t k = 0; k < nk; ++k) {
+                const int64_t j = pos[k];
                 const int64_t phys = block_table[b * bt_stride + j / page];
-                const double p = exp(x[j - lo] - M) / Z;
-                row_axpy(cache, phys, (int)(j % page), kvh, p, o, dv);
+                row_axpy(cache, phys, (int)(j % page), kvh, exp(x[k] - M) / Z, o, dv);
             }
             lse_rows[r] = M + log(Z);
         }
         free(x);
+        free(pos);
     }
     return status;
 }
@@ -217,7 +243,7 @@ int oracle_mla_decode_rows(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_
     if (!k_cache) return -1;
     cache_t c = {k_cache, NULL, NULL, num_pages, page, h_kv, d};
     return decode_rows(q, qs_b, qs_s, qs_h, batch, s_q, h_q, d, &c, block_table, bt_stride, cache_seqlens,
-                       kv_begin, kv_end, dv, scale, causal, rows, n_rows, out_rows, lse_rows);
+                       kv_begin, kv_end, NULL, NULL, dv, scale, causal, rows, n_rows, out_rows, lse_rows);
 }
 
 /* The same decode over an FP8 (E4M3 + per-token fp32 scale) latent cache. */
@@ -233,5 +259,26 @@ int oracle_mla_decode_rows_fp8(const uint16_t *q, int64_t qs_b, int64_t qs_s, in
     if (!k8 || !k_scale) return -1;
     cache_t c = {NULL, k8, k_scale, num_pages, page, h_kv, d};
     return decode_rows(q, qs_b, qs_s, qs_h, batch, s_q, h_q, d, &c, block_table, bt_stride, cache_seqlens,
-                       kv_begin, kv_end, dv, scale, causal, rows, n_rows, out_rows, lse_rows);
+                       kv_begin, kv_end, NULL, NULL, dv, scale, causal, rows, n_rows, out_rows, lse_rows);
+}
+
+/* Token-level sparse decode over a bf16 latent cache: each query token (b, s) attends to the
+ * listed key positions col_idx[row_ptr[b * s_q + s] .. row_ptr[b * s_q + s + 1]) that lie in
+ * [0, n) (header, last paragraph).  row_ptr has batch * s_q + 1 entries, non-decreasing. */
+int oracle_mla_decode_rows_sparse(const uint16_t *q, int64_t qs_b, int64_t qs_s, int64_t qs_h,
+                                  int batch, int s_q, int h_q, int d,
+                                  const uint16_t *k_cache, int64_t num_pages, int page, int h_kv,
+                                  const int32_t *block_table, int64_t bt_stride,
+                                  const int32_t *cache_seqlens,
+                                  const int32_t *row_ptr, const int32_t *col_idx,
+                                  const int32_t *kv_begin, const int32_t *kv_end,
+                                  int dv, double scale, int causal,
+                                  const int32_t *rows, int64_t n_rows,
+                                  double *out_rows, double *lse_rows) {
+    if (!k_cache || !row_ptr || !col_idx) return -1;
+    for (int64_t i = 0; i < (int64_t)batch * s_q; ++i)
+        if (row_ptr[i + 1] < row_ptr[i] || row_ptr[0] < 0) return -1;
+    cache_t c = {k_cache, NULL, NULL, num_pages, page, h_kv, d};
+    return decode_rows(q, qs_b, qs_s, qs_h, batch, s_q, h_q, d, &c, block_table, bt_stride, cache_seqlens,
+                       kv_begin, kv_end, row_ptr, col_idx, dv, scale, causal, rows, n_rows, out_rows, lse_rows);
 }

@@ -185,6 +185,67 @@ def make_inputs_fp8(w: Workload, seed: int = 0, max_pages: Optional[int] = None)
     return x
 
 
+# Token-level sparse decode: the memory-bound query shape (64 sequences, 16 heads) over
+# longer contexts, each query token keeping 2,048 key positions (Top-K) of its sequence.
+SPARSE = Workload("sparse b64 h16 L~U[4096,32768] top-2048", 64, 1, 16, 1, ("uniform", 4096, 32768))
+SPARSE_TOPK = 2048
+
+
+def make_sparse_lists(seqlens: Sequence[int], s_q: int, topk: int, seed: int = 0, causal: bool = True,
+                      pad: bool = False) -> tuple[torch.Tensor, torch.Tensor]:
+    """Key lists in CSR form for the token-level sparse decode.
+
+    Query token (b, s) keeps min(topk, n) distinct positions drawn uniformly from [0, n) (n =
+    L_b, less s_q - 1 - s under the causal rule), in increasing order; with ``pad`` every
+    list is filled up to topk entries with -1 (a fixed-width Top-K buffer).  Drawn with
+    torch.randperm from one CPU generator seeded with ``seed``, token by token in (b, s)
+    order.  Returns (row_ptr [batch * s_q + 1], col_idx [nnz]) int32."""
+    g = torch.Generator().manual_seed(seed)
+    lists = []
+    for L in (int(x) for x in seqlens):
+        for s in range(s_q):
+            n = max(0, L - (s_q - 1 - s)) if causal else L
+            k = min(topk, n)
+            pos = torch.sort(torch.randperm(n, generator=g)[:k])[0].to(torch.int32) if k else torch.zeros(0, dtype=torch.int32)
+            if pad and k < topk:
+                pos = torch.cat([pos, torch.full((topk - k,), -1, dtype=torch.int32)])
+            lists.append(pos)
+    row_ptr = torch.zeros(len(lists) + 1, dtype=torch.int32)
+    row_ptr[1:] = torch.cumsum(torch.tensor([len(x) for x in lists], dtype=torch.int64), 0).to(torch.int32)
+    col_idx = torch.cat(lists) if int(row_ptr[-1]) else torch.zeros(0, dtype=torch.int32)
+    return row_ptr, col_idx
+
+
+def make_inputs_sparse(w: Workload, topk: int, seed: int = 0, pad: bool = False) -> dict:
+    """make_inputs plus the key lists (make_sparse_lists, drawn with seed + 1): adds row_ptr,
+    col_idx and topk."""
+    x = make_inputs(w, seed)
+    x["row_ptr"], x["col_idx"] = make_sparse_lists(x["cache_seqlens"].tolist(), w.s_q, topk, seed + 1, w.causal, pad)
+    x["topk"] = topk
+    return x
+
+
+def sparse_work(row_ptr, col_idx, cache_seqlens, s_q: int, h_q: int, h_kv: int, causal: bool,
+                d: int = D_QK, dv: int = D_V) -> tuple[int, int]:
+    """Algorithmic (bytes, flops) of one sparse decode call: every visible listed key row read
+    once per latent head (d * 2 bytes) plus its 4-byte list entry, the query read and the
+    output written once; flops 2 (d + dv) per visible key and query head."""
+    rp = [int(v) for v in row_ptr]
+    ci = col_idx.tolist() if hasattr(col_idx, "tolist") else list(col_idx)
+    lens = [int(v) for v in cache_seqlens]
+    keys = 0
+    entries = rp[-1] - rp[0]
+    for i in range(len(rp) - 1):
+        b, s = divmod(i, s_q)
+        n = max(0, lens[b] - (s_q - 1 - s)) if causal else lens[b]
+        keys += sum(1 for j in ci[rp[i]:rp[i + 1]] if 0 <= j < n)
+    batch = len(lens)
+    g = h_q // h_kv
+    byts = keys * h_kv * d * 2 + entries * 4 + batch * s_q * h_q * (d * 2 + dv * 2 + 4)
+    flops = keys * g * 2 * (d + dv) * h_kv
+    return byts, flops
+
+
 D_NOPE = 128   # non-positional query / key columns per head
 D_ROPE = 64    # positional (rope) columns, stored in the cache as they are
 D_HEAD_V = 128  # value columns per head after the output up-projection
