@@ -217,19 +217,37 @@ class ClockSampler:
 # latent head), decoded by mla_decode_paged_fp8; the name maps to the bf16 workload it stores.
 FP8_WORKLOADS = {"memory_bound_fp8": "memory_bound"}
 FP8_TOKEN_BYTES = 576 + 4
+# Token-level sparse decode (mla_decode_sparse): each query token keeps SPARSE_TOPK listed key
+# positions of its sequence.
+SPARSE_WORKLOADS = {"sparse": (W.SPARSE, W.SPARSE_TOPK)}
+ALL_WORKLOADS = list(W.WORKLOADS) + list(FP8_WORKLOADS) + list(SPARSE_WORKLOADS)
 
 
 def workload_spec(name):
-    """(Workload, is_fp8) of a bench workload name."""
+    """(Workload, kind) of a bench workload name; kind is "bf16", "fp8" or "sparse"."""
     if name in FP8_WORKLOADS:
-        return W.WORKLOADS[FP8_WORKLOADS[name]], True
-    return W.WORKLOADS[name], False
+        return W.WORKLOADS[FP8_WORKLOADS[name]], "fp8"
+    if name in SPARSE_WORKLOADS:
+        return SPARSE_WORKLOADS[name][0], "sparse"
+    return W.WORKLOADS[name], "bf16"
 
 
-def workload_work(x, w, fp8=False):
+def make_workload_inputs(name, seed):
+    w, kind = workload_spec(name)
+    if kind == "fp8":
+        return W.make_inputs_fp8(w, seed=seed)
+    if kind == "sparse":
+        return W.make_inputs_sparse(w, SPARSE_WORKLOADS[name][1], seed=seed)
+    return W.make_inputs(w, seed=seed)
+
+
+def workload_work(x, w, kind="bf16"):
+    if kind == "sparse":
+        return W.sparse_work(x["row_ptr"], x["col_idx"], x["cache_seqlens"].tolist(), w.s_q, w.h_q, w.h_kv,
+                             w.causal)
     lens = x["cache_seqlens"].tolist()
     nbytes, flops = W.algorithmic_work(lens, w.s_q, w.h_q, w.h_kv, w.causal,
-                                       token_bytes=FP8_TOKEN_BYTES if fp8 else None)
+                                       token_bytes=FP8_TOKEN_BYTES if kind == "fp8" else None)
     return nbytes, flops
 
 
@@ -243,12 +261,15 @@ def metric_of(w_name):
 METRIC = "paged MLA decode on 1 B200: HBM GB/s (mem-bound), TFLOPS (compute-bound)"
 
 
-def workload_config(w, fp8=False):
+def workload_config(w, kind="bf16"):
     lens = w.seqlens
-    cache = ("FP8 cache (E4M3 codes of the bf16 ~N(0,1) pool, one fp32 scale per token)" if fp8
+    cache = ("FP8 cache (E4M3 codes of the bf16 ~N(0,1) pool, one fp32 scale per token)" if kind == "fp8"
              else "bf16 q/cache ~N(0,1)")
-    return {"workload": f"{w.name}{' fp8' if fp8 else ''}: batch={w.batch}, s_q={w.s_q}, h_q={w.h_q}, "
-                        f"h_kv={w.h_kv}, d=576, dv=512, page 64, seqlens {lens}, causal={w.causal}, "
+    if kind == "sparse":
+        cache += (f", key lists: min({W.SPARSE_TOPK}, visible length) distinct uniform positions per "
+                  f"query token, sorted, CSR (seed 1)")
+    return {"workload": f"{w.name}{' fp8' if kind == 'fp8' else ''}: batch={w.batch}, s_q={w.s_q}, "
+                        f"h_q={w.h_q}, h_kv={w.h_kv}, d=576, dv=512, page 64, seqlens {lens}, causal={w.causal}, "
                         f"scale={w.scale:.6g}, {cache}, random block_table over one pool, seed 0"}
 
 
@@ -262,6 +283,19 @@ def oracle_sample(x, w, seqs):
     rows = np.array(rows, dtype=np.int32)
     fp8 = "k8" in x
     t0 = time.perf_counter()
+    if "row_ptr" in x:
+        oracle.mla_decode_rows_sparse(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], x["row_ptr"],
+                                      x["col_idx"], rows, dv=512, softmax_scale=w.scale, causal=w.causal)
+        dt = time.perf_counter() - t0
+        nb = fl = 0
+        rp = x["row_ptr"]
+        for b in seqs:
+            i0, i1 = b * w.s_q, (b + 1) * w.s_q
+            sub_rp = rp[i0:i1 + 1] - rp[i0]
+            bb, ff = W.sparse_work(sub_rp, x["col_idx"][int(rp[i0]):int(rp[i1])], [int(x["cache_seqlens"][b])],
+                                   w.s_q, w.h_q, w.h_kv, w.causal)
+            nb, fl = nb + bb, fl + ff
+        return dt, nb, fl
     if fp8:
         oracle.mla_decode_rows_fp8(x["q"], x["k8"], x["k_scale"], x["block_table"], x["cache_seqlens"], rows,
                                    dv=512, softmax_scale=w.scale, causal=w.causal)
@@ -278,16 +312,25 @@ def pick_sample(x, w, seconds):
     """Whole sequences, cycling from a start index, totalling about `seconds` of oracle work."""
     dt, nb, fl = oracle_sample(x, w, [0])
     per_flop = dt / max(fl, 1)
-    lens = x["cache_seqlens"].tolist()
     order = list(range(w.batch))
     chosen, acc = [], 0.0
     for b in order:
-        _, f = W.algorithmic_work([lens[b]], w.s_q, w.h_q, w.h_kv, w.causal)
+        f = sequence_flops(x, w, b)
         chosen.append(b)
         acc += f * per_flop
         if acc >= seconds:
             break
     return chosen
+
+
+def sequence_flops(x, w, b):
+    """Algorithmic flops of sequence b's query rows (its key lists for the sparse decode)."""
+    if "row_ptr" in x:
+        rp = x["row_ptr"]
+        i0, i1 = b * w.s_q, (b + 1) * w.s_q
+        return W.sparse_work(rp[i0:i1 + 1] - rp[i0], x["col_idx"][int(rp[i0]):int(rp[i1])],
+                             [int(x["cache_seqlens"][b])], w.s_q, w.h_q, w.h_kv, w.causal)[1]
+    return W.algorithmic_work([int(x["cache_seqlens"][b])], w.s_q, w.h_q, w.h_kv, w.causal)[1]
 
 
 def cpu_baseline(x, w, unit, seconds=10.0):
@@ -311,14 +354,13 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle
-    w, fp8 = workload_spec(args.workload)
-    x = W.make_inputs_fp8(w, seed=0) if fp8 else W.make_inputs(w, seed=0)
+    w, kind = workload_spec(args.workload)
+    x = make_workload_inputs(args.workload, 0)
     unit, _ = metric_of(args.workload)
     budget = 90.0 / max(args.steps + args.warmup, 1)
     per_step = min(2.0, max(0.05, budget))
     # samples are consecutive runs of whole sequences, cycling over the batch
     dt1, _, fl1 = oracle_sample(x, w, [0])
-    lens = x["cache_seqlens"].tolist()
     per_flop = dt1 / max(fl1, 1)
     cursor = 0
 
@@ -327,7 +369,7 @@ def run_reference(args):
         seqs, acc = [], 0.0
         while acc < per_step and len(seqs) < 64 * w.batch:  # the batch cycled if it is quick
             b = cursor % w.batch
-            _, f = W.algorithmic_work([lens[b]], w.s_q, w.h_q, w.h_kv, w.causal)
+            f = sequence_flops(x, w, b)
             seqs.append(b)
             acc += f * per_flop
             cursor += 1
@@ -352,7 +394,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(w, fp8),
+        "data": "synthetic", "config": workload_config(w, kind),
         "cpu_baseline": {"value": val, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -376,16 +418,17 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     the CPU oracle's throughput on a bounded sample.  Returns a dict of results."""
     from paged_mla_decode_11_b200 import ops
     barrier, max_over_ranks = group.barrier, group.max
-    w, fp8 = workload_spec(name)
-    R = w.rows_per_kv_head
+    w, kind = workload_spec(name)
+    fp8, sparse = kind == "fp8", kind == "sparse"
+    # rows per tile: every query token is a tile of its own in the sparse decode
+    R = w.h_q // w.h_kv if sparse else w.rows_per_kv_head
+    x = make_workload_inputs(name, args.seed + rank)
     if fp8:
-        x = W.make_inputs_fp8(w, seed=args.seed + rank)
         del x["k_cache"]  # the bf16 source of the codes stays on the host
         per_rep = x["k8"].numel() + x["k_scale"].numel() * 4
     else:
-        x = W.make_inputs(w, seed=args.seed + rank)
         per_rep = x["k_cache"].numel() * 2
-    nbytes, flops = workload_work(x, w, fp8)
+    nbytes, flops = workload_work(x, w, kind)
     unit, bound = metric_of(name)
     n_rep = max(2, math.ceil(1.5 * L2_BYTES / per_rep) + 1)
 
@@ -400,7 +443,17 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
         d["lse"] = torch.empty(w.batch, w.h_q, w.s_q, dtype=torch.float32, device=dev)
         reps.append(d)
 
+    def plan(d, **kw):
+        if sparse:
+            return ops.get_mla_metadata_csr(d["row_ptr"], R, w.h_kv)
+        return ops.get_mla_metadata(d["cache_seqlens"], R, w.h_kv, **kw)
+
     def decode(d, tile, splits, kernel_only=False):
+        if sparse:
+            ops.mla_decode_sparse(d["q"], d["k_cache"], d["block_table"], d["cache_seqlens"], d["row_ptr"],
+                                  d["col_idx"], 512, tile, splits, softmax_scale=w.scale, causal=w.causal,
+                                  workspace=d["ws"], out=d["out"], lse=d["lse"], skip_combine=kernel_only)
+            return
         if fp8:
             ops.mla_decode_paged_fp8(d["q"], d["k8"], d["k_scale"], d["block_table"], d["cache_seqlens"], 512, tile,
                                      splits, softmax_scale=w.scale, causal=w.causal, workspace=d["ws"],
@@ -411,7 +464,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
                              out=d["out"], lse=d["lse"], skip_combine=kernel_only, kernel=args.kernel)
 
     def step(d):
-        tile, splits = ops.get_mla_metadata(d["cache_seqlens"], R, w.h_kv)
+        tile, splits = plan(d)
         decode(d, tile, splits)
 
     # eager warm-up (first launches, allocator, tensor maps), then graph capture
@@ -433,7 +486,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
             step(reps[i % n_rep])
     with torch.cuda.stream(stream):
         for d in reps:
-            d["plan"] = ops.get_mla_metadata(d["cache_seqlens"], R, w.h_kv)
+            d["plan"] = plan(d)
     kgraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(kgraph, stream=stream):
         for i in range(args.steps):
@@ -444,13 +497,18 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     with torch.cuda.graph(mgraph, stream=stream):
         for i in range(args.steps):
             d = reps[i % n_rep]
-            ops.get_mla_metadata(d["cache_seqlens"], R, w.h_kv)
+            plan(d)
     cgraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(cgraph, stream=stream):
         for i in range(args.steps):
             d = reps[i % n_rep]
             tile, splits = d["plan"]
-            ops.mla_combine(splits, w.s_q, w.h_q, w.h_kv, tile.shape[0], d["ws"], d["out"], d["lse"])
+            if sparse:  # one-position lists: out [b * s_q, 1, h_q, 512], lse in [b, s_q, h_q] order
+                ops.mla_combine(splits, 1, w.h_q, w.h_kv, tile.shape[0], d["ws"],
+                                d["out"].view(w.batch * w.s_q, 1, w.h_q, 512),
+                                d["lse"].view(w.batch * w.s_q, w.h_q, 1))
+            else:
+                ops.mla_combine(splits, w.s_q, w.h_q, w.h_kv, tile.shape[0], d["ws"], d["out"], d["lse"])
     torch.cuda.synchronize(dev)
     graph.replay()  # first replay uploads the graph; not timed
     kgraph.replay()
@@ -505,7 +563,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
             d = reps[i % n_rep]
             flush.fill_(float(i))
             ev[n_iso + i][0].record(stream)
-            ops.get_mla_metadata(d["cache_seqlens"], R, w.h_kv)
+            plan(d)
             ev[n_iso + i][1].record(stream)
     torch.cuda.synchronize(dev)
     iso_s = max_over_ranks(statistics.median(ev[i][0].elapsed_time(ev[i][1]) for i in range(n_iso)) * 1e-3)
@@ -532,9 +590,10 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     achieved = work / kernel_s
     iso_achieved = work / iso_s
     # the summaries were taken with the library's own kernel choice
-    traffic = recorded_traffic(name, decode_kernel_for(R, w.h_q // w.h_kv)) if args.kernel == "auto" else None
+    traffic = (recorded_traffic(name, "decode_mma16_kernel" if sparse else decode_kernel_for(R, w.h_q // w.h_kv))
+               if args.kernel == "auto" else None)
     res = {
-        "workload": name, "config": workload_config(w, fp8), "unit": unit, "value": value,
+        "workload": name, "config": workload_config(w, kind), "unit": unit, "value": value,
         "ms_per_step": per_step * 1e3, "n_rep": n_rep, "per_rep_bytes": per_rep,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
                      "frac": achieved / peak, "traffic": traffic,
@@ -547,7 +606,8 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
                                          f"each after a {FLUSH_BYTES >> 20} MB L2-flush write"),
                      "frac_of_nominal": achieved / nominal, "nominal_peak": nominal,
                      "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
-                     "whole_page_bytes_per_launch": (W.whole_page_bytes(x["cache_seqlens"].tolist(), w.h_kv) *
+                     "whole_page_bytes_per_launch": (None if sparse else
+                                                     W.whole_page_bytes(x["cache_seqlens"].tolist(), w.h_kv) *
                                                      FP8_TOKEN_BYTES // (2 * 576) if fp8 else
                                                      W.whole_page_bytes(x["cache_seqlens"].tolist(), w.h_kv)),
                      "scheduler_ms": sched_s * 1e3, "scheduler_isolated_ms": iso_sched_s * 1e3,
@@ -557,7 +617,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
 
     if with_e2e:
         res["e2e"] = e2e_leg(args, w, x, reps[0], dev, nparts, R, unit, total_bytes, total_flops,
-                             barrier, max_over_ranks, fp8)
+                             barrier, max_over_ranks, kind)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and cpu_seconds > 0:
         res["cpu_baseline"] = cpu_baseline(x, w, unit, seconds=cpu_seconds)
     for g in (warm_graph, graph, kgraph, mgraph, cgraph):
@@ -567,7 +627,7 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     return res
 
 
-def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barrier, max_over_ranks, fp8=False):
+def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barrier, max_over_ranks, kind="bf16"):
     """End to end through the public API from pinned host buffers (the latent page pool is
     resident device state; each step sends q, block_table and cache_seqlens and reads back
     out and lse).  Two steps are in flight, as a serving loop would run them: step i+1's
@@ -577,9 +637,14 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
     step's copies and its result's arrival on the host are inside the timed region."""
     from paged_mla_decode_11_b200 import ops
     e2e_steps = min(args.steps, 50)
+    fp8, sparse = kind == "fp8", kind == "sparse"
     hq = x["q"].pin_memory()
     hbt = x["block_table"].pin_memory()
     hsl = x["cache_seqlens"].pin_memory()
+    # the sparse decode's key lists travel with the step's inputs
+    hrp = x["row_ptr"].pin_memory() if sparse else None
+    hci = x["col_idx"].pin_memory() if sparse else None
+    n_lists = w.batch * w.s_q if sparse else w.batch
     ws_e2e = d0["ws"]
     kstream = torch.cuda.current_stream(dev)  # the API launches on the current stream
     up_stream = torch.cuda.Stream(device=dev)
@@ -590,7 +655,9 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
             "q": torch.empty_like(d0["q"]), "bt": torch.empty_like(d0["block_table"]),
             "sl": torch.empty_like(d0["cache_seqlens"]),
             "tile": torch.empty(nparts, ops.TILE_FIELDS, dtype=torch.int32, device=dev),
-            "splits": torch.empty(w.batch + 1, dtype=torch.int32, device=dev),
+            "splits": torch.empty(n_lists + 1, dtype=torch.int32, device=dev),
+            "rp": torch.empty_like(d0["row_ptr"]) if sparse else None,
+            "ci": torch.empty_like(d0["col_idx"]) if sparse else None,
             "out": torch.empty(w.batch, w.s_q, w.h_q, 512, dtype=torch.bfloat16, device=dev),
             "lse": torch.empty(w.batch, w.h_q, w.s_q, dtype=torch.float32, device=dev),
             "hout": torch.empty(w.batch, w.s_q, w.h_q, 512, dtype=torch.bfloat16).pin_memory(),
@@ -605,19 +672,30 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
             sl_["q"].copy_(hq, non_blocking=True)
             sl_["bt"].copy_(hbt, non_blocking=True)
             sl_["sl"].copy_(hsl, non_blocking=True)
+            if sparse:
+                sl_["rp"].copy_(hrp, non_blocking=True)
+                sl_["ci"].copy_(hci, non_blocking=True)
             sl_["up"].record(up_stream)
         kstream.wait_event(sl_["up"])
         if i >= 2:
             kstream.wait_event(sl_["back"])      # step i-2's result has left this slot
         # the plan goes into this slot's buffers: the previous user of the slot (step i-2)
         # ran earlier on the same stream
-        tile, splits = ops.get_mla_metadata(sl_["sl"], R, w.h_kv, tile_metadata=sl_["tile"],
-                                            num_splits=sl_["splits"])
-        if fp8:
+        if sparse:
+            tile, splits = ops.get_mla_metadata_csr(sl_["rp"], R, w.h_kv, tile_metadata=sl_["tile"],
+                                                    num_splits=sl_["splits"])
+            ops.mla_decode_sparse(sl_["q"], d0["k_cache"], sl_["bt"], sl_["sl"], sl_["rp"], sl_["ci"], 512, tile,
+                                  splits, softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
+                                  out=sl_["out"], lse=sl_["lse"])
+        elif fp8:
+            tile, splits = ops.get_mla_metadata(sl_["sl"], R, w.h_kv, tile_metadata=sl_["tile"],
+                                                num_splits=sl_["splits"])
             ops.mla_decode_paged_fp8(sl_["q"], d0["k8"], d0["k_scale"], sl_["bt"], sl_["sl"], 512, tile, splits,
                                      softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
                                      out=sl_["out"], lse=sl_["lse"])
         else:
+            tile, splits = ops.get_mla_metadata(sl_["sl"], R, w.h_kv, tile_metadata=sl_["tile"],
+                                                num_splits=sl_["splits"])
             ops.flash_mla_with_kvcache(sl_["q"], d0["k_cache"], sl_["bt"], sl_["sl"], 512, tile, splits,
                                        softmax_scale=w.scale, causal=w.causal, workspace=ws_e2e,
                                        out=sl_["out"], lse=sl_["lse"], kernel=args.kernel)
@@ -650,6 +728,8 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
     e2e_val = (total_bytes / e2e_s / 1e9) if unit == "GB/s" else (total_flops / e2e_s / 1e12)
     hout, hlse = slots[0]["hout"], slots[0]["hlse"]
     h2d = hq.numel() * 2 + hbt.numel() * 4 + hsl.numel() * 4
+    if sparse:
+        h2d += hrp.numel() * 4 + hci.numel() * 4
     d2h = hout.numel() * 2 + hlse.numel() * 4
     return {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": e2e_s * 1e3, "steps_in_flight": 2}
@@ -669,7 +749,7 @@ def run_ours(args):
     per_workload = None
     if world == 1 and not args.no_per_workload:
         per_workload = {}
-        for name in list(W.WORKLOADS) + list(FP8_WORKLOADS):
+        for name in ALL_WORKLOADS:
             r = head if name == args.workload else measure(name, args, dev, group, rank, world,
                                                             with_e2e=False, cpu_seconds=2.0)
             per_workload[name] = {k: r[k] for k in ("config", "unit", "value", "ms_per_step", "roofline",
@@ -705,7 +785,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="memory_bound", choices=sorted(list(W.WORKLOADS) + list(FP8_WORKLOADS)))
+    ap.add_argument("--workload", default="memory_bound", choices=sorted(ALL_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -214,6 +214,48 @@ MLA_API int mla_decode_paged_fp8(const void *q, const int64_t q_strides[3], int 
                                  size_t workspace_bytes, unsigned flags, mla_stream_t stream);
 
 /*
+ * mla_get_metadata_csr -- split plan for the token-level sparse decode.  The same balanced
+ * cuts as mla_get_metadata, over n_lists key lists (one per query token, n_lists = batch *
+ * s_q) whose lengths are row_ptr[i + 1] - row_ptr[i] (row_ptr: device int32 [n_lists + 1]).
+ * rows_per_kv_head = h_q / h_kv (one query token per tile); num_parts from
+ * mla_metadata_size(n_lists, rows_per_kv_head, h_kv, ...).  tile_metadata [num_parts][8] and
+ * num_splits [n_lists + 1] as for mla_get_metadata, positions counted in list entries.
+ * Errors: MLA_ERR_ARG, MLA_ERR_CUDA.
+ */
+MLA_API int mla_get_metadata_csr(const int32_t *row_ptr, int n_lists, int rows_per_kv_head, int num_parts,
+                                 int32_t *tile_metadata, int32_t *num_splits, mla_stream_t stream);
+
+/*
+ * mla_decode_sparse -- token-level sparse decode (the Baidu page on Flash MLA, section 三.3:
+ * only the Top-K key connections of a query are kept, the pattern stored in CSR form).
+ * Query token (b, s) attends, with all its heads, to the key positions
+ * col_idx[row_ptr[b * s_q + s] .. row_ptr[b * s_q + s + 1]) of sequence b that it may see
+ * (0 <= position < L_b, and with causal the bottom-right rule: position < L_b - (s_q - 1 -
+ * s)); other entries (padding such as -1, positions past the sequence) are pruned, and a
+ * position listed twice counts twice.  A query token whose list has no visible entry gets
+ * out = 0 and lse = -inf.
+ *   row_ptr   device int32 [batch * s_q + 1], non-decreasing, row_ptr[0] = 0 not required
+ *   col_idx   device int32 [row_ptr[batch * s_q]] key positions within the sequence
+ *   tile_metadata / num_parts / num_splits: from mla_get_metadata_csr over the same row_ptr
+ * Other arguments, layouts and results as mla_decode_paged; the workspace size of
+ * mla_workspace_size(batch, s_q, h_q, h_kv, num_parts) suffices.  h_q / h_kv <= 16 (one
+ * query token's heads form a 16-row warp-MMA tile), batch * s_q <= MLA_MAX_BATCH.  flags:
+ * 0 or MLA_FLAG_SKIP_COMBINE; the partials left in the workspace are those of batch * s_q
+ * lists of one position each: mla_combine(num_splits, batch * s_q, 1, h_q, ...) merges them
+ * into out (same memory order) and writes lse in [batch, s_q, h_q] order.
+ * Key rows are fetched one token row at a time (1,152 bytes per latent head).
+ * Errors: MLA_ERR_ARG, MLA_ERR_UNSUPPORTED (d, dv, page size, more than 16 heads per latent
+ * head, not sm_100), MLA_ERR_WORKSPACE, MLA_ERR_CUDA.
+ */
+MLA_API int mla_decode_sparse(const void *q, const int64_t q_strides[3], int batch, int s_q, int h_q, int d,
+                              const void *k_cache, int64_t num_pages, int page_size, int h_kv,
+                              const int32_t *block_table, int64_t block_table_stride, const int32_t *cache_seqlens,
+                              const int32_t *row_ptr, const int32_t *col_idx, int dv,
+                              const int32_t *tile_metadata, int num_parts, const int32_t *num_splits,
+                              float softmax_scale, int causal, void *out, float *lse, void *workspace,
+                              size_t workspace_bytes, unsigned flags, mla_stream_t stream);
+
+/*
  * mla_combine -- log-sum-exp merge of split-KV partials: for every sequence with more
  * than one split and every query row, lse = ln sum_k exp(lse_k) and
  * out = sum_k exp(lse_k - lse) * o_k (partials with lse_k = -inf weigh nothing).

@@ -238,6 +238,21 @@ int mla_get_metadata(const int32_t *cache_seqlens, int batch, int rows_per_kv_he
   return MLA_OK;
 }
 
+int mla_get_metadata_csr(const int32_t *row_ptr, int n_lists, int rows_per_kv_head, int num_parts,
+                         int32_t *tile_metadata, int32_t *num_splits, mla_stream_t stream) {
+  if (!row_ptr || !tile_metadata || !num_splits) return fail(MLA_ERR_ARG, "null pointer argument");
+  if (n_lists < 1 || n_lists > MLA_MAX_BATCH)
+    return fail(MLA_ERR_ARG, "n_lists must be in [1, %d] (got %d)", MLA_MAX_BATCH, n_lists);
+  if (rows_per_kv_head < 1 || rows_per_kv_head > (1 << 20))
+    return fail(MLA_ERR_ARG, "rows_per_kv_head must be in [1, 2^20]");
+  if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
+  const int ovh = std::max(1, (rows_per_kv_head + MLA_SPLIT_OVERHEAD_ROWS - 1) / MLA_SPLIT_OVERHEAD_ROWS);
+  cudaError_t e = launch_metadata(row_ptr, n_lists, ovh, num_parts, tile_metadata, num_splits,
+                                  reinterpret_cast<cudaStream_t>(stream), true);
+  if (e != cudaSuccess) return cuda_fail(e, "metadata kernel launch");
+  return MLA_OK;
+}
+
 int mla_workspace_size(int batch, int s_q, int h_q, int h_kv, int num_parts, size_t *bytes) {
   if (!bytes) return fail(MLA_ERR_ARG, "bytes is null");
   int rc = check_common(batch, s_q, h_q, h_kv, kDV);
@@ -440,6 +455,90 @@ int mla_decode_paged_fp8(const void *q, const int64_t q_strides[3], int batch, i
   if (e != cudaSuccess) return cuda_fail(e, "fp8 decode kernel launch");
   if (!(flags & MLA_FLAG_SKIP_COMBINE)) {
     e = launch_combine(num_splits, batch, s_q, h_q, h_kv, p.lse_accum, p.o_accum, p.out, lse, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+  }
+  return MLA_OK;
+}
+
+int mla_decode_sparse(const void *q, const int64_t q_strides[3], int batch, int s_q, int h_q, int d,
+                      const void *k_cache, int64_t num_pages, int page_size, int h_kv, const int32_t *block_table,
+                      int64_t block_table_stride, const int32_t *cache_seqlens, const int32_t *row_ptr,
+                      const int32_t *col_idx, int dv, const int32_t *tile_metadata, int num_parts,
+                      const int32_t *num_splits, float softmax_scale, int causal, void *out, float *lse,
+                      void *workspace, size_t workspace_bytes, unsigned flags, mla_stream_t stream) {
+  if (!q || !q_strides || !k_cache || !block_table || !cache_seqlens || !row_ptr || !col_idx || !tile_metadata ||
+      !num_splits || !out || !lse)
+    return fail(MLA_ERR_ARG, "null pointer argument");
+  int rc = check_common(batch, s_q, h_q, h_kv, dv);
+  if (rc) return rc;
+  if (d != kD) return fail(MLA_ERR_UNSUPPORTED, "d must be %d (got %d)", kD, d);
+  if (page_size != kPage) return fail(MLA_ERR_UNSUPPORTED, "page_size must be %d (got %d)", kPage, page_size);
+  const int g = h_q / h_kv;
+  if (g > 16)
+    return fail(MLA_ERR_UNSUPPORTED, "the sparse decode takes up to 16 query heads per latent head (got %d)", g);
+  if (int64_t(batch) * s_q > MLA_MAX_BATCH)
+    return fail(MLA_ERR_ARG, "batch * s_q must be <= %d (got %lld)", MLA_MAX_BATCH, (long long)batch * s_q);
+  if (num_pages < 1 || num_pages > (int64_t(1) << 25))
+    return fail(MLA_ERR_ARG, "num_pages must be in [1, 2^25]");
+  if (block_table_stride < 1) return fail(MLA_ERR_ARG, "block_table_stride must be >= 1");
+  if (num_parts < 1) return fail(MLA_ERR_ARG, "num_parts must be >= 1");
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale))
+    return fail(MLA_ERR_ARG, "softmax_scale must be positive and finite");
+  if (flags & ~MLA_FLAG_SKIP_COMBINE) return fail(MLA_ERR_ARG, "unknown flags 0x%x", flags);
+  for (int i = 0; i < 3; ++i)
+    if (q_strides[i] < 0 || q_strides[i] % 8 != 0)
+      return fail(MLA_ERR_ARG, "q strides must be non-negative multiples of 8 elements");
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return fail(MLA_ERR_ARG, "q, k_cache and out must be 16-byte aligned, lse 4-byte aligned");
+  rc = check_device();
+  if (rc) return rc;
+  const int n_tok = batch * s_q;
+  const WorkspaceLayout wl = workspace_layout(n_tok, g, h_kv, num_parts);
+  if (!workspace) return fail(MLA_ERR_WORKSPACE, "workspace is null");
+  if (!aligned(workspace, 256)) return fail(MLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (workspace_bytes < wl.total)
+    return fail(MLA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", workspace_bytes, wl.total);
+
+  // one query token per tile: all g heads of position s of sequence b
+  CUtensorMap qmap;
+  rc = encode_q_map(&qmap, q, batch, s_q, h_q, g, 1, q_strides);
+  if (rc) return rc;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.q_sb = q_strides[0];
+  p.q_ss = q_strides[1];
+  p.q_sh = q_strides[2];
+  p.batch = n_tok;  // query tokens are the tile "sequences"
+  p.s_q = 1;
+  p.h_q = h_q;
+  p.h_kv = h_kv;
+  p.g = g;
+  p.R = g;
+  p.block_table = block_table;
+  p.bt_stride = block_table_stride;
+  p.kv_base = static_cast<const uint8_t *>(k_cache);
+  p.kv_token_bytes = int64_t(h_kv) * kD * 2;
+  p.seqlens = cache_seqlens;
+  p.tile_md = tile_metadata;
+  p.num_parts = num_parts;
+  p.num_splits = num_splits;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.out = static_cast<__nv_bfloat16 *>(out);
+  p.lse = lse;
+  p.lse_accum = reinterpret_cast<float *>(ws + wl.lse_off);
+  p.o_accum = reinterpret_cast<float *>(ws + wl.o_off);
+  p.status = reinterpret_cast<int *>(ws);
+  p.watchdog_ns = kWatchdogNs;
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.sq_fold = s_q;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_decode_sparse16(qmap, p, st);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse decode kernel launch");
+  if (!(flags & MLA_FLAG_SKIP_COMBINE)) {
+    e = launch_combine(num_splits, n_tok, 1, h_q, h_kv, p.lse_accum, p.o_accum, p.out, lse, st, s_q);
     if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
   }
   return MLA_OK;

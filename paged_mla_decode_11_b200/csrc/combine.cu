@@ -21,7 +21,7 @@ constexpr int kBatch = 8;                  // splits whose partial rows are load
 
 // 4 CTAs per SM bound the registers to 128 per thread (eight splits' rows in flight).
 __global__ void __launch_bounds__(kCombineWarps * 32, 4)
-    combine_kernel(const int32_t *__restrict__ num_splits, int s_q, int h_q, int h_kv, int R,
+    combine_kernel(const int32_t *__restrict__ num_splits, int s_q, int h_q, int h_kv, int R, int sq_fold,
                    const float *__restrict__ lse_accum, const float *__restrict__ o_accum,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
   // the next kernel may start its prologue; the scheduler kernel of a next step computes its
@@ -107,16 +107,18 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 4)
     u.y = pack_bf16x2(acc[i].z, acc[i].w);
     *reinterpret_cast<uint2 *>(dst + 4 * (lane + 32 * i)) = u;
   }
-  if (lane == 0 && half == 0) lse[(int64_t(b) * h_q + h) * s_q + s] = tot;
+  // sq_fold > 1 (sparse decode): "sequence" b is query token b % sq_fold of sequence b / sq_fold
+  if (lane == 0 && half == 0)
+    lse[(int64_t(b / sq_fold) * h_q + h) * (int64_t(s_q) * sq_fold) + int64_t(b % sq_fold) * s_q + s] = tot;
 }
 
 cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_q, int h_kv,
                            const float *lse_accum, const float *o_accum, __nv_bfloat16 *out,
-                           float *lse, cudaStream_t stream) {
+                           float *lse, cudaStream_t stream, int sq_fold) {
   const int R = s_q * (h_q / h_kv);
   dim3 grid((R + kCombineWarps / 2 - 1) / (kCombineWarps / 2), batch, h_kv);
   return launch_early(combine_kernel, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv, R,
-                      lse_accum, o_accum, out, lse);
+                      sq_fold, lse_accum, o_accum, out, lse);
 }
 
 // A CTA that waits on a barrier nothing completes, with the decode kernels' bounded

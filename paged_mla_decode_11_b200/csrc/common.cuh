@@ -43,7 +43,19 @@ struct DecodeParams {
   float *o_accum;                  // [splits, h_kv, R, 512]
   int *status;                     // workspace status block
   unsigned long long watchdog_ns;  // limit of every device-side wait
+  // token-level sparse decode only: "sequence" index i = b * sq_fold + s is one query token,
+  // whose keys are the positions col_idx[row_ptr[i] .. row_ptr[i + 1]) of sequence b
+  const int32_t *row_ptr = nullptr;
+  const int32_t *col_idx = nullptr;
+  int sq_fold = 1;
 };
+
+// Index of (query-tile "sequence" seq, position sq, head h) in lse [batch, h_q, s_q]: with
+// sq_fold > 1 a tile sequence is one query token of a real sequence (seq / sq_fold).
+__device__ __forceinline__ int64_t lse_index(const DecodeParams &p, int seq, int sq, int h) {
+  const int f = p.sq_fold;
+  return (int64_t(seq / f) * p.h_q + h) * (int64_t(p.s_q) * f) + int64_t(seq % f) * p.s_q + sq;
+}
 
 // ------------------------------------------------------------------------------------
 // Timers and the watchdog.
@@ -149,6 +161,17 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
       "[%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+
+// One contiguous copy global -> shared (untiled bulk copy; both addresses 16-byte aligned,
+// bytes a multiple of 16), completing on an mbarrier of this CTA.
+__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                               uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
 }
 

@@ -360,15 +360,23 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
 // Each hand-off is a producer/consumer named barrier pair (full / empty), so the S warps
 // run up to two chunks ahead of the softmax, which runs up to two chunks ahead of PV.
 // ---------------------------------------------------------------------------------------
-struct Mma16 {
+// Sparse variant (kSparse): the keys of a chunk are 32 listed token rows of one query token,
+// gathered row by row with untiled bulk copies into a row-major chunk (rows of 576 bf16
+// padded to 1,168 bytes, so that 8 consecutive rows of a ldmatrix fall in distinct banks);
+// the producer also records which of the 32 entries are real keys (a validity mask).
+template <bool kSparse>
+struct Mma16T {
   static constexpr int KC = 32;                           // keys per chunk
   static constexpr int NS = 5;                            // ring depth
   static constexpr int kSWarps = 4, kSmWarp = 4, kPVWarp0 = 5, kPVWarps = 4, kProducer = 9;
   static constexpr int kThreads = 10 * 32;
   static constexpr int kChunkBlock = KC * 128;            // one 64-column block: 4 KB
-  static constexpr int kChunkBytes = kColBlocks * kChunkBlock;
+  static constexpr int kChunkBytes = kColBlocks * kChunkBlock;  // bytes a chunk's copies deliver
+  static constexpr int kRowBytes = kD * 2 + 16;           // sparse: padded row of a chunk
+  // ring slot stride (1 KB multiple, so that the Q tile after the ring stays 1 KB aligned)
+  static constexpr int kSlotBytes = kSparse ? (KC * kRowBytes + 1023) / 1024 * 1024 : kChunkBytes;
   static constexpr int kOffRing = 0;
-  static constexpr int kOffQ = NS * kChunkBytes;          // 16 rows x 576, 9 blocks of 2 KB
+  static constexpr int kOffQ = NS * kSlotBytes;           // 16 rows x 576, 9 blocks of 2 KB
   static constexpr int kOffP = kOffQ + kColBlocks * 16 * 128;   // 2 x [16 rows x 32 keys] bf16
   static constexpr int kOffS = kOffP + 2 * 16 * 128;            // 2 x [4 warps][8][32] f32 partial S
   static constexpr int kOffAlpha = kOffS + 2 * 4 * 8 * 32 * 4;  // alpha[2][16]
@@ -377,30 +385,42 @@ struct Mma16 {
   static constexpr int kOffBar = kOffM + 2 * 16 * 4;
   enum { FULL = 0, EMPTY = FULL + NS, QFULL = EMPTY + NS, QFREE = QFULL + 1, NBARS = QFREE + 1 };
   static constexpr int kOffAbort = kOffBar + NBARS * 8;
-  static constexpr int kSmemBytes = kOffAbort + 16 + 1024;
+  static constexpr int kOffMask = kOffAbort + 16;          // sparse: vmask[NS] (per slot), smask[2]
+  static constexpr int kSmemBytes = kOffMask + (NS + 2) * 4 + 1024;
   // named barriers (id, id + 1 for the two buffers): S tile full / empty, P tile full / empty
   static constexpr int kBarSFull = 1, kBarSEmpty = 3, kBarPFull = 5, kBarPEmpty = 7;
   static constexpr int kSPair = (kSWarps + 1) * 32, kPPair = (kPVWarps + 1) * 32;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+  // Shared address of 16-byte column chunk col16 (0..71) of key row `row` of a ring chunk:
+  // nine 128-byte-swizzled 32-row column blocks (tiled TMA), or padded rows (sparse).
+  static __device__ __forceinline__ uint32_t key_addr(uint32_t chunk, int row, int col16) {
+    if constexpr (kSparse) return chunk + row * kRowBytes + col16 * 16;
+    else return chunk + (col16 >> 3) * kChunkBlock + sw128(row, col16 & 7);
+  }
 };
+using Mma16 = Mma16T<false>;
 
 __device__ __forceinline__ void named_bar_arrive(int id, int nthreads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Token range and 32-key chunk count of sequence `seq` within part `pc`.
+// Token range and 32-key chunk count of sequence `seq` within part `pc` (sparse: the range of
+// entries of query token `seq`'s key list).
+template <bool kSparse = false>
 __device__ __forceinline__ int chunk_range(const DecodeParams &p, const PartCursor &pc, int seq, int &L,
                                            int &t0, int &t1) {
-  L = p.seqlens[seq];
+  L = kSparse ? p.row_ptr[seq + 1] - p.row_ptr[seq] : p.seqlens[seq];
   t0 = seq == pc.bi ? pc.bt : 0;
   t1 = seq == pc.ei ? pc.et : L;
   return t1 > t0 ? (t1 - t0 + Mma16::KC - 1) / Mma16::KC : 0;
 }
 
+template <bool kSparse>
 __global__ void __launch_bounds__(Mma16::kThreads, 1)
     decode_mma16_kernel(const __grid_constant__ CUtensorMap kv_map,
                         const __grid_constant__ CUtensorMap q_map, const DecodeParams p) {
-  using T = Mma16;
+  using T = Mma16T<kSparse>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -415,6 +435,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
   float *alpha_sm = reinterpret_cast<float *>(smem + T::kOffAlpha);
   float *l_sm = reinterpret_cast<float *>(smem + T::kOffL);
   float *m_sm = reinterpret_cast<float *>(smem + T::kOffM);
+  uint32_t *vmask = reinterpret_cast<uint32_t *>(smem + T::kOffMask);  // [NS], then smask[2]
   const unsigned long long lim_ns = p.watchdog_ns;
 
   if (threadIdx.x == 0) {
@@ -446,7 +467,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
     bool ok = true;
     for (int seq = pc.bi; ok && part_has(pc, seq); ++seq) {
       int L, t0, t1;
-      const int nch = chunk_range(p, pc, seq, L, t0, t1);
+      const int nch = chunk_range<kSparse>(p, pc, seq, L, t0, t1);
       if (nch == 0) continue;
       int good = 1;
       if (lane == 0) {
@@ -455,13 +476,79 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
         } else {
           mbar_arrive_expect_tx(bar(T::QFULL), uint32_t(kColBlocks * p.R * 128));
 #pragma unroll
-          for (int c = 0; c < kColBlocks; ++c)
-            tma_load_4d(sQ + c * 16 * 128, &q_map, bar(T::QFULL), c * 64, kvh * p.g, 0, seq);
+          for (int c = 0; c < kColBlocks; ++c) {
+            if constexpr (kSparse)  // one query token: position seq % s_q of sequence seq / s_q
+              tma_load_4d(sQ + c * 16 * 128, &q_map, bar(T::QFULL), c * 64, kvh * p.g, seq % p.sq_fold,
+                          seq / p.sq_fold);
+            else
+              tma_load_4d(sQ + c * 16 * 128, &q_map, bar(T::QFULL), c * 64, kvh * p.g, 0, seq);
+          }
           last_q = qs;
         }
       }
       ok = __shfl_sync(0xffffffffu, good, 0) != 0;
       ++qs;
+      if constexpr (kSparse) {
+        // Entry t0 + 32 n + lane of the list goes to row `lane` of chunk n.  Lists are read four
+        // chunks at a time (one coalesced index load and one block-table load per lane and
+        // chunk), the next group's indices while the current group's copies are issued.
+        const int b = seq / p.sq_fold, sq = seq % p.sq_fold;
+        const int Lb = p.seqlens[b];
+        const int nvis = p.causal ? Lb - (p.sq_fold - 1 - sq) : Lb;
+        const int32_t *list = p.col_idx + p.row_ptr[seq];
+        const int32_t *bt = p.block_table + (int64_t)b * p.bt_stride;
+        auto fetch = [&](int grp, int (&idx)[4]) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int e = t0 + (grp * 4 + k) * T::KC + lane;
+            idx[k] = e < t1 ? list[e] : -1;
+          }
+        };
+        // a pruned entry copies token 0 of page 0 (finite data; its score is masked)
+        auto resolve = [&](const int (&idx)[4], const uint8_t *(&src)[4], unsigned &valid) {
+          valid = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const bool v = idx[k] >= 0 && idx[k] < nvis;
+            const int64_t phys = v ? bt[idx[k] / kPage] : 0;
+            const int64_t row = phys * kPage + (v ? idx[k] % kPage : 0);
+            src[k] = p.kv_base + (row * p.h_kv + kvh) * (kD * 2);
+            valid |= unsigned(v) << k;
+          }
+        };
+        const int ngrp = (nch + 3) / 4;
+        int idx[4];
+        const uint8_t *src[4];
+        unsigned valid;
+        fetch(0, idx);
+        resolve(idx, src, valid);
+        for (int grp = 0; ok && grp < ngrp; ++grp) {
+          if (grp + 1 < ngrp) fetch(grp + 1, idx);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int n = grp * 4 + k;
+            if (!ok || n >= nch) break;
+            const unsigned vm = __ballot_sync(0xffffffffu, (valid >> k) & 1u);
+            const int s = it % T::NS;
+            int g2 = 1;
+            if (lane == 0) {
+              if (!mbar_wait(bar(T::EMPTY + s), ((it / T::NS) & 1) ^ 1, abort, p.status, lim_ns)) {
+                g2 = 0;
+              } else {
+                vmask[s] = vm;
+                mbar_arrive_expect_tx(bar(T::FULL + s), T::KC * kD * 2);
+                last_chunk[s] = it;
+              }
+            }
+            ok = __shfl_sync(0xffffffffu, g2, 0) != 0;
+            if (ok) bulk_load_hint(sRing + s * T::kSlotBytes + lane * T::kRowBytes, src[k], kD * 2,
+                                   bar(T::FULL + s), policy);
+            ++it;
+          }
+          if (grp + 1 < ngrp) resolve(idx, src, valid);
+        }
+        continue;
+      }
       const int32_t *bt_row = p.block_table + (int64_t)seq * p.bt_stride + t0 / kPage;
       for (int base = 0; ok && base < nch; base += 32) {
         const int mine = base + lane < nch ? bt_row[(base + lane) >> 1] : 0;
@@ -475,7 +562,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
               g2 = 0;
             } else {
               mbar_arrive_expect_tx(bar(T::FULL + s), T::kChunkBytes);
-              const uint32_t dst = sRing + s * T::kChunkBytes;
+              const uint32_t dst = sRing + s * T::kSlotBytes;
               const int row = phys * kPage + ((base + i) & 1) * T::KC;
 #pragma unroll
               for (int c = 0; c < kColBlocks; ++c)
@@ -503,7 +590,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
       int L, t0, t1;
-      const int nch = chunk_range(p, pc, seq, L, t0, t1);
+      const int nch = chunk_range<kSparse>(p, pc, seq, L, t0, t1);
       if (nch == 0) continue;
       ok = ok && mbar_wait(bar(T::QFULL), qs & 1, abort, p.status, lim_ns);
       if (ok) {
@@ -522,11 +609,10 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
         float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         if (ok) {
           // key fragments loaded one k-step ahead; four independent accumulator chains
-          const uint32_t chunk = sRing + (it % T::NS) * T::kChunkBytes;
+          const uint32_t chunk = sRing + (it % T::NS) * T::kSlotBytes;
           float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
           auto kaddr = [&](int k) {
-            return chunk + (k >> 2) * T::kChunkBlock +
-                   sw128(kn * 16 + (lane & 7) + (lane >> 4) * 8, (k & 3) * 2 + ((lane >> 3) & 1));
+            return T::key_addr(chunk, kn * 16 + (lane & 7) + (lane >> 4) * 8, 2 * k + ((lane >> 3) & 1));
           };
           uint32_t b[2][4];
           ldsm_x4(kaddr(kh * (kD / 32)), b[0][0], b[0][1], b[0][2], b[0][3]);
@@ -547,6 +633,8 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
           }
         }
         if (it >= 2) named_bar_sync(T::kBarSEmpty + sb, T::kSPair);
+        // the chunk's validity mask travels with the S tile (read after this warp's FULL wait)
+        if (kSparse && warp == 0 && lane == 0) vmask[T::NS + sb] = ok ? vmask[it % T::NS] : 0u;
         float *dst = sbuf + (sb * 4 + warp) * 8 * 32;
 #pragma unroll
         for (int e = 0; e < 8; ++e) dst[e * 32 + lane] = sc[e >> 2][e & 3];
@@ -560,7 +648,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
     int it = 0, qs = 0;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
       int L, t0, t1;
-      const int nch = chunk_range(p, pc, seq, L, t0, t1);
+      const int nch = chunk_range<kSparse>(p, pc, seq, L, t0, t1);
       if (nch == 0) continue;
       int lim[2];
 #pragma unroll
@@ -580,6 +668,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             sc[kn][e] = src[(kn * 8 + e) * 32 + lane] + src[((2 + kn) * 8 + e) * 32 + lane];
+        const unsigned vm = kSparse ? vmask[T::NS + sb] : 0u;
         named_bar_arrive(T::kBarSEmpty + sb, T::kSPair);
         float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -587,8 +676,9 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int r = (e >> 1) & 1;
-            const int key = t0 + n * T::KC + kn * 16 + (e >> 2) * 8 + c4 * 2 + (e & 1);
-            const float v = key < lim[r] ? sc[kn][e] * p.scale_log2 : -INFINITY;
+            const int kc = kn * 16 + (e >> 2) * 8 + c4 * 2 + (e & 1);
+            const bool vis = kSparse ? (lim[r] >= 0 && ((vm >> kc) & 1u)) : t0 + n * T::KC + kc < lim[r];
+            const float v = vis ? sc[kn][e] * p.scale_log2 : -INFINITY;
             sc[kn][e] = v;
             mx[r] = fmaxf(mx[r], v);
           }
@@ -650,7 +740,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
       int L, t0, t1;
-      const int nch = chunk_range(p, pc, seq, L, t0, t1);
+      const int nch = chunk_range<kSparse>(p, pc, seq, L, t0, t1);
       const int ns0 = split_base(p.num_splits, seq);
       const int nsplit = split_base(p.num_splits, seq + 1) - ns0;
       const int ord = seq == pc.bi ? pc.bord : 0;
@@ -667,7 +757,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
         }
         if (tid < p.R) {
           if (nsplit == 1)
-            p.lse[((int64_t)seq * p.h_q + kvh * p.g + tid % p.g) * p.s_q + tid / p.g] = -INFINITY;
+            p.lse[lse_index(p, seq, tid / p.g, kvh * p.g + tid % p.g)] = -INFINITY;
           else
             p.lse_accum[acc_row0 + tid] = -INFINITY;
         }
@@ -696,7 +786,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
           o[j][2] *= a1;
           o[j][3] *= a1;
         }
-        const uint32_t chunk = sRing + s * T::kChunkBytes;
+        const uint32_t chunk = sRing + s * T::kSlotBytes;
         const uint32_t ptile = sP + pb * (16 * 128);
         ok = ok && !*abort;
         if (ok) {
@@ -709,8 +799,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
 #pragma unroll
             for (int jp = 0; jp < 8; ++jp) {
               const int dv0 = v * 128 + jp * 16;
-              ldsm_x4_t(chunk + (dv0 / 64) * T::kChunkBlock + sw128(key, (dv0 % 64) / 8 + (lane >> 4)), b[jp][0],
-                        b[jp][1], b[jp][2], b[jp][3]);
+              ldsm_x4_t(T::key_addr(chunk, key, dv0 / 8 + (lane >> 4)), b[jp][0], b[jp][1], b[jp][2], b[jp][3]);
             }
 #pragma unroll
             for (int jp = 0; jp < 8; ++jp) {
@@ -736,7 +825,7 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             *reinterpret_cast<uint32_t *>(orow + j * 8) = pack_bf16x2(o[j][2 * r] * inv, o[j][2 * r + 1] * inv);
-          if (v == 0 && c4 == 0) p.lse[((int64_t)seq * p.h_q + h) * p.s_q + sq] = lse_v;
+          if (v == 0 && c4 == 0) p.lse[lse_index(p, seq, sq, h)] = lse_v;
         } else {
           float *orow = p.o_accum + (acc_row0 + row) * kDV + v * 128 + c4 * 2;
 #pragma unroll
@@ -754,11 +843,20 @@ __global__ void __launch_bounds__(Mma16::kThreads, 1)
 
 cudaError_t launch_decode_mma16(const CUtensorMap &kv_map, const CUtensorMap &q_map, const DecodeParams &p,
                                 cudaStream_t stream) {
-  using T = Mma16;
-  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(decode_mma16_kernel), T::kSmemBytes);
+  using T = Mma16T<false>;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(decode_mma16_kernel<false>), T::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_parts, 1, p.h_kv);
-  return launch_early(decode_mma16_kernel, grid, dim3(T::kThreads), T::kSmemBytes, stream, kv_map, q_map, p);
+  return launch_early(decode_mma16_kernel<false>, grid, dim3(T::kThreads), T::kSmemBytes, stream, kv_map, q_map, p);
+}
+
+cudaError_t launch_decode_sparse16(const CUtensorMap &q_map, const DecodeParams &p, cudaStream_t stream) {
+  using T = Mma16T<true>;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(decode_mma16_kernel<true>), T::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.num_parts, 1, p.h_kv);
+  // the key rows are addressed through p.kv_base; the tensor-map slot is unused
+  return launch_early(decode_mma16_kernel<true>, grid, dim3(T::kThreads), T::kSmemBytes, stream, q_map, q_map, p);
 }
 
 template <int BM, int DVS>

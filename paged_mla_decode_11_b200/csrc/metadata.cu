@@ -44,9 +44,12 @@ __device__ long long block_exclusive_scan(long long v, long long *scratch, long 
   return before + incl - v;
 }
 
+template <bool kOffsets>
 __global__ void __launch_bounds__(kMetaThreads)
     metadata_kernel(const int32_t *__restrict__ seqlens, int batch, int ovh, int num_parts,
                     int32_t *__restrict__ tile_md, int32_t *__restrict__ num_splits) {
+  // length of sequence b: an entry, or the difference of two offsets (a CSR row_ptr)
+  auto len = [&](int b) { return kOffsets ? seqlens[b + 1] - seqlens[b] : seqlens[b]; };
   extern __shared__ long long start[];  // [batch + 1]
   __shared__ long long scratch[32];
   grid_launch_dependents();  // the decode kernel may start its prologue now
@@ -55,12 +58,12 @@ __global__ void __launch_bounds__(kMetaThreads)
 
   // 1. start_b = exclusive prefix sum of (OVH + pages_b)
   long long mine = 0;
-  for (int b = lo; b < hi; ++b) mine += ovh + (max(seqlens[b], 0) + kPage - 1) / kPage;
+  for (int b = lo; b < hi; ++b) mine += ovh + (max(len(b), 0) + kPage - 1) / kPage;
   long long total;
   long long run = block_exclusive_scan(mine, scratch, &total);
   for (int b = lo; b < hi; ++b) {
     start[b] = run;
-    run += ovh + (max(seqlens[b], 0) + kPage - 1) / kPage;
+    run += ovh + (max(len(b), 0) + kPage - 1) / kPage;
   }
   if (threadIdx.x == 0) start[batch] = total;
   __syncthreads();
@@ -131,16 +134,16 @@ __global__ void __launch_bounds__(kMetaThreads)
 }
 
 cudaError_t launch_metadata(const int32_t *seqlens, int batch, int ovh, int num_parts, int32_t *tile_md,
-                            int32_t *num_splits, cudaStream_t stream) {
+                            int32_t *num_splits, cudaStream_t stream, bool lengths_are_offsets) {
   const size_t smem = size_t(batch + 1) * sizeof(long long);
+  auto kern = lengths_are_offsets ? metadata_kernel<true> : metadata_kernel<false>;
   if (smem > 48 * 1024) {
-    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(metadata_kernel),
-                                  int((MLA_MAX_BATCH + 1) * sizeof(long long)));
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), int((MLA_MAX_BATCH + 1) * sizeof(long long)));
     if (e != cudaSuccess) return e;
   }
   // launched early: the plan is computed while the previous kernel finishes (see above)
-  return launch_early(metadata_kernel, dim3(1), dim3(kMetaThreads), smem, stream, seqlens, batch, ovh, num_parts,
-                      tile_md, num_splits);
+  return launch_early(kern, dim3(1), dim3(kMetaThreads), smem, stream, seqlens, batch, ovh, num_parts, tile_md,
+                      num_splits);
 }
 
 }  // namespace pagedmla

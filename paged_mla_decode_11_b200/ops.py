@@ -41,7 +41,7 @@ EXPORTED = (
     "mla_device_sm_count", "mla_num_parts", "mla_metadata_size", "mla_get_metadata", "mla_workspace_size",
     "mla_decode_paged", "mla_combine", "mla_query_status", "mla_watchdog_selftest",
     "mla_last_error_string", "mla_decode_paged_static", "mla_query_status_static", "mla_decode_paged_fp8",
-    "mla_merge_partials", "mla_absorb_query", "mla_absorb_output",
+    "mla_merge_partials", "mla_absorb_query", "mla_absorb_output", "mla_get_metadata_csr", "mla_decode_sparse",
 )
 
 _lib = None
@@ -85,6 +85,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "mla_absorb_output": [P, P, P, I, I, P, P],
             "mla_decode_paged_fp8": [P, P, I, I, I, I, P, P, I64, I, I, P, I64, P, I, P, I, P,
                                      ctypes.c_float, I, P, P, P, ctypes.c_size_t, ctypes.c_uint, P],
+            "mla_get_metadata_csr": [P, I, I, I, P, P, P],
+            "mla_decode_sparse": [P, P, I, I, I, I, P, I64, I, I, P, I64, P, P, P, I, P, I, P,
+                                  ctypes.c_float, I, P, P, P, ctypes.c_size_t, ctypes.c_uint, P],
         }
         for name, args in sig.items():
             fn = getattr(lib, name)
@@ -180,6 +183,33 @@ def get_mla_metadata(cache_seqlens: torch.Tensor, rows_per_kv_head: int, h_kv: i
             raise ValueError("num_splits must be a contiguous [batch + 1] tensor")
     _check(load_library().mla_get_metadata(cache_seqlens.data_ptr(), batch, rows_per_kv_head, num_parts,
                                            tile_metadata.data_ptr(), num_splits.data_ptr(), _stream_ptr(dev)))
+    return tile_metadata, num_splits
+
+
+def get_mla_metadata_csr(row_ptr: torch.Tensor, rows_per_kv_head: int, h_kv: int,
+                         num_parts: Optional[int] = None, tile_metadata: Optional[torch.Tensor] = None,
+                         num_splits: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split plan for the token-level sparse decode: the balanced cuts over key lists whose
+    lengths are the differences of ``row_ptr`` (contiguous int32 [n_lists + 1], one list per
+    query token).  rows_per_kv_head = h_q / h_kv.  Returns (tile_metadata [num_parts, 8],
+    num_splits [n_lists + 1]); buffers may be passed for reuse as in get_mla_metadata."""
+    _require_cuda(row_ptr, "row_ptr", torch.int32)
+    if row_ptr.dim() != 1 or row_ptr.numel() < 2 or not row_ptr.is_contiguous():
+        raise ValueError("row_ptr must be a contiguous 1-D int32 tensor of n_lists + 1 offsets")
+    dev = row_ptr.device
+    n_lists = row_ptr.numel() - 1
+    if num_parts is None:
+        num_parts = num_parts_for(device_sm_count(dev), rows_per_kv_head, h_kv)
+    if tile_metadata is None:
+        tile_metadata = torch.empty(num_parts, TILE_FIELDS, dtype=torch.int32, device=dev)
+    elif tile_metadata.shape != (num_parts, TILE_FIELDS) or not tile_metadata.is_contiguous():
+        raise ValueError(f"tile_metadata must be a contiguous [{num_parts}, {TILE_FIELDS}] tensor")
+    if num_splits is None:
+        num_splits = torch.empty(n_lists + 1, dtype=torch.int32, device=dev)
+    elif num_splits.shape != (n_lists + 1,) or not num_splits.is_contiguous():
+        raise ValueError("num_splits must be a contiguous [n_lists + 1] tensor")
+    _check(load_library().mla_get_metadata_csr(row_ptr.data_ptr(), n_lists, rows_per_kv_head, num_parts,
+                                               tile_metadata.data_ptr(), num_splits.data_ptr(), _stream_ptr(dev)))
     return tile_metadata, num_splits
 
 
@@ -354,6 +384,66 @@ def mla_combine(num_splits: torch.Tensor, s_q: int, h_q: int, h_kv: int, num_par
     _check(load_library().mla_combine(num_splits.data_ptr(), b, s_q, h_q, h_kv, dv, num_parts,
                                       workspace.data_ptr(), workspace.numel(), out.data_ptr(),
                                       lse.data_ptr(), _stream_ptr(out.device)))
+
+
+def mla_decode_sparse(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor,
+                      cache_seqlens: torch.Tensor, row_ptr: torch.Tensor, col_idx: torch.Tensor, dv: int,
+                      tile_metadata: torch.Tensor, num_splits: torch.Tensor,
+                      softmax_scale: Optional[float] = None, causal: bool = False,
+                      workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                      lse: Optional[torch.Tensor] = None, skip_combine: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Token-level sparse decode: query token (b, s) attends to the key positions
+    col_idx[row_ptr[b * s_q + s] : row_ptr[b * s_q + s + 1]] of sequence b that it may see
+    (others pruned).  row_ptr int32 [b * s_q + 1], col_idx int32 [nnz]; the plan comes from
+    get_mla_metadata_csr(row_ptr, h_q // h_kv, h_kv).  Up to 16 query heads per latent head.
+    Other arguments and results as mla_decode_paged; with skip_combine the split partials stay
+    in the workspace (mla_combine over batch * s_q one-position lists merges them)."""
+    for t, n in ((q, "q"), (k_cache, "k_cache")):
+        _require_cuda(t, n, torch.bfloat16)
+    for t, n in ((block_table, "block_table"), (cache_seqlens, "cache_seqlens"), (row_ptr, "row_ptr"),
+                 (col_idx, "col_idx"), (tile_metadata, "tile_metadata"), (num_splits, "num_splits")):
+        _require_cuda(t, n, torch.int32)
+    if q.dim() != 4 or k_cache.dim() != 4 or block_table.dim() != 2:
+        raise ValueError("q and k_cache must be 4-D, block_table 2-D")
+    b, s_q, h_q, d = q.shape
+    num_pages, page, h_kv, d2 = k_cache.shape
+    if d2 != d:
+        raise ValueError("q and k_cache disagree on the latent width")
+    if q.stride(3) != 1 or not k_cache.is_contiguous():
+        raise ValueError("q's last dimension and k_cache must be contiguous")
+    if block_table.stride(1) != 1 or block_table.shape[0] != b:
+        raise ValueError("block_table must be [batch, max_pages] with contiguous rows")
+    if cache_seqlens.shape != (b,) or not cache_seqlens.is_contiguous():
+        raise ValueError("cache_seqlens must be a contiguous [batch] tensor")
+    if row_ptr.shape != (b * s_q + 1,) or not row_ptr.is_contiguous() or not col_idx.is_contiguous():
+        raise ValueError("row_ptr must be a contiguous [batch * s_q + 1] tensor, col_idx contiguous")
+    tshape = tile_metadata.shape
+    if len(tshape) != 2 or tshape[1] != TILE_FIELDS or not tile_metadata.is_contiguous():
+        raise ValueError("tile_metadata must be a contiguous [num_parts, 8] tensor")
+    if num_splits.shape != (b * s_q + 1,):
+        raise ValueError("num_splits must be [batch * s_q + 1]")
+    dev = q.device
+    num_parts = tshape[0]
+    scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    if out is None:
+        out = torch.empty(b, s_q, h_q, dv, dtype=torch.bfloat16, device=dev)
+    elif out.shape != (b, s_q, h_q, dv) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 [b, s_q, h_q, dv] tensor")
+    if lse is None:
+        lse = torch.empty(b, h_q, s_q, dtype=torch.float32, device=dev)
+    elif lse.shape != (b, h_q, s_q) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [b, h_q, s_q] tensor")
+    if workspace is None:
+        workspace = _default_workspace(workspace_size(b, s_q, h_q, h_kv, num_parts), dev)
+    col = col_idx if col_idx.numel() > 0 else torch.zeros(1, dtype=torch.int32, device=dev)
+    qst = q.stride()
+    _check(load_library().mla_decode_sparse(
+        q.data_ptr(), _I64x3(qst[0], qst[1], qst[2]), b, s_q, h_q, d, k_cache.data_ptr(), num_pages, page, h_kv,
+        block_table.data_ptr(), block_table.stride(0), cache_seqlens.data_ptr(), row_ptr.data_ptr(), col.data_ptr(),
+        dv, tile_metadata.data_ptr(), num_parts, num_splits.data_ptr(), scale, int(bool(causal)), out.data_ptr(),
+        lse.data_ptr(), workspace.data_ptr(), workspace.numel(), MLA_FLAG_SKIP_COMBINE if skip_combine else 0,
+        _stream_ptr(dev)))
+    return out, lse
 
 
 def mla_merge_partials(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: Optional[torch.Tensor] = None,
