@@ -12,8 +12,11 @@
 //   - a chunk is 5 TMA boxes of 128 code columns x 32 tokens (128-byte swizzle; the last
 //     box's columns 576-639 lie outside the tensor and are filled with zeros) plus one box of
 //     the chunk's 32 scales;
-//   - codes become bf16 in registers (E4M3 -> f16 with cvt.rn.f16x2.e4m3x2, exact; f16 ->
-//     bf16 through fp32, exact for every E4M3 value), so Q, P and both MMAs stay bf16;
+//   - both MMAs run in f16 on the codes' exact f16 form (cvt.rn.f16x2.e4m3x2: one conversion
+//     per two codes, every E4M3 value being an f16 value); the query tile is carried in f16
+//     after a power-of-two scale of the tile (its largest |q| in [2^14, 2^15)), and P times
+//     the key scale in f16 after a power-of-two scale of the chunk (every product below
+//     2^15), the accumulator carrying that factor from chunk to chunk through the rescale;
 //   - score: ldmatrix (no transpose) of a code tile gives each thread 4 consecutive columns
 //     of one key, which is the B fragment of m16n8k16 up to a permutation of the 16 K
 //     columns of each step; the Q fragments are read with the same permutation;
@@ -46,7 +49,8 @@ struct Fp8x16 {
   static constexpr int kOffAlpha = kOffS + 2 * 4 * 8 * 32 * 4;  // alpha[2][16]
   static constexpr int kOffL = kOffAlpha + 2 * 16 * 4;          // l[2 segs][16]
   static constexpr int kOffM = kOffL + 2 * 16 * 4;              // m[2 segs][16]
-  static constexpr int kOffBar = kOffM + 2 * 16 * 4;
+  static constexpr int kOffT = kOffM + 2 * 16 * 4;              // 2^-t of a segment's last chunk [2]
+  static constexpr int kOffBar = kOffT + 16;
   enum { FULL = 0, EMPTY = FULL + NS, QFULL = EMPTY + NS, QFREE = QFULL + 1, NBARS = QFREE + 1 };
   static constexpr int kOffAbort = kOffBar + NBARS * 8;
   static constexpr int kSmemBytes = kOffAbort + 16 + 1024;
@@ -61,13 +65,27 @@ __device__ __forceinline__ void fp8_bar_arrive(int id, int nthreads) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Two E4M3 codes (low byte first) -> bf16x2 (low half first), exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes) {
-  uint32_t h2;
-  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h2) : "r"(two_codes));
-  const __half2 hh = *reinterpret_cast<const __half2 *>(&h2);
-  const float2 f = __half22float2(hh);
-  return pack_bf16x2(f.x, f.y);
+// Four E4M3 codes (low byte first) -> two f16x2 (codes 0-1, codes 2-3), exact: every E4M3
+// value is an f16 value.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(codes));
+}
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two bf16 (low half first) times the power of two s -> f16x2; exact while the products are
+// f16 normal numbers.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t v, float s) {
+  const __half2 h = __floats2half2_rn(__uint_as_float(v << 16) * s, __uint_as_float(v & 0xffff0000u) * s);
+  return *reinterpret_cast<const uint32_t *>(&h);
 }
 
 __device__ __forceinline__ void ldsm_x4_b8(uint32_t addr, uint32_t (&r)[4]) {
@@ -110,6 +128,7 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
   float *alpha_sm = reinterpret_cast<float *>(smem + T::kOffAlpha);
   float *l_sm = reinterpret_cast<float *>(smem + T::kOffL);
   float *m_sm = reinterpret_cast<float *>(smem + T::kOffM);
+  float *t_sm = reinterpret_cast<float *>(smem + T::kOffT);
   const unsigned long long lim_ns = p.watchdog_ns;
 
   if (threadIdx.x == 0) {
@@ -200,8 +219,16 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
     // columns 16k + 4 c4 + {0, 1, 2, 3} of one key; in m16n8k16 those are the K positions
     // {2 c4, 2 c4 + 1, 2 c4 + 8, 2 c4 + 9}, so the A fragments take Q's columns in the same
     // order: a0/a1 = columns 4 c4, 4 c4 + 1 of rows g4, g4 + 8; a2/a3 = 4 c4 + 2, 4 c4 + 3.
+    //
+    // The score MMAs run in f16: the codes' f16 form is exact (one conversion per two codes),
+    // and the query tile is carried in f16 after a power-of-two scale 2^e that puts its
+    // largest |q| in [2^14, 2^15): every bf16 value of the tile within 2^28 of that maximum
+    // is exact in f16, and smaller ones are rounded to f16 subnormals (an error below 2^-39 of
+    // the largest product, far under the fp32 accumulation's rounding).  The partial scores
+    // are multiplied back by 2^-e.
     const int kh = warp >> 1, kn = warp & 1;
     uint32_t qf[kD / 32][4];
+    float qs_inv = 1.f;
     int it = 0, qs = 0;
     bool ok = true;
     for (int seq = pc.bi; part_has(pc, seq); ++seq) {
@@ -209,6 +236,29 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
       const int nch = fp8_chunk_range(p, pc, seq, L, t0, t1);
       if (nch == 0) continue;
       ok = ok && mbar_wait(bar(T::QFULL), qs & 1, abort, p.status, lim_ns);
+      float q_scale = 1.f;
+      if (ok) {
+        // largest |q| over the tile's R rows (row r of a 16-row column block: bytes r*128..)
+        uint32_t mx = 0;
+        for (int i = lane; i < kColBlocks * p.R * 8; i += 32) {
+          const int c = i / (p.R * 8), rem = i % (p.R * 8);
+          uint32_t v0, v1, v2, v3;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                       : "r"(sQ + c * 2048 + rem * 16));
+          const uint32_t w[4] = {v0, v1, v2, v3};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) mx = max(mx, max(w[k] & 0x7fffu, (w[k] >> 16) & 0x7fffu));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        // exponent of the largest |q| (bf16 field, bias 127); e = 14 - (exp - 127), kept
+        // within the fp32 normal range
+        const int ex = int(mx >> 7);
+        const int e = mx == 0 ? 0 : max(-120, min(120, 141 - ex));
+        q_scale = __uint_as_float(uint32_t(127 + e) << 23);
+        qs_inv = __uint_as_float(uint32_t(127 - e) << 23);
+      }
       if (ok) {
 #pragma unroll
         for (int kk = 0; kk < kD / 32; ++kk) {
@@ -217,10 +267,10 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
           uint32_t lo0, hi0, lo1, hi1;
           asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(sQ + cb * 2048 + sw128(g4, ch) + off));
           asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo1), "=r"(hi1) : "r"(sQ + cb * 2048 + sw128(g4 + 8, ch) + off));
-          qf[kk][0] = lo0;
-          qf[kk][1] = lo1;
-          qf[kk][2] = hi0;
-          qf[kk][3] = hi1;
+          qf[kk][0] = bf16x2_to_f16x2_scaled(lo0, q_scale);
+          qf[kk][1] = bf16x2_to_f16x2_scaled(lo1, q_scale);
+          qf[kk][2] = bf16x2_to_f16x2_scaled(hi0, q_scale);
+          qf[kk][3] = bf16x2_to_f16x2_scaled(hi1, q_scale);
         }
       }
       __syncwarp();
@@ -249,16 +299,16 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
               float(&a1)[4] = dk ? sd[1] : sc[1];
 #pragma unroll
               for (int nt = 0; nt < 2; ++nt) {
-                const uint32_t codes = r[2 * dk + nt];
-                const uint32_t b0 = e4m3x2_to_bf16x2(codes & 0xffffu), b1 = e4m3x2_to_bf16x2(codes >> 16);
-                mma_bf16_16816(nt ? a1 : a0, qf[kk + dk], b0, b1);
+                uint32_t b0, b1;
+                e4m3x4_to_f16x2x2(r[2 * dk + nt], b0, b1);
+                mma_f16_16816(nt ? a1 : a0, qf[kk + dk], b0, b1);
               }
             }
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            sc[0][e] += sd[0][e];
-            sc[1][e] += sd[1][e];
+            sc[0][e] = (sc[0][e] + sd[0][e]) * qs_inv;
+            sc[1][e] = (sc[1][e] + sd[1][e]) * qs_inv;
           }
         }
         if (it >= 2) named_bar_sync(T::kBarSEmpty + sb, T::kSPair);
@@ -284,6 +334,7 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
         lim[r] = row < p.R ? min(t1, p.causal ? L - (p.s_q - 1 - row / p.g) : L) : -1;
       }
       float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      int t_prev = 0;
       for (int n = 0; n < nch; ++n, ++it) {
         const int sb = it & 1, pb = it & 1;
         named_bar_sync(T::kBarSFull + sb, T::kSPair);
@@ -305,6 +356,21 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
           for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int u = 0; u < 2; ++u) kscale[kn][2 * t + u] = ksc[kn * 16 + t * 8 + c4 * 2 + u];
+        // P V runs in f16: P times the key's scale times 2^t, with the power of two t of this
+        // chunk chosen from its largest scale c so that every product (P <= 1) is below 2^15;
+        // the accumulator carries the factor 2^t, changed between chunks through alpha
+        float cmax = 0.f;
+#pragma unroll
+        for (int kn = 0; kn < 2; ++kn)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) cmax = fmaxf(cmax, kscale[kn][k]);
+        cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
+        cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
+        const int t_chunk = max(-120, min(120, 14 - (int((__float_as_uint(cmax) >> 23) & 0xff) - 127)));
+        const float p_scale = __uint_as_float(uint32_t(127 + t_chunk) << 23);
+        const int dt = max(-126, min(126, n == 0 ? 0 : t_chunk - t_prev));
+        const float t_step = __uint_as_float(uint32_t(127 + dt) << 23);
+        t_prev = t_chunk;
         float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
         for (int kn = 0; kn < 2; ++kn)
@@ -339,16 +405,17 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
             l[0] += p0 + p1;
             l[1] += p2 + p3;
             // the value row of a key is its scale times the codes: scale the probability
-            const float s0 = kscale[kn][2 * t], s1 = kscale[kn][2 * t + 1];
+            const float s0 = kscale[kn][2 * t] * p_scale, s1 = kscale[kn][2 * t + 1] * p_scale;
             const int kl = kn * 16 + t * 8 + c4 * 2;
+            const __half2 h01 = __floats2half2_rn(p0 * s0, p1 * s1), h23 = __floats2half2_rn(p2 * s0, p3 * s1);
             asm volatile("st.shared.b32 [%0], %1;" ::"r"(ptile + sw128(g4, kl / 8) + (kl % 8) * 2),
-                         "r"(pack_bf16x2(p0 * s0, p1 * s1)));
+                         "r"(*reinterpret_cast<const uint32_t *>(&h01)));
             asm volatile("st.shared.b32 [%0], %1;" ::"r"(ptile + sw128(g4 + 8, kl / 8) + (kl % 8) * 2),
-                         "r"(pack_bf16x2(p2 * s0, p3 * s1)));
+                         "r"(*reinterpret_cast<const uint32_t *>(&h23)));
           }
         if (c4 == 0) {
-          alpha_sm[pb * 16 + g4] = alpha[0];
-          alpha_sm[pb * 16 + g4 + 8] = alpha[1];
+          alpha_sm[pb * 16 + g4] = alpha[0] * t_step;
+          alpha_sm[pb * 16 + g4 + 8] = alpha[1] * t_step;
         }
         if (n == nch - 1) {
           // row sums and the row maximum for the epilogue of this sequence
@@ -364,6 +431,7 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
             m_sm[(qs & 1) * 16 + g4] = m[0];
             m_sm[(qs & 1) * 16 + g4 + 8] = m[1];
           }
+          if (lane == 0) t_sm[qs & 1] = __uint_as_float(uint32_t(127 - t_chunk) << 23);
         }
         fp8_bar_arrive(T::kBarPFull + pb, T::kPPair);
       }
@@ -410,7 +478,7 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
       float o[16][4];
 #pragma unroll
       for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-      float lt[2] = {0.f, 0.f}, mr[2] = {-INFINITY, -INFINITY};
+      float lt[2] = {0.f, 0.f}, mr[2] = {-INFINITY, -INFINITY}, t_inv = 1.f;
       for (int n = 0; n < nch; ++n, ++it) {
         const int s = it % T::NS, pb = it & 1;
         named_bar_sync(T::kBarPFull + pb, T::kPPair);
@@ -422,6 +490,7 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
             lt[r] = l_sm[(qs & 1) * 16 + g4 + 8 * r];
             mr[r] = m_sm[(qs & 1) * 16 + g4 + 8 * r];
           }
+          t_inv = t_sm[qs & 1];
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -449,8 +518,11 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
                 const int j = jp * 2 + h;
                 const uint32_t lo = __byte_perm(r[2 * h], 0u, 0x3120), hi = __byte_perm(r[2 * h + 1], 0u, 0x3120);
                 // even columns: low halves; odd columns: high halves
-                mma_bf16_16816(o[2 * j], a, e4m3x2_to_bf16x2(lo & 0xffffu), e4m3x2_to_bf16x2(hi & 0xffffu));
-                mma_bf16_16816(o[2 * j + 1], a, e4m3x2_to_bf16x2(lo >> 16), e4m3x2_to_bf16x2(hi >> 16));
+                uint32_t le, lod, he, hod;
+                e4m3x4_to_f16x2x2(lo, le, lod);
+                e4m3x4_to_f16x2x2(hi, he, hod);
+                mma_f16_16816(o[2 * j], a, le, he);
+                mma_f16_16816(o[2 * j + 1], a, lod, hod);
               }
             }
           }
@@ -464,7 +536,8 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
       for (int r = 0; r < 2; ++r) {
         const int row = g4 + 8 * r;
         if (row >= p.R || !ok) continue;
-        const float inv = lt[r] > 0.f ? 1.f / lt[r] : 0.f;
+        // the accumulator carries 2^t of the sequence's last chunk
+        const float inv = lt[r] > 0.f ? t_inv / lt[r] : 0.f;
         const int sq = row / p.g, h = kvh * p.g + row % p.g;
         const float lse_v = lt[r] > 0.f ? (mr[r] + fast_log2(lt[r])) * 0.69314718055994531f : -INFINITY;
         if (nsplit == 1) {

@@ -85,6 +85,35 @@ def test_fp8_parity_outliers_and_growing_maximum():
     fp8_parity(x)
 
 
+@pytest.mark.parametrize("q_exp", [40, -40, 0])
+def test_fp8_parity_query_magnitudes(q_exp):
+    # the score path carries the query tile in f16 after a power-of-two scale: queries far from
+    # unit size (scaled by 2^q_exp, exact in bf16; the softmax scale compensates so the scores
+    # stay the same), and a tile whose rows differ in size by 2^20 (row 3 large, row 5 small)
+    x = W.make_inputs_fp8(W.custom(2, 1, 16, 1, [700, 130], causal=True), seed=17)
+    q = x["q"].float() * 2.0 ** q_exp
+    q[:, :, 3] *= 2.0 ** 10
+    q[:, :, 5] *= 2.0 ** -10
+    x["q"] = q.to(torch.bfloat16)
+    assert torch.equal(x["q"].float(), q)
+    x["softmax_scale"] = 576 ** -0.5 * 2.0 ** -q_exp
+    fp8_parity(x)
+
+
+def test_fp8_parity_subnormal_codes():
+    # codes drawn from the whole E4M3 set, subnormals (exponent field 0) included, with
+    # scales of a few binades: the codes' exact widening is exercised code by code
+    x = W.make_inputs(W.custom(2, 1, 16, 1, [300, 77], causal=False), seed=23)
+    g = torch.Generator().manual_seed(23)
+    k8 = torch.randint(0, 256, x["k_cache"].shape, generator=g, dtype=torch.int32).to(torch.uint8)
+    k8[(k8 & 0x7f) == 0x7f] = 0x01           # no NaN codes; more subnormals
+    sub = torch.rand(k8.shape, generator=g) < 0.3
+    k8[sub] = k8[sub] & 0x87                 # exponent field 0: subnormal (or zero) codes
+    x["k8"] = k8
+    x["k_scale"] = (2.0 ** torch.randint(-9, -5, (1, k8.shape[0], 64), generator=g)).float()
+    fp8_parity(x)
+
+
 def test_fp8_separate_combine_matches_fused():
     x = W.make_inputs_fp8(W.custom(2, 1, 16, 1, [5000, 300], causal=True), seed=9)
     out_a, lse_a, tile, splits, _ = run_fp8(x)
