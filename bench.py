@@ -64,6 +64,7 @@ KERNEL_SOURCES = {
     "decode_mma16_kernel": ["common.cuh", "decode_mma.cu"],
     "decode_wide_kernel": ["common.cuh", "decode_wide.cu"],
     "decode_pair_kernel": ["common.cuh", "decode_pair.cu"],
+    "decode_fp8_kernel": ["common.cuh", "decode_fp8.cu"],
 }
 
 
@@ -590,15 +591,16 @@ def measure(name, args, dev, group, rank, world, with_e2e, cpu_seconds):
     achieved = work / kernel_s
     iso_achieved = work / iso_s
     # the summaries were taken with the library's own kernel choice
-    traffic = (recorded_traffic(name, "decode_mma16_kernel" if sparse else decode_kernel_for(R, w.h_q // w.h_kv))
-               if args.kernel == "auto" else None)
+    kernel_name = ("decode_fp8_kernel" if fp8 else "decode_mma16_kernel" if sparse else
+                   decode_kernel_for(R, w.h_q // w.h_kv))
+    traffic = recorded_traffic(name, kernel_name) if args.kernel == "auto" else None
     res = {
         "workload": name, "config": workload_config(w, kind), "unit": unit, "value": value,
         "ms_per_step": per_step * 1e3, "n_rep": n_rep, "per_rep_bytes": per_rep,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": r_unit,
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
-                     "kernel": "decode", "kernel_ms": kernel_s * 1e3,
+                     "kernel": kernel_name, "kernel_ms": kernel_s * 1e3,
                      "kernel_timing": f"average over a graph of {args.steps} back-to-back decode launches",
                      "isolated_ms": iso_s * 1e3, "isolated_achieved": iso_achieved,
                      "isolated_frac": iso_achieved / peak,
