@@ -737,6 +737,90 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
             "ms_per_step": e2e_s * 1e3, "steps_in_flight": 2}
 
 
+ABSORB_TOKENS, ABSORB_HEADS = 128, 128  # the compute-bound decode batch: 128 tokens x 128 heads
+
+
+def absorb_work(T, H):
+    """Algorithmic bytes and flops of one absorb_query + absorb_output pass: q_nope, q_rope,
+    W^UK read, q' written; o_latent, W^UV read, o written (bf16); 2 flops per multiply-add."""
+    nbytes = 2 * (T * H * 128 + T * H * 64 + H * 128 * 512 + T * H * 576 + T * H * 512 + H * 128 * 512 + T * H * 128)
+    flops = 2 * T * H * 128 * 512 * 2
+    return nbytes, flops
+
+
+def measure_absorb(args, dev, group, cpu_seconds):
+    """The absorption products around the decode (query into latent space, output out of it)
+    at the compute-bound decode batch: a graph of K passes over rotating input copies (more
+    bytes than L2 in all), the weight and activation bytes against the HBM peak."""
+    from paged_mla_decode_11_b200 import ops
+    T, H = ABSORB_TOKENS, ABSORB_HEADS
+    x = W.make_absorb_inputs(T, H, seed=args.seed)
+    nbytes, flops = absorb_work(T, H)
+    n_rep = max(2, math.ceil(1.5 * L2_BYTES / nbytes) + 1)
+    reps = []
+    for _ in range(n_rep):
+        d = {k: v.to(dev).clone() for k, v in x.items()}
+        d["q_abs"] = torch.empty(T, H, 576, dtype=torch.bfloat16, device=dev)
+        d["o"] = torch.empty(T, H, 128, dtype=torch.bfloat16, device=dev)
+        reps.append(d)
+
+    def step(d):
+        ops.absorb_query(d["q_nope"], d["q_rope"], d["w_uk"], out=d["q_abs"])
+        ops.absorb_output(d["o_latent"], d["w_uv"], out=d["o"])
+
+    for i in range(max(args.warmup, 3)):
+        step(reps[i % n_rep])
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.Stream(device=dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(args.steps):
+            step(reps[i % n_rep])
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index)
+    group.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    per_step = group.max(a.elapsed_time(b) * 1e-3 / args.steps)
+    graph.reset()
+    peaks, peak_kind = load_peaks()
+    achieved = nbytes / per_step / 1e9
+    res = {
+        "config": {"workload": f"absorption products: T={T} tokens, H={H} heads, W^UK and W^UV [H, 128, 512] "
+                               f"bf16 ~N(0, 1/fan-in), q_nope [T, H, 128], q_rope [T, H, 64], o_latent [T, H, 512] "
+                               f"~N(0,1) bf16, seed {args.seed}"},
+        "unit": "GB/s", "value": achieved, "ms_per_step": per_step * 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peak_kind} (hbm_gbs)", "kernel": "absorb_gemm_kernel (both products)",
+                     "kernel_ms": per_step * 1e3,
+                     "kernel_timing": f"average over a graph of {args.steps} passes (three launches each)",
+                     "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
+                     "achieved_tflops": flops / per_step / 1e12},
+        "clocks": clocks,
+    }
+    if cpu_seconds > 0 and not args.no_cpu_baseline:
+        import oracle
+        t0, runs = time.perf_counter(), 0
+        while runs == 0 or time.perf_counter() - t0 < cpu_seconds:
+            oracle.absorb_query(x["q_nope"].double().numpy(), x["q_rope"].double().numpy(), x["w_uk"].double().numpy())
+            oracle.absorb_output(x["o_latent"].double().numpy(), x["w_uv"].double().numpy())
+            runs += 1
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": runs * nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                               "sample": f"the whole pass, {runs} time(s), {dt:.1f} s of fp64 numpy einsum (one thread)"}
+    del reps
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     rank, local_rank, world = dist_env()
     if args.gpus != world:
@@ -757,6 +841,7 @@ def run_ours(args):
             per_workload[name] = {k: r[k] for k in ("config", "unit", "value", "ms_per_step", "roofline",
                                                     "clocks") if k in r}
             per_workload[name]["cpu_baseline"] = r.get("cpu_baseline")
+        per_workload["absorb"] = measure_absorb(args, dev, group, cpu_seconds=2.0)
     group.close()
     if rank != 0:
         return
