@@ -305,7 +305,8 @@ MLA_API int mla_merge_partials(const void *o_parts, const float *lse_parts, int 
  *   w_uv     device bf16 [heads][128][512], contiguous
  *   out      device bf16 [tokens][heads][128], contiguous
  * bf16 inputs, fp32 accumulation (warp MMA), bf16 results; strides in elements, multiples of
- * 8.  Errors: MLA_ERR_ARG, MLA_ERR_CUDA.
+ * 8; q_nope, q_rope, o_latent, the weights and q_out 16-byte aligned, out 4-byte aligned.
+ * Errors: MLA_ERR_ARG, MLA_ERR_CUDA.
  */
 MLA_API int mla_absorb_query(const void *q_nope, const int64_t nope_strides[2], const void *q_rope,
                              const int64_t rope_strides[2], const void *w_uk, int tokens, int heads, void *q_out,

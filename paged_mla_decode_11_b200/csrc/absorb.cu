@@ -6,58 +6,119 @@
 //     q'[t, h, 512:576] = q_rope[t, h, 0:64]                             (passes through)
 //   after the decode:
 //     o[t, h, d] = sum_c o_lat[t, h, c] * W^UV[h, d, c]                  (K = 512)
-// Both are per-head GEMMs C[M x N] = A[M x K] B[K x N] with M = tokens (batch x s_q).  One
-// warp computes 16 tokens x 64 columns with mma.sync m16n8k16 bf16 (fp32 accumulate),
-// fragments loaded straight from global memory (the weights are read once per 64 tokens).
+// Both are per-head GEMMs C[M x N] = A[M x K] B[K x N] with M = tokens (batch x s_q).  At
+// decode batch sizes they are bound by reading the weights (128 KB per head and product), so
+// they run on warp MMA (mma.sync m16n8k16 bf16, fp32 accumulate): a CTA computes a 64-token x
+// BN-column tile of one head (BN = 128 for q', 64 for the output), its four warps 16 tokens x
+// BN columns each, over K chunks of 64 staged in shared memory by cp.async (three stages: two
+// chunks load while one is multiplied).  Tile rows are padded by 16 bytes, so the 8 rows of
+// an ldmatrix fall in distinct banks.
 #include "launch.h"
 
 namespace pagedmla {
 
-constexpr int kAbsorbWarps = 4;  // 64 tokens per CTA
+constexpr int kAbBM = 64, kAbBK = 64, kAbWarps = 4, kAbStages = 3;
+
+template <bool kKN, int BN>
+struct AbsorbTile {
+  static constexpr int kARow = kAbBK * 2 + 16;                       // A chunk [64 tokens][64 k]
+  static constexpr int kABytes = kAbBM * kARow;
+  // B chunk: [64 k][BN n] when B is given as [K][N], else [BN n][64 k]
+  static constexpr int kBRow = kKN ? BN * 2 + 16 : kAbBK * 2 + 16;
+  static constexpr int kBBytes = kKN ? kAbBK * kBRow : BN * kBRow;
+  static constexpr int kStage = kABytes + kBBytes;
+  static constexpr int kSmem = kAbStages * kStage;
+};
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // B given as [K][N] (W^UK: k = d, n = latent column) when kKN, else as [N][K] (W^UV: n = d,
-// k = latent column).
-template <bool kKN>
-__global__ void __launch_bounds__(kAbsorbWarps * 32)
-    absorb_gemm_kernel(const __nv_bfloat16 *__restrict__ A, int64_t a_row, int64_t a_head, const __nv_bfloat16 *__restrict__ B,
-                       __nv_bfloat16 *__restrict__ C, int64_t c_row, int64_t c_head, int M, int N, int K) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+// k = latent column).  M, N, K: tokens (any), columns (a multiple of BN), contraction (a
+// multiple of 64).
+template <bool kKN, int BN>
+__global__ void __launch_bounds__(kAbWarps * 32)
+    absorb_gemm_kernel(const __nv_bfloat16 *__restrict__ A, int64_t a_row, int64_t a_head,
+                       const __nv_bfloat16 *__restrict__ B, __nv_bfloat16 *__restrict__ C, int64_t c_row,
+                       int64_t c_head, int M, int N, int K) {
+  using T = AbsorbTile<kKN, BN>;
+  extern __shared__ __align__(16) uint8_t absorb_smem[];
+  const uint32_t sbase = smem_u32(absorb_smem);
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int g4 = lane >> 2, c4 = lane & 3;
-  const int n0 = blockIdx.x * 64, h = blockIdx.y, m0 = blockIdx.z * 64 + warp * 16;
-  const __nv_bfloat16 *Ah = A + h * a_head;
+  const int n0 = blockIdx.x * BN, h = blockIdx.y, m0 = blockIdx.z * kAbBM;
+  const __nv_bfloat16 *Ah = A + int64_t(h) * a_head;
   const __nv_bfloat16 *Bh = B + int64_t(h) * K * N;
-  auto a_pair = [&](int m, int k) -> uint32_t {
-    if (m >= M) return 0u;
-    return __ldg(reinterpret_cast<const uint32_t *>(Ah + m * a_row + k));
-  };
-  auto b_pair = [&](int k, int n) -> uint32_t {
-    if (kKN) {
-      const uint16_t lo = __ldg(reinterpret_cast<const uint16_t *>(Bh + int64_t(k) * N + n));
-      const uint16_t hi = __ldg(reinterpret_cast<const uint16_t *>(Bh + int64_t(k + 1) * N + n));
-      return uint32_t(lo) | (uint32_t(hi) << 16);
+
+  auto load_stage = [&](int st, int k0) {
+    const uint32_t sa = sbase + st * T::kStage, sb = sa + T::kABytes;
+    for (int i = tid; i < kAbBM * (kAbBK / 8); i += kAbWarps * 32) {
+      const int r = i / (kAbBK / 8), c = i % (kAbBK / 8), t = m0 + r;
+      cp_async16_zfill(sa + r * T::kARow + c * 16, Ah + int64_t(min(t, M - 1)) * a_row + k0 + c * 8, t < M ? 16u : 0u);
     }
-    return __ldg(reinterpret_cast<const uint32_t *>(Bh + int64_t(n) * K + k));
+    if constexpr (kKN) {
+      for (int i = tid; i < kAbBK * (BN / 8); i += kAbWarps * 32) {
+        const int r = i / (BN / 8), c = i % (BN / 8);
+        cp_async16_zfill(sb + r * T::kBRow + c * 16, Bh + int64_t(k0 + r) * N + n0 + c * 8, 16u);
+      }
+    } else {
+      for (int i = tid; i < BN * (kAbBK / 8); i += kAbWarps * 32) {
+        const int r = i / (kAbBK / 8), c = i % (kAbBK / 8);
+        cp_async16_zfill(sb + r * T::kBRow + c * 16, Bh + int64_t(n0 + r) * K + k0 + c * 8, 16u);
+      }
+    }
+    cp_async_commit();
   };
-  float acc[8][4];
+
+  float acc[BN / 8][4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  for (int k = 0; k < K; k += 16) {
-    const int k0 = k + 2 * c4;
-    const uint32_t a[4] = {a_pair(m0 + g4, k0), a_pair(m0 + g4 + 8, k0), a_pair(m0 + g4, k0 + 8),
-                           a_pair(m0 + g4 + 8, k0 + 8)};
+  for (int j = 0; j < BN / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  const int nk = K / kAbBK;
+  // one commit group per chunk (empty past the end), so "all but the newest S - 2 groups
+  // landed" means chunk kc has landed
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int n = n0 + 8 * j + g4;
-      mma_bf16_16816(acc[j], a, b_pair(k0, n), b_pair(k0 + 8, n));
+  for (int st = 0; st < kAbStages - 1; ++st) {
+    if (st < nk) load_stage(st, st * kAbBK);
+    else cp_async_commit();
+  }
+  for (int kc = 0; kc < nk; ++kc) {
+    cp_async_wait<kAbStages - 2>();
+    __syncthreads();  // chunk kc is visible to all warps; chunk kc - 1's stage is free
+    const int kn = kc + kAbStages - 1;
+    if (kn < nk) load_stage(kn % kAbStages, kn * kAbBK);
+    else cp_async_commit();
+    const uint32_t sa = sbase + (kc % kAbStages) * T::kStage, sb = sa + T::kABytes;
+#pragma unroll
+    for (int ks = 0; ks < kAbBK / 16; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(sa + (warp * 16 + (lane & 15)) * T::kARow + (ks * 16 + (lane >> 4) * 8) * 2, a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int jp = 0; jp < BN / 16; ++jp) {
+        uint32_t b[4];
+        if constexpr (kKN)
+          ldsm_x4_t(sb + (ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * T::kBRow + (jp * 16 + (lane >> 4) * 8) * 2,
+                    b[0], b[1], b[2], b[3]);
+        else
+          ldsm_x4(sb + (jp * 16 + (lane & 7) + (lane >> 4) * 8) * T::kBRow + (ks * 16 + ((lane >> 3) & 1) * 8) * 2,
+                  b[0], b[1], b[2], b[3]);
+        mma_bf16_16816(acc[2 * jp], a, b[0], b[1]);
+        mma_bf16_16816(acc[2 * jp + 1], a, b[2], b[3]);
+      }
     }
   }
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    const int m = m0 + g4 + 8 * r;
-    if (m >= M) continue;
-    __nv_bfloat16 *crow = C + int64_t(h) * c_head + int64_t(m) * c_row + n0 + 2 * c4;
+    const int t = m0 + warp * 16 + g4 + 8 * r;
+    if (t >= M) continue;
+    __nv_bfloat16 *crow = C + int64_t(h) * c_head + int64_t(t) * c_row + n0 + 2 * c4;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < BN / 8; ++j)
       *reinterpret_cast<uint32_t *>(crow + 8 * j) = pack_bf16x2(acc[j][2 * r], acc[j][2 * r + 1]);
   }
 }
@@ -75,10 +136,14 @@ __global__ void rope_copy_kernel(const __nv_bfloat16 *__restrict__ q_rope, int64
 cudaError_t launch_absorb_q(const __nv_bfloat16 *q_nope, int64_t n_row, int64_t n_head, const __nv_bfloat16 *q_rope,
                             int64_t r_row, int64_t r_head, const __nv_bfloat16 *w_uk, __nv_bfloat16 *q_out, int T,
                             int H, cudaStream_t stream) {
-  dim3 grid(512 / 64, H, (T + 63) / 64);
-  absorb_gemm_kernel<true><<<grid, kAbsorbWarps * 32, 0, stream>>>(q_nope, n_row, n_head, w_uk, q_out,
+  constexpr int kBN = 128;
+  constexpr int kSmem = AbsorbTile<true, kBN>::kSmem;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(absorb_gemm_kernel<true, kBN>), kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(512 / kBN, H, (T + kAbBM - 1) / kAbBM);
+  absorb_gemm_kernel<true, kBN><<<grid, kAbWarps * 32, kSmem, stream>>>(q_nope, n_row, n_head, w_uk, q_out,
                                                                    int64_t(H) * kD, kD, T, 512, 128);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n = int64_t(T) * H * 8;
   rope_copy_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(q_rope, r_row, r_head, q_out, T, H);
@@ -87,8 +152,12 @@ cudaError_t launch_absorb_q(const __nv_bfloat16 *q_nope, int64_t n_row, int64_t 
 
 cudaError_t launch_absorb_out(const __nv_bfloat16 *o_lat, int64_t l_row, int64_t l_head, const __nv_bfloat16 *w_uv,
                               __nv_bfloat16 *out, int T, int H, cudaStream_t stream) {
-  dim3 grid(128 / 64, H, (T + 63) / 64);
-  absorb_gemm_kernel<false><<<grid, kAbsorbWarps * 32, 0, stream>>>(o_lat, l_row, l_head, w_uv, out,
+  constexpr int kBN = 64;
+  constexpr int kSmem = AbsorbTile<false, kBN>::kSmem;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(absorb_gemm_kernel<false, kBN>), kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(128 / kBN, H, (T + kAbBM - 1) / kAbBM);
+  absorb_gemm_kernel<false, kBN><<<grid, kAbWarps * 32, kSmem, stream>>>(o_lat, l_row, l_head, w_uv, out,
                                                                     int64_t(H) * 128, 128, T, 128, 512);
   return cudaGetLastError();
 }

@@ -590,8 +590,8 @@ int mla_absorb_query(const void *q_nope, const int64_t nope_strides[2], const vo
   for (int i = 0; i < 2; ++i)
     if (nope_strides[i] < 0 || nope_strides[i] % 8 || rope_strides[i] < 0 || rope_strides[i] % 8)
       return fail(MLA_ERR_ARG, "strides must be non-negative multiples of 8 elements");
-  if (!aligned(q_nope, 16) || !aligned(q_rope, 16) || !aligned(w_uk, 4) || !aligned(q_out, 16))
-    return fail(MLA_ERR_ARG, "q_nope, q_rope and q_out must be 16-byte aligned, w_uk 4-byte aligned");
+  if (!aligned(q_nope, 16) || !aligned(q_rope, 16) || !aligned(w_uk, 16) || !aligned(q_out, 16))
+    return fail(MLA_ERR_ARG, "q_nope, q_rope, w_uk and q_out must be 16-byte aligned");
   cudaError_t e = launch_absorb_q(static_cast<const __nv_bfloat16 *>(q_nope), nope_strides[0], nope_strides[1],
                                   static_cast<const __nv_bfloat16 *>(q_rope), rope_strides[0], rope_strides[1],
                                   static_cast<const __nv_bfloat16 *>(w_uk), static_cast<__nv_bfloat16 *>(q_out), tokens,
@@ -608,8 +608,8 @@ int mla_absorb_output(const void *o_latent, const int64_t latent_strides[2], con
   for (int i = 0; i < 2; ++i)
     if (latent_strides[i] < 0 || latent_strides[i] % 8)
       return fail(MLA_ERR_ARG, "strides must be non-negative multiples of 8 elements");
-  if (!aligned(o_latent, 16) || !aligned(w_uv, 4) || !aligned(out, 4))
-    return fail(MLA_ERR_ARG, "o_latent must be 16-byte aligned, w_uv and out 4-byte aligned");
+  if (!aligned(o_latent, 16) || !aligned(w_uv, 16) || !aligned(out, 4))
+    return fail(MLA_ERR_ARG, "o_latent and w_uv must be 16-byte aligned, out 4-byte aligned");
   cudaError_t e = launch_absorb_out(static_cast<const __nv_bfloat16 *>(o_latent), latent_strides[0], latent_strides[1],
                                     static_cast<const __nv_bfloat16 *>(w_uv), static_cast<__nv_bfloat16 *>(out), tokens,
                                     heads, reinterpret_cast<cudaStream_t>(stream));
