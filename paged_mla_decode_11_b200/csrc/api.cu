@@ -572,6 +572,8 @@ int mla_merge_partials(const void *o_parts, const float *lse_parts, int n_parts,
   if (n_parts < 1 || batch < 1 || s_q < 1 || h_q < 1)
     return fail(MLA_ERR_ARG, "n_parts, batch, s_q and h_q must be >= 1");
   if (dv != kDV) return fail(MLA_ERR_UNSUPPORTED, "dv must be %d (got %d)", kDV, dv);
+  if (int64_t(batch) * s_q * h_q > (int64_t(1) << 31))
+    return fail(MLA_ERR_ARG, "batch * s_q * h_q must be <= 2^31");
   if (!aligned(o_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) || !aligned(lse, 4))
     return fail(MLA_ERR_ARG, "o_parts and out must be 16-byte aligned, lse_parts and lse 4-byte aligned");
   cudaError_t e = launch_merge(static_cast<const __nv_bfloat16 *>(o_parts), lse_parts, n_parts, batch, s_q, h_q,

@@ -163,3 +163,68 @@ def test_decode_rejects_before_calling_the_library(fake, over, exc, msg):
     with pytest.raises(exc, match=msg):
         ops.mla_decode_paged(**_bad(**over))
     assert not [n for n, _ in fake.calls if n == "mla_decode_paged"]
+
+
+def test_fp8_decode_marshalling(fake):
+    q, kc, bt, sl, tile, splits, ws = _inputs(b=3, s_q=1, h_q=16)
+    k8 = torch.zeros(10, 64, 1, 576, dtype=torch.uint8)
+    ks = torch.zeros(1, 10, 64, dtype=torch.float32)
+    out, lse = ops.mla_decode_paged_fp8(q, k8, ks, bt, sl, 512, tile, splits, causal=True, workspace=ws,
+                                        skip_combine=True)
+    a = fake.last("mla_decode_paged_fp8")
+    assert a[0] == q.data_ptr() and a[2:6] == (3, 1, 16, 576)
+    assert a[6:11] == (k8.data_ptr(), ks.data_ptr(), 10, 64, 1)
+    assert a[11:15] == (bt.data_ptr(), 6, sl.data_ptr(), 512)
+    assert a[15:18] == (tile.data_ptr(), 5, splits.data_ptr())
+    assert a[19] == 1 and a[20:24] == (out.data_ptr(), lse.data_ptr(), ws.data_ptr(), 4096)
+    assert a[24] == ops.MLA_FLAG_SKIP_COMBINE and a[25] == 4242
+    # float8 codes are passed as their bytes; a scale tensor of the wrong shape is refused
+    ops.mla_decode_paged_fp8(q, k8.view(torch.float8_e4m3fn), ks, bt, sl, 512, tile, splits, workspace=ws)
+    with pytest.raises(ValueError, match="k_scale"):
+        ops.mla_decode_paged_fp8(q, k8, ks[:, :5], bt, sl, 512, tile, splits, workspace=ws)
+
+
+def test_sparse_decode_and_plan_marshalling(fake):
+    q, kc, bt, sl, tile, splits, ws = _inputs(b=3, s_q=2, h_q=16)
+    row_ptr = torch.zeros(3 * 2 + 1, dtype=torch.int32)
+    col = torch.zeros(40, dtype=torch.int32)
+    t2, s2 = ops.get_mla_metadata_csr(row_ptr, 16, 1)
+    a = fake.last("mla_get_metadata_csr")
+    assert a[0] == row_ptr.data_ptr() and a[1:4] == (6, 16, ops.num_parts_for(148, 16, 1))
+    assert t2.shape == (a[3], 8) and s2.shape == (7,)
+    sp = torch.zeros(7, dtype=torch.int32)
+    out, lse = ops.mla_decode_sparse(q, kc, bt, sl, row_ptr, col, 512, tile, sp, causal=True, workspace=ws)
+    a = fake.last("mla_decode_sparse")
+    assert a[2:6] == (3, 2, 16, 576) and a[6:10] == (kc.data_ptr(), 10, 64, 1)
+    assert a[10:16] == (bt.data_ptr(), 6, sl.data_ptr(), row_ptr.data_ptr(), col.data_ptr(), 512)
+    assert a[16:19] == (tile.data_ptr(), 5, sp.data_ptr()) and a[20] == 1 and a[25] == 0
+    assert out.shape == (3, 2, 16, 512) and lse.shape == (3, 16, 2)
+    # num_splits is per query token; row_ptr must have batch * s_q + 1 entries
+    with pytest.raises(ValueError, match="num_splits"):
+        ops.mla_decode_sparse(q, kc, bt, sl, row_ptr, col, 512, tile, splits, workspace=ws)
+    with pytest.raises(ValueError, match="row_ptr"):
+        ops.mla_decode_sparse(q, kc, bt, sl, row_ptr[:5], col, 512, tile, sp, workspace=ws)
+
+
+def test_merge_and_absorb_marshalling(fake):
+    o = torch.zeros(3, 2, 1, 16, 512, dtype=torch.bfloat16)
+    l = torch.zeros(3, 2, 16, 1, dtype=torch.float32)
+    out, lse = ops.mla_merge_partials(o, l)
+    a = fake.last("mla_merge_partials")
+    assert a[:7] == (o.data_ptr(), l.data_ptr(), 3, 2, 1, 16, 512) and a[7:9] == (out.data_ptr(), lse.data_ptr())
+    with pytest.raises(ValueError, match="lse_parts"):
+        ops.mla_merge_partials(o, l[:2])
+    # the two column ranges of one [T, H, 192] projection: strides in elements
+    qkv = torch.zeros(5, 4, 192, dtype=torch.bfloat16)
+    w = torch.zeros(4, 128, 512, dtype=torch.bfloat16)
+    q_abs = ops.absorb_query(qkv[..., :128], qkv[..., 128:], w)
+    a = fake.last("mla_absorb_query")
+    assert a[0] == qkv.data_ptr() and list(a[1]) == [768, 192] and a[2] == qkv.data_ptr() + 256
+    assert list(a[3]) == [768, 192] and a[4] == w.data_ptr() and a[5:7] == (5, 4) and a[7] == q_abs.data_ptr()
+    assert q_abs.shape == (5, 4, 576)
+    lat = torch.zeros(5, 4, 512, dtype=torch.bfloat16)
+    o2 = ops.absorb_output(lat, w)
+    a = fake.last("mla_absorb_output")
+    assert a[0] == lat.data_ptr() and list(a[1]) == [2048, 512] and a[2:6] == (w.data_ptr(), 5, 4, o2.data_ptr())
+    with pytest.raises(ValueError):
+        ops.absorb_output(lat[..., :256], w)

@@ -115,3 +115,45 @@ def test_static_entry_host_rejections(lib):
             ctypes.c_float(0.04), 1, None, None, 0, None)
     assert rc == -3
     assert b"static scratch holds" in lib.mla_last_error_string()
+
+
+def test_sparse_fp8_merge_absorb_host_rejections(lib):
+    """The later entry points refuse bad arguments on the host, before any device call."""
+    s3 = (ctypes.c_int64 * 3)(576, 576, 576)
+    f = ctypes.c_float(0.04)
+    # mla_decode_sparse(q, strides, b, s_q, h_q, d, k, pages, page, h_kv, bt, bt_stride, lens,
+    #                   row_ptr, col_idx, dv, tile, parts, splits, scale, causal, out, lse, ws, ws_bytes, flags, stream)
+    def sparse(h_q=16, d=576, dv=512, flags=0, row_ptr=16):
+        return lib.mla_decode_sparse(16, s3, 1, 1, h_q, d, 16, 1, 64, 1, 16, 1, 16, row_ptr, 16, dv, 16, 1, 16, f, 1,
+                                     16, 16, 256, 1 << 20, flags, None)
+    assert sparse(d=512) == -2 and b"d must be 576" in lib.mla_last_error_string()
+    assert sparse(h_q=32) == -2 and b"up to 16 query heads" in lib.mla_last_error_string()
+    assert sparse(flags=2) == -1 and b"flags" in lib.mla_last_error_string()
+    assert sparse(row_ptr=None) == -1 and b"null" in lib.mla_last_error_string()
+    assert sparse(dv=256) == -2
+    # mla_get_metadata_csr(row_ptr, n_lists, rows_per_kv_head, num_parts, tile, splits, stream)
+    assert lib.mla_get_metadata_csr(None, 4, 16, 10, 16, 16, None) == -1
+    assert lib.mla_get_metadata_csr(16, 0, 16, 10, 16, 16, None) == -1
+    assert lib.mla_get_metadata_csr(16, 4, 0, 10, 16, 16, None) == -1
+    assert lib.mla_get_metadata_csr(16, 4, 16, 0, 16, 16, None) == -1
+    # mla_decode_paged_fp8: more than 16 rows per latent head is the 16-row kernel's limit
+    rc = lib.mla_decode_paged_fp8(16, s3, 1, 1, 32, 576, 16, 16, 1, 64, 1, 16, 1, 16, 512, 16, 1, 16, f, 1, 16, 16,
+                                  256, 1 << 20, 0, None)
+    assert rc == -2 and b"16-row kernel" in lib.mla_last_error_string()
+    # mla_merge_partials(o_parts, lse_parts, n, b, s_q, h_q, dv, out, lse, stream)
+    assert lib.mla_merge_partials(None, 16, 2, 1, 1, 16, 512, 16, 16, None) == -1
+    assert lib.mla_merge_partials(16, 16, 0, 1, 1, 16, 512, 16, 16, None) == -1
+    assert lib.mla_merge_partials(16, 16, 2, 1, 1, 16, 256, 16, 16, None) == -2
+    assert lib.mla_merge_partials(18, 16, 2, 1, 1, 16, 512, 16, 16, None) == -1     # misaligned partials
+    # mla_absorb_query(q_nope, strides, q_rope, strides, w_uk, T, H, q_out, stream)
+    s2 = (ctypes.c_int64 * 2)(192 * 16, 192)
+    bad = (ctypes.c_int64 * 2)(192 * 16, 190)
+    assert lib.mla_absorb_query(None, s2, 272, s2, 16, 4, 16, 16, None) == -1
+    assert lib.mla_absorb_query(16, s2, 272, s2, 16, 0, 16, 16, None) == -1
+    assert lib.mla_absorb_query(16, bad, 272, s2, 16, 4, 16, 16, None) == -1
+    assert lib.mla_absorb_query(16, s2, 272, s2, 20, 4, 16, 16, None) == -1           # weights not 16-byte aligned
+    # mla_absorb_output(o_latent, strides, w_uv, T, H, out, stream)
+    assert lib.mla_absorb_output(None, s2, 16, 4, 16, 16, None) == -1
+    assert lib.mla_absorb_output(16, s2, 16, 4, 0, 16, None) == -1
+    assert lib.mla_absorb_output(16, bad, 16, 4, 16, 16, None) == -1
+    assert lib.mla_absorb_output(16, s2, 24, 4, 16, 16, None) == -1
