@@ -41,6 +41,10 @@ class FakeLib:
 def fake(monkeypatch):
     lib = FakeLib()
     monkeypatch.setattr(ops, "_lib", lib)
+    # the binding memoises pure shape functions: keep the stand-in's answers out of them
+    monkeypatch.setattr(ops, "_parts_cache", {})
+    monkeypatch.setattr(ops, "_ws_size_cache", {})
+    monkeypatch.setattr(ops, "_ws_cache", {})
 
     def dtype_only(t, name, dtype):
         if t.dtype != dtype:
