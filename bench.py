@@ -821,6 +821,76 @@ def measure_absorb(args, dev, group, cpu_seconds):
     return res
 
 
+MERGE_SHARDS, MERGE_BATCH, MERGE_SQ, MERGE_HQ = 8, 32, 2, 128  # the causal multi-token query shape
+
+
+def measure_merge(args, dev, group, cpu_seconds):
+    """The on-device step of the sequence-sharded decode: the log-sum-exp merge of the
+    partials (bf16 out and fp32 lse) that the GPUs of a node exchange, here 8 shards of the
+    causal multi-token query shape, their bytes read and the output written against the HBM
+    peak.  (The exchange itself, one all-gather, needs several GPUs.)"""
+    from paged_mla_decode_11_b200 import ops
+    n, b, s_q, h_q = MERGE_SHARDS, MERGE_BATCH, MERGE_SQ, MERGE_HQ
+    g = torch.Generator().manual_seed(args.seed)
+    o = torch.randn(n, b, s_q, h_q, 512, generator=g).to(torch.bfloat16)
+    l = torch.randn(n, b, h_q, s_q, generator=g) * 3
+    rows = b * s_q * h_q
+    nbytes = n * rows * (512 * 2 + 4) + rows * (512 * 2 + 4)
+    n_rep = max(2, math.ceil(1.5 * L2_BYTES / nbytes) + 1)
+    reps = [(o.to(dev).clone(), l.to(dev).clone(), torch.empty(b, s_q, h_q, 512, dtype=torch.bfloat16, device=dev),
+             torch.empty(b, h_q, s_q, dtype=torch.float32, device=dev)) for _ in range(n_rep)]
+    for i in range(max(args.warmup, 3)):
+        d = reps[i % n_rep]
+        ops.mla_merge_partials(d[0], d[1], out=d[2], lse=d[3])
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.Stream(device=dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(args.steps):
+            d = reps[i % n_rep]
+            ops.mla_merge_partials(d[0], d[1], out=d[2], lse=d[3])
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index)
+    group.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        graph.replay()
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    per_step = group.max(a.elapsed_time(e) * 1e-3 / args.steps)
+    graph.reset()
+    peaks, peak_kind = load_peaks()
+    achieved = nbytes / per_step / 1e9
+    res = {
+        "config": {"workload": f"shard merge: {n} shards' partials of batch={b}, s_q={s_q}, h_q={h_q} "
+                               f"(out bf16 [n, b, s_q, h_q, 512] ~N(0,1), lse fp32 ~N(0,9)), seed {args.seed}"},
+        "unit": "GB/s", "value": achieved, "ms_per_step": per_step * 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peak_kind} (hbm_gbs)",
+                     "kernel": "merge_kernel", "kernel_ms": per_step * 1e3,
+                     "kernel_timing": f"average over a graph of {args.steps} merge launches",
+                     "algorithmic_bytes_per_launch": nbytes},
+        "clocks": clocks,
+    }
+    if cpu_seconds > 0 and not args.no_cpu_baseline:
+        import oracle
+        on, ln = o.double().numpy(), l.double().numpy().transpose(0, 1, 3, 2)
+        t0, runs = time.perf_counter(), 0
+        while runs == 0 or time.perf_counter() - t0 < cpu_seconds:
+            oracle.combine(ln, on)
+            runs += 1
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": runs * nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                               "sample": f"the whole merge, {runs} time(s), {dt:.1f} s of fp64 numpy (one thread)"}
+    del reps
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     rank, local_rank, world = dist_env()
     if args.gpus != world:
@@ -842,6 +912,7 @@ def run_ours(args):
                                                     "clocks") if k in r}
             per_workload[name]["cpu_baseline"] = r.get("cpu_baseline")
         per_workload["absorb"] = measure_absorb(args, dev, group, cpu_seconds=2.0)
+        per_workload["shard_merge"] = measure_merge(args, dev, group, cpu_seconds=2.0)
     group.close()
     if rank != 0:
         return
