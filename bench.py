@@ -737,6 +737,14 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
             "ms_per_step": e2e_s * 1e3, "steps_in_flight": 2}
 
 
+def load_for(graph, dev, seconds):
+    """Replays a captured graph for about `seconds` (a loaded GPU before a timed region)."""
+    t_end = time.perf_counter() + seconds
+    while time.perf_counter() < t_end:
+        graph.replay()
+        torch.cuda.synchronize(dev)
+
+
 ABSORB_TOKENS, ABSORB_HEADS = 128, 128  # the compute-bound decode batch: 128 tokens x 128 heads
 
 
@@ -779,6 +787,7 @@ def measure_absorb(args, dev, group, cpu_seconds):
     graph.replay()
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(dev.index)
+    load_for(graph, dev, 1.0)  # the sampled clocks describe the load
     group.barrier()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
@@ -852,6 +861,7 @@ def measure_merge(args, dev, group, cpu_seconds):
     graph.replay()
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(dev.index)
+    load_for(graph, dev, 1.0)  # the sampled clocks describe the load
     group.barrier()
     a = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
