@@ -313,3 +313,44 @@ def test_full_size_workloads(name):
                                          dv=512, softmax_scale=x["softmax_scale"], causal=x["causal"])
     stats = assert_parity(out, lse, ref_out, ref_lse)
     print(f"{name}: " + ", ".join(f"{k} {v:.3e}" for k, v in stats.items()))
+
+
+# ---------------------------------------------------------------------------------------
+# Maximum sizes: the largest batch the scheduler takes, and one sequence long enough that
+# every part holds a piece of it (the combine then merges as many partials as there are parts).
+# ---------------------------------------------------------------------------------------
+def test_largest_batch_sampled():
+    # MLA_MAX_BATCH sequences of 1..64 tokens (one page each): the plan's block scans run over
+    # 16,384 lengths (shared memory above 48 KB), and parts walk hundreds of sequences each
+    batch = 16384
+    rng = np.random.default_rng(16)
+    lens = rng.integers(1, 65, size=batch).tolist()
+    x = W.make_inputs(W.custom(batch, 1, 16, 1, lens, causal=True), seed=16)
+    out, lse, tile, splits = run_gpu(x)
+    check_metadata(x, tile, splits)
+    rows = sample_rows(x, per_seq=1, seed=16)[::61]
+    ro, rl = oracle.mla_decode_rows(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], rows,
+                                    dv=512, softmax_scale=x["softmax_scale"], causal=True)
+    o = out.double().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    l = lse.double().cpu().numpy()[rows[:, 0], rows[:, 2], rows[:, 1]]
+    assert np.abs(o - ro).max() <= OUT_TOL * np.abs(ro).max()
+    assert (np.abs(l - rl) / np.maximum(np.abs(rl), 1.0)).max() <= LSE_RTOL
+    assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("h_q", [16, 64, 128], ids=["16-row-kernel", "64-row-kernel", "cta-pair-kernel"])
+def test_one_sequence_over_every_part(h_q):
+    # 131,072 tokens (2,048 pages) in one sequence: every part decodes a piece of it and the
+    # combine merges 148 (or 74) partials per row, more than one warp's worth of split LSEs
+    L = 131072
+    x = W.make_inputs(W.custom(1, 1, h_q, 1, [L], causal=True), seed=h_q)
+    out, lse, tile, splits = run_gpu(x)
+    check_metadata(x, tile, splits)
+    assert int(splits[1] - splits[0]) > 32
+    rows = np.array([(0, 0, h) for h in range(0, h_q, max(1, h_q // 16))], dtype=np.int32)
+    ro, rl = oracle.mla_decode_rows(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"], rows,
+                                    dv=512, softmax_scale=x["softmax_scale"], causal=True)
+    o = out.double().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    l = lse.double().cpu().numpy()[rows[:, 0], rows[:, 2], rows[:, 1]]
+    assert np.abs(o - ro).max() <= OUT_TOL * np.abs(ro).max()
+    assert (np.abs(l - rl) / np.maximum(np.abs(rl), 1.0)).max() <= LSE_RTOL

@@ -25,7 +25,7 @@ def lengths(batch, seed):
     return lens.astype(np.int32)
 
 
-@pytest.mark.parametrize("batch", [1, 2, 31, 32, 33, 95, 1000, 1023, 1024, 1025, 3000])
+@pytest.mark.parametrize("batch", [1, 2, 31, 32, 33, 95, 1000, 1023, 1024, 1025, 3000, 16384])
 @pytest.mark.parametrize("rows", [16, 128])
 def test_plan_matches_specification(batch, rows):
     for num_parts in (1, 7, 148, batch + 5):
@@ -44,3 +44,17 @@ def test_metadata_size_is_the_default_part_count(rows, h_kv):
     tile, splits = ops.get_mla_metadata(lens, rows, h_kv)
     assert ops.metadata_size(40, rows, h_kv) == tile.shape[0]
     assert tile.shape[0] == ops.num_parts_for(ops.device_sm_count(), rows, h_kv)
+
+
+@pytest.mark.parametrize("n_lists", [1, 33, 1000, 16384])
+def test_csr_plan_matches_specification(n_lists):
+    # the sparse decode's plan: the same specification over key-list lengths given as offsets
+    counts = lengths(n_lists, seed=n_lists)
+    row_ptr = np.zeros(n_lists + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum(counts)
+    for rows, num_parts in ((16, 148), (8, 7)):
+        tile, splits = ops.get_mla_metadata_csr(torch.from_numpy(row_ptr).cuda(), rows, 1, num_parts=num_parts)
+        torch.cuda.synchronize()
+        want_tiles, want_splits = spec.schedule(counts.tolist(), num_parts, rows)
+        assert tile.cpu().tolist() == want_tiles
+        assert splits.cpu().tolist() == want_splits
