@@ -643,31 +643,46 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
     from paged_mla_decode_11_b200 import ops
     e2e_steps = min(args.steps, 50)
     fp8, sparse = kind == "fp8", kind == "sparse"
-    hq = x["q"].pin_memory()
-    hbt = x["block_table"].pin_memory()
-    hsl = x["cache_seqlens"].pin_memory()
-    # the sparse decode's key lists travel with the step's inputs
-    hrp = x["row_ptr"].pin_memory() if sparse else None
-    hci = x["col_idx"].pin_memory() if sparse else None
+    # a step's inputs packed in one pinned buffer (q, block_table, cache_seqlens and, for the
+    # sparse decode, the key lists), its results in one device buffer (out, lse): one copy
+    # each way; the API reads and writes views of them
+    ins = [("q", x["q"]), ("bt", x["block_table"]), ("sl", x["cache_seqlens"])]
+    if sparse:
+        ins += [("rp", x["row_ptr"]), ("ci", x["col_idx"])]
+
+    def layout(specs):
+        offs, n = {}, 0
+        for name, shape, dtype in specs:
+            offs[name] = (n, shape, dtype)
+            n += (math.prod(shape) * torch.empty(0, dtype=dtype).element_size() + 255) // 256 * 256
+        return offs, n
+
+    def views(buf, offs):
+        return {k: buf[o:o + math.prod(sh) * torch.empty(0, dtype=dt).element_size()].view(dt).view(sh)
+                for k, (o, sh, dt) in offs.items()}
+
+    in_offs, in_bytes = layout([(k, tuple(v.shape), v.dtype) for k, v in ins])
+    out_offs, out_bytes = layout([("out", (w.batch, w.s_q, w.h_q, 512), torch.bfloat16),
+                                  ("lse", (w.batch, w.h_q, w.s_q), torch.float32)])
+    hin = torch.zeros(in_bytes, dtype=torch.uint8).pin_memory()
+    for k, v in views(hin, in_offs).items():
+        v.copy_(dict(ins)[k])
     n_lists = w.batch * w.s_q if sparse else w.batch
     kstream = torch.cuda.Stream(device=dev)   # the API launches on the current stream
     up_stream = torch.cuda.Stream(device=dev)
     down_stream = torch.cuda.Stream(device=dev)
     slots = []
     for _ in range(2):
-        slots.append({
-            "q": torch.empty_like(d0["q"]), "bt": torch.empty_like(d0["block_table"]),
-            "sl": torch.empty_like(d0["cache_seqlens"]),
-            "tile": torch.empty(nparts, ops.TILE_FIELDS, dtype=torch.int32, device=dev),
-            "splits": torch.empty(n_lists + 1, dtype=torch.int32, device=dev),
-            "rp": torch.empty_like(d0["row_ptr"]) if sparse else None,
-            "ci": torch.empty_like(d0["col_idx"]) if sparse else None,
-            "out": torch.empty(w.batch, w.s_q, w.h_q, 512, dtype=torch.bfloat16, device=dev),
-            "lse": torch.empty(w.batch, w.h_q, w.s_q, dtype=torch.float32, device=dev),
-            "hout": torch.empty(w.batch, w.s_q, w.h_q, 512, dtype=torch.bfloat16).pin_memory(),
-            "hlse": torch.empty(w.batch, w.h_q, w.s_q, dtype=torch.float32).pin_memory(),
-            "ws": ops.new_workspace(ops.workspace_size(w.batch, w.s_q, w.h_q, w.h_kv, nparts), dev),
-            "up": torch.cuda.Event(), "done": torch.cuda.Event(), "back": torch.cuda.Event()})
+        din = torch.empty(in_bytes, dtype=torch.uint8, device=dev)
+        dout = torch.empty(out_bytes, dtype=torch.uint8, device=dev)
+        sl_ = {"din": din, "dout": dout, "hout": torch.empty(out_bytes, dtype=torch.uint8).pin_memory(),
+               "tile": torch.empty(nparts, ops.TILE_FIELDS, dtype=torch.int32, device=dev),
+               "splits": torch.empty(n_lists + 1, dtype=torch.int32, device=dev),
+               "ws": ops.new_workspace(ops.workspace_size(w.batch, w.s_q, w.h_q, w.h_kv, nparts), dev),
+               "up": torch.cuda.Event(), "done": torch.cuda.Event(), "back": torch.cuda.Event()}
+        sl_.update(views(din, in_offs))
+        sl_.update(views(dout, out_offs))
+        slots.append(sl_)
 
     def kernels(sl_):
         # the plan goes into this slot's buffers: the previous user of the slot (step i-2)
@@ -705,12 +720,7 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
         with torch.cuda.stream(up_stream):
             if i >= 2:
                 up_stream.wait_event(sl_["done"])  # step i-2's kernels have read this slot
-            sl_["q"].copy_(hq, non_blocking=True)
-            sl_["bt"].copy_(hbt, non_blocking=True)
-            sl_["sl"].copy_(hsl, non_blocking=True)
-            if sparse:
-                sl_["rp"].copy_(hrp, non_blocking=True)
-                sl_["ci"].copy_(hci, non_blocking=True)
+            sl_["din"].copy_(hin, non_blocking=True)
             sl_["up"].record(up_stream)
         kstream.wait_event(sl_["up"])
         if i >= 2:
@@ -720,8 +730,7 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
         sl_["done"].record(kstream)
         with torch.cuda.stream(down_stream):
             down_stream.wait_event(sl_["done"])
-            sl_["hout"].copy_(sl_["out"], non_blocking=True)
-            sl_["hlse"].copy_(sl_["lse"], non_blocking=True)
+            sl_["hout"].copy_(sl_["dout"], non_blocking=True)
             sl_["back"].record(down_stream)
 
     def e2e_run(n, e_start=None, e_end=None):
@@ -746,17 +755,15 @@ def e2e_leg(args, w, x, d0, dev, nparts, R, unit, total_bytes, total_flops, barr
     e2e_val = (total_bytes / e2e_s / 1e9) if unit == "GB/s" else (total_flops / e2e_s / 1e12)
     for sl_ in slots:
         sl_["graph"].reset()
-    hout, hlse = slots[0]["hout"], slots[0]["hlse"]
-    h2d = hq.numel() * 2 + hbt.numel() * 4 + hsl.numel() * 4
-    if sparse:
-        h2d += hrp.numel() * 4 + hci.numel() * 4
-    d2h = hout.numel() * 2 + hlse.numel() * 4
+    h2d = in_bytes
+    d2h = out_bytes
     return {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": e2e_s * 1e3, "steps_in_flight": 2,
-            "method": "pinned host buffers; per step: inputs up on an upload stream, the slot's scheduler, decode "
-                      "and combine calls (recorded once per slot through the public API in a CUDA graph) "
-                      "replayed, results down on a download stream; two slots, the host waiting for step "
-                      "i-1's result before issuing step i+1"}
+            "method": "pinned host buffers; per step: the inputs packed in one buffer go up in one copy on an "
+                      "upload stream, the slot's scheduler, decode and combine calls (recorded once per slot "
+                      "through the public API in a CUDA graph) are replayed on views of it, out and lse come "
+                      "down in one copy on a download stream; two slots, the host waiting for step i-1's "
+                      "result before issuing step i+1"}
 
 
 def load_for(graph, dev, seconds):
