@@ -121,14 +121,14 @@ int encode_q_map(CUtensorMap *map, const void *q, int batch, int s_q, int h_q, i
 }
 
 // FP8 latent cache codes [num_pages * 64 tokens][h_kv][576] bytes as a 3-D map (columns, latent
-// head, token); one box = 128 columns (128 bytes, 128-byte swizzle) x 1 head x 32 tokens.  A box
+// head, token); one box = 128 columns (128 bytes, 128-byte swizzle) x 1 head x 64 tokens.  A box
 // at column 512 reaches past column 575; TMA fills those columns with zeros.
 int encode_k8_map(CUtensorMap *map, const void *k8, int64_t num_pages, int h_kv) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(h_kv), cuuint64_t(num_pages) * kPage};
   cuuint64_t strides[2] = {cuuint64_t(kD), cuuint64_t(h_kv) * kD};
-  cuuint32_t box[3] = {128, 1, 32};
+  cuuint32_t box[3] = {128, 1, 64};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(k8), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -138,13 +138,13 @@ int encode_k8_map(CUtensorMap *map, const void *k8, int64_t num_pages, int h_kv)
 }
 
 // Token scales [h_kv][num_pages][64] fp32 as a 3-D map (slot, page, latent head); one box =
-// the 32 scales of a 32-token chunk.
+// the 64 scales of a page.
 int encode_scale_map(CUtensorMap *map, const float *k_scale, int64_t num_pages, int h_kv) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
   cuuint64_t dims[3] = {cuuint64_t(kPage), cuuint64_t(num_pages), cuuint64_t(h_kv)};
   cuuint64_t strides[2] = {cuuint64_t(kPage) * 4, cuuint64_t(num_pages) * kPage * 4};
-  cuuint32_t box[3] = {32, 1, 1};
+  cuuint32_t box[3] = {64, 1, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(k_scale), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,

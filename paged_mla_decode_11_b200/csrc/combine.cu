@@ -7,6 +7,13 @@
 // covers 512 contiguous bytes.  CTAs are small (4 warps) so that many of them are resident
 // as soon as the decode kernel's CTAs exit.
 //
+// Two instantiations: up to eight splits' rows in flight per warp at four CTAs per SM, for
+// grids of at most two such waves (the 16-row shapes: one wave, where fewer CTAs per SM
+// spread the grid over more SMs), and five splits at six CTAs per SM for larger grids (the
+// 128-row shapes: many waves of CTAs, each one or two round trips to L2 long, so more
+// resident warps matter more).  Measured alone: 2.7 against 3.1 us on the memory-bound
+// shape; 16.4 against 19.1 us (compute-bound) and 11.6 against 14.2 us (causal, s_q = 2).
+//
 // The kernel is launched early (programmatic dependent launch) and runs after the decode
 // kernel's last CTA, so its latency is the tail of every decode call.  It therefore reads
 // the plan before waiting for the decode kernel (the scheduler kernel wrote num_splits and
@@ -17,10 +24,11 @@
 namespace pagedmla {
 
 constexpr int kCombineWarps = 4;           // two rows x two column halves
-constexpr int kBatch = 8;                  // splits whose partial rows are loaded together
 
-// 4 CTAs per SM bound the registers to 128 per thread (eight splits' rows in flight).
-__global__ void __launch_bounds__(kCombineWarps * 32, 4)
+// kBatch: splits whose partial rows are loaded together; kCtas CTAs per SM bound the registers
+// (128 per thread for 8 splits at 4 CTAs, 85 for 5 at 6).
+template <int kBatch, int kCtas>
+__global__ void __launch_bounds__(kCombineWarps * 32, kCtas)
     combine_kernel(const int32_t *__restrict__ num_splits, int s_q, int h_q, int h_kv, int R, int sq_fold,
                    const float *__restrict__ lse_accum, const float *__restrict__ o_accum,
                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
@@ -37,7 +45,13 @@ __global__ void __launch_bounds__(kCombineWarps * 32, 4)
   // through the non-coherent read-only path.
   const int ns0 = __ldcg(num_splits + b);
   const int n = __ldcg(num_splits + b + 1) - ns0;
-  if (n <= 1 || row >= R) return;
+  if (n <= 1 || row >= R) {
+    // one CTA waits for the decode kernel even when nothing is split, so that this grid
+    // never completes before its predecessor (the next kernel in the stream may write the
+    // plan the decode kernel reads)
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) grid_dependency_wait();
+    return;
+  }
   const int g = h_q / h_kv;
   const int64_t stride = int64_t(h_kv) * R;  // between consecutive splits
   const int64_t base = (int64_t(ns0) * h_kv + kvh) * R + row;
@@ -117,7 +131,14 @@ cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_
                            float *lse, cudaStream_t stream, int sq_fold) {
   const int R = s_q * (h_q / h_kv);
   dim3 grid((R + kCombineWarps / 2 - 1) / (kCombineWarps / 2), batch, h_kv);
-  return launch_early(combine_kernel, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv, R,
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (int64_t(grid.x) * grid.y * grid.z <= int64_t(2) * 4 * sms)
+    return launch_early(combine_kernel<8, 4>, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv,
+                        R, sq_fold, lse_accum, o_accum, out, lse);
+  return launch_early(combine_kernel<5, 6>, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv, R,
                       sq_fold, lse_accum, o_accum, out, lse);
 }
 

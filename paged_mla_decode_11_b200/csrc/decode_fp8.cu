@@ -8,10 +8,12 @@
 // bytes of the bf16 cache stream from HBM.
 //
 // The kernel is the 16-row warp-MMA pipeline of the bf16 cache (producer, four S warps, one
-// softmax warp, four PV warps, chunks of 32 keys in a TMA ring) with these changes:
-//   - a chunk is 5 TMA boxes of 128 code columns x 32 tokens (128-byte swizzle; the last
-//     box's columns 576-639 lie outside the tensor and are filled with zeros) plus one box of
-//     the chunk's 32 scales;
+// softmax warp, four PV warps, chunks in a TMA ring) with these changes:
+//   - a chunk is a whole 64-token page: 5 TMA boxes of 128 code columns x 64 tokens
+//     (128-byte swizzle; the last box's columns 576-639 lie outside the tensor and are
+//     filled with zeros) plus one box of the page's 64 scales.  At half the bytes of a bf16
+//     page, twice the keys per chunk halve the stages' per-chunk costs (hand-offs between
+//     warps, the accumulator rescale), which bound this pipeline rather than HBM;
 //   - both MMAs run in f16 on the codes' exact f16 form (cvt.rn.f16x2.e4m3x2: one conversion
 //     per two codes, every E4M3 value being an f16 value); the query tile is carried in f16
 //     after a power-of-two scale of the tile (its largest |q| in [2^14, 2^15)), and P times
@@ -33,20 +35,20 @@
 namespace pagedmla {
 
 struct Fp8x16 {
-  static constexpr int KC = 32;                           // keys per chunk
-  static constexpr int NS = 6;                            // ring depth
+  static constexpr int KC = 64;                           // keys per chunk (one page)
+  static constexpr int NS = 4;                            // ring depth
   static constexpr int kSWarps = 4, kSmWarp = 4, kPVWarp0 = 5, kPVWarps = 4, kProducer = 9;
   static constexpr int kThreads = 10 * 32;
   static constexpr int kBoxes = 5;                        // 128-column boxes per chunk (576 -> 640)
-  static constexpr int kBoxBytes = KC * 128;              // 32 tokens x 128 codes: 4 KB
-  static constexpr int kChunkBytes = kBoxes * kBoxBytes;  // 20 KB
-  static constexpr int kScaleBytes = KC * 4;              // 32 fp32 scales
+  static constexpr int kBoxBytes = KC * 128;              // 64 tokens x 128 codes: 8 KB
+  static constexpr int kChunkBytes = kBoxes * kBoxBytes;  // 40 KB
+  static constexpr int kScaleBytes = KC * 4;              // 64 fp32 scales
   static constexpr int kOffRing = 0;
   static constexpr int kOffScale = kOffRing + NS * kChunkBytes;
   static constexpr int kOffQ = kOffScale + NS * 1024;     // 16 rows x 576 bf16, 9 blocks of 2 KB
-  static constexpr int kOffP = kOffQ + kColBlocks * 16 * 128;   // 2 x [16 rows x 32 keys] bf16
-  static constexpr int kOffS = kOffP + 2 * 16 * 128;            // 2 x [4 warps][8][32] f32 partial S
-  static constexpr int kOffAlpha = kOffS + 2 * 4 * 8 * 32 * 4;  // alpha[2][16]
+  static constexpr int kOffP = kOffQ + kColBlocks * 16 * 128;   // 2 x [16 rows x 64 keys] f16
+  static constexpr int kOffS = kOffP + 2 * 16 * 128;            // 2 x [4 warps][16][32] f32 partial S
+  static constexpr int kOffAlpha = kOffS + 2 * 4 * 16 * 32 * 4; // alpha[2][16]
   static constexpr int kOffL = kOffAlpha + 2 * 16 * 4;          // l[2 segs][16]
   static constexpr int kOffM = kOffL + 2 * 16 * 4;              // m[2 segs][16]
   static constexpr int kOffT = kOffM + 2 * 16 * 4;              // 2^-t of a segment's last chunk [2]
@@ -100,7 +102,8 @@ __device__ __forceinline__ void ldsm_x4_t_b8(uint32_t addr, uint32_t (&r)[4]) {
                : "r"(addr));
 }
 
-// Token range and 32-key chunk count of sequence `seq` within part `pc`.
+// Token range and page (chunk) count of sequence `seq` within part `pc` (part boundaries fall
+// on page multiples).
 __device__ __forceinline__ int fp8_chunk_range(const DecodeParams &p, const PartCursor &pc, int seq, int &L, int &t0,
                                                int &t1) {
   L = p.seqlens[seq];
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
       ++qs;
       const int32_t *bt_row = p.block_table + (int64_t)seq * p.bt_stride + t0 / kPage;
       for (int base = 0; ok && base < nch; base += 32) {
-        const int mine = base + lane < nch ? bt_row[(base + lane) >> 1] : 0;
+        const int mine = base + lane < nch ? bt_row[base + lane] : 0;
         const int cnt = min(32, nch - base);
         for (int i = 0; ok && i < cnt; ++i, ++it) {
           const int phys = __shfl_sync(0xffffffffu, mine, i);
@@ -191,13 +194,11 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
             } else {
               mbar_arrive_expect_tx(bar(T::FULL + s), T::kChunkBytes + T::kScaleBytes);
               const uint32_t dst = sRing + s * T::kChunkBytes;
-              const int half = (base + i) & 1;
-              const int row = phys * kPage + half * T::KC;
+              const int row = phys * kPage;
 #pragma unroll
               for (int c = 0; c < T::kBoxes; ++c)
                 tma_load_3d_hint(dst + c * T::kBoxBytes, &k8_map, bar(T::FULL + s), c * 128, kvh, row, policy);
-              tma_load_3d_hint(sbase + T::kOffScale + s * 1024, &scale_map, bar(T::FULL + s), half * T::KC, phys, kvh,
-                               policy);
+              tma_load_3d_hint(sbase + T::kOffScale + s * 1024, &scale_map, bar(T::FULL + s), 0, phys, kvh, policy);
               last_chunk[s] = it;
             }
           }
@@ -278,43 +279,49 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
       for (int n = 0; n < nch; ++n, ++it) {
         const int sb = it & 1;
         ok = ok && mbar_wait(bar(T::FULL + it % T::NS), (it / T::NS) & 1, abort, p.status, lim_ns);
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // this warp's 32 keys (kn * 32 ..) as four 8-key tiles: four independent accumulator
+        // chains per K step
+        float sc[4][4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[t][e] = 0.f;
         if (ok) {
           const uint32_t chunk = sRing + (it % T::NS) * T::kChunkBytes;
-          float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-          // matrix m of an x4 load: key tile m & 1 (keys kn*16 + 8 (m & 1) ..), K step k + (m >> 1)
-          const int m = lane >> 3, key = kn * 16 + (m & 1) * 8 + (lane & 7);
-          auto kaddr = [&](int k) {
+          // matrix m of an x4 load: key tile 2 h + (m & 1) (keys kn*32 + 16 h + 8 (m & 1) ..),
+          // K step k + (m >> 1)
+          const int m = lane >> 3;
+          auto kaddr = [&](int k, int h) {
+            const int key = kn * 32 + h * 16 + (m & 1) * 8 + (lane & 7);
             const int kc = k + (m >> 1);
             return chunk + (kc >> 3) * T::kBoxBytes + sw128(key, kc & 7);
           };
 #pragma unroll
           for (int kk = 0; kk < kD / 32; kk += 2) {
             const int k = kh * (kD / 32) + kk;
-            uint32_t r[4];
-            ldsm_x4_b8(kaddr(k), r);
+            uint32_t r[2][4];
+            ldsm_x4_b8(kaddr(k, 0), r[0]);
+            ldsm_x4_b8(kaddr(k, 1), r[1]);
 #pragma unroll
-            for (int dk = 0; dk < 2; ++dk) {
-              float(&a0)[4] = dk ? sd[0] : sc[0];
-              float(&a1)[4] = dk ? sd[1] : sc[1];
+            for (int dk = 0; dk < 2; ++dk)
 #pragma unroll
-              for (int nt = 0; nt < 2; ++nt) {
-                uint32_t b0, b1;
-                e4m3x4_to_f16x2x2(r[2 * dk + nt], b0, b1);
-                mma_f16_16816(nt ? a1 : a0, qf[kk + dk], b0, b1);
-              }
-            }
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                  uint32_t b0, b1;
+                  e4m3x4_to_f16x2x2(r[h][2 * dk + nt], b0, b1);
+                  mma_f16_16816(sc[2 * h + nt], qf[kk + dk], b0, b1);
+                }
           }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            sc[0][e] = (sc[0][e] + sd[0][e]) * qs_inv;
-            sc[1][e] = (sc[1][e] + sd[1][e]) * qs_inv;
-          }
+          for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[t][e] *= qs_inv;
         }
         if (it >= 2) named_bar_sync(T::kBarSEmpty + sb, T::kSPair);
-        float *dst = sbuf + (sb * 4 + warp) * 8 * 32;
+        float *dst = sbuf + (sb * 4 + warp) * 16 * 32;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dst[e * 32 + lane] = sc[e >> 2][e & 3];
+        for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = sc[e >> 2][e & 3];
         fp8_bar_arrive(T::kBarSFull + sb, T::kSPair);
       }
       ++qs;
@@ -338,24 +345,30 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
       for (int n = 0; n < nch; ++n, ++it) {
         const int sb = it & 1, pb = it & 1;
         named_bar_sync(T::kBarSFull + sb, T::kSPair);
-        // this thread's 16 scores: key halves kn = 0, 1; per half 2 key tiles x 4 values
-        float sc[2][8];
-        const float *src = sbuf + sb * 4 * 8 * 32;
+        // this thread's 32 scores: key halves kn = 0, 1; per half 4 key tiles x 4 values
+        // (value e of tile e >> 2: row g4 + 8 ((e >> 1) & 1), key 8 (e >> 2) + 2 c4 + (e & 1))
+        float sc[2][16];
+        const float *src = sbuf + sb * 4 * 16 * 32;
 #pragma unroll
         for (int kn = 0; kn < 2; ++kn)
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            sc[kn][e] = src[(kn * 8 + e) * 32 + lane] + src[((2 + kn) * 8 + e) * 32 + lane];
+          for (int e = 0; e < 16; ++e)
+            sc[kn][e] = src[(kn * 16 + e) * 32 + lane] + src[((2 + kn) * 16 + e) * 32 + lane];
         fp8_bar_arrive(T::kBarSEmpty + sb, T::kSPair);
-        // the chunk's token scales (landed with its codes; the S warps waited for them)
+        // the chunk's token scales (landed with its codes; the S warps waited for them); the
+        // slots past the piece's last token are not read, so that whatever the page holds
+        // there enters neither the chunk's scale factor nor a product with a zero probability
         const float *ksc = scale_sm + (it % T::NS) * 256;
-        float kscale[2][4];
+        float kscale[2][8];
 #pragma unroll
         for (int kn = 0; kn < 2; ++kn)
 #pragma unroll
-          for (int t = 0; t < 2; ++t)
+          for (int t = 0; t < 4; ++t)
 #pragma unroll
-            for (int u = 0; u < 2; ++u) kscale[kn][2 * t + u] = ksc[kn * 16 + t * 8 + c4 * 2 + u];
+            for (int u = 0; u < 2; ++u) {
+              const int kc = kn * 32 + t * 8 + c4 * 2 + u;
+              kscale[kn][2 * t + u] = t0 + n * T::KC + kc < t1 ? ksc[kc] : 0.f;
+            }
         // P V runs in f16: P times the key's scale times 2^t, with the power of two t of this
         // chunk chosen from its largest scale c so that every product (P <= 1) is below 2^15;
         // the accumulator carries the factor 2^t, changed between chunks through alpha
@@ -363,7 +376,7 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
 #pragma unroll
         for (int kn = 0; kn < 2; ++kn)
 #pragma unroll
-          for (int k = 0; k < 4; ++k) cmax = fmaxf(cmax, kscale[kn][k]);
+          for (int k = 0; k < 8; ++k) cmax = fmaxf(cmax, kscale[kn][k]);
         cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
         cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
         const int t_chunk = max(-120, min(120, 14 - (int((__float_as_uint(cmax) >> 23) & 0xff) - 127)));
@@ -375,10 +388,10 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
 #pragma unroll
         for (int kn = 0; kn < 2; ++kn)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < 16; ++e) {
             const int r = (e >> 1) & 1;
             const int kin = (e >> 2) * 2 + (e & 1);  // key tile * 2 + pair element
-            const int key = t0 + n * T::KC + kn * 16 + (e >> 2) * 8 + c4 * 2 + (e & 1);
+            const int key = t0 + n * T::KC + kn * 32 + (e >> 2) * 8 + c4 * 2 + (e & 1);
             const float v = key < lim[r] ? sc[kn][e] * kscale[kn][kin] * p.scale_log2 : -INFINITY;
             sc[kn][e] = v;
             mx[r] = fmaxf(mx[r], v);
@@ -399,14 +412,14 @@ __global__ void __launch_bounds__(Fp8x16::kThreads, 1)
 #pragma unroll
         for (int kn = 0; kn < 2; ++kn)
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
+          for (int t = 0; t < 4; ++t) {
             const float p0 = fast_exp2(sc[kn][t * 4 + 0] - base[0]), p1 = fast_exp2(sc[kn][t * 4 + 1] - base[0]);
             const float p2 = fast_exp2(sc[kn][t * 4 + 2] - base[1]), p3 = fast_exp2(sc[kn][t * 4 + 3] - base[1]);
             l[0] += p0 + p1;
             l[1] += p2 + p3;
             // the value row of a key is its scale times the codes: scale the probability
             const float s0 = kscale[kn][2 * t] * p_scale, s1 = kscale[kn][2 * t + 1] * p_scale;
-            const int kl = kn * 16 + t * 8 + c4 * 2;
+            const int kl = kn * 32 + t * 8 + c4 * 2;
             const __half2 h01 = __floats2half2_rn(p0 * s0, p1 * s1), h23 = __floats2half2_rn(p2 * s0, p3 * s1);
             asm volatile("st.shared.b32 [%0], %1;" ::"r"(ptile + sw128(g4, kl / 8) + (kl % 8) * 2),
                          "r"(*reinterpret_cast<const uint32_t *>(&h01)));

@@ -369,10 +369,12 @@ struct Mma16T {
   static constexpr int KC = 32;                           // keys per chunk
   static constexpr int NS = 5;                            // ring depth
   static constexpr int kSWarps = 4, kSmWarp = 4, kPVWarp0 = 5, kPVWarps = 4, kProducer = 9;
-  // sparse: a second producer warp; one warp's row copies are issued one request at a time
-  // and top out near 2.9 TB/s over the GPU, two reach about 5.1 TB/s (measured)
-  static constexpr int kProducer2 = 10;
-  static constexpr int kThreads = (kSparse ? 11 : 10) * 32;
+  // sparse: two producer warps (9 and 10), chunk `it` issued by warp 9 + it % 2.  One warp's
+  // row copies are issued one request at a time and top out near 2.9 TB/s over the GPU; two
+  // warps reach about 5.1 TB/s (measured).  A third warp measured slower (33.6 against
+  // 32.4 us on the random top-2048 workload): 162 registers, and the copies gain little.
+  static constexpr int kNP = kSparse ? 2 : 1;
+  static constexpr int kThreads = (kProducer + kNP) * 32;
   static constexpr int kChunkBlock = KC * 128;            // one 64-column block: 4 KB
   static constexpr int kChunkBytes = kColBlocks * kChunkBlock;  // bytes a chunk's copies deliver
   static constexpr int kRowBytes = kD * 2 + 16;           // sparse: padded row of a chunk
@@ -456,10 +458,10 @@ __global__ void __launch_bounds__(Mma16T<kSparse>::kThreads, 1)
   const PartCursor pc = load_part(p.tile_md, part);
   const int g4 = lane >> 2, c4 = lane & 3;
 
-  if (warp == T::kProducer || (kSparse && warp == T::kProducer2)) {
+  if (warp >= T::kProducer) {
     // ------------------------- producer: query tiles and key chunks -------------------------
-    // (sparse: producer pid takes the chunks with it % 2 == pid; the first also loads Q)
-    const int pid = warp == T::kProducer ? 0 : 1;
+    // (sparse: producer pid takes the chunks with it % kNP == pid; the first also loads Q)
+    const int pid = warp - T::kProducer;
     if (lane == 0) {
       prefetch_tensormap(&kv_map);
       prefetch_tensormap(&q_map);
@@ -533,7 +535,7 @@ __global__ void __launch_bounds__(Mma16T<kSparse>::kThreads, 1)
           for (int k = 0; k < 4; ++k) {
             const int n = grp * 4 + k;
             if (!ok || n >= nch) break;
-            if ((it & 1) != pid) {  // the other producer's chunk
+            if (it % T::kNP != pid) {  // another producer's chunk
               ++it;
               continue;
             }
