@@ -7,12 +7,15 @@
 // covers 512 contiguous bytes.  CTAs are small (4 warps) so that many of them are resident
 // as soon as the decode kernel's CTAs exit.
 //
-// Two instantiations: up to eight splits' rows in flight per warp at four CTAs per SM, for
-// grids of at most two such waves (the 16-row shapes: one wave, where fewer CTAs per SM
-// spread the grid over more SMs), and five splits at six CTAs per SM for larger grids (the
-// 128-row shapes: many waves of CTAs, each one or two round trips to L2 long, so more
-// resident warps matter more).  Measured alone: 2.7 against 3.1 us on the memory-bound
-// shape; 16.4 against 19.1 us (compute-bound) and 11.6 against 14.2 us (causal, s_q = 2).
+// Two instantiations: up to eight splits' rows in flight per warp at four CTAs per SM, and
+// five splits at six CTAs per SM.  The second serves grids of more than two waves with 128 or
+// more rows per latent head (the compute-bound shapes: a few dozen parts, so few splits per
+// sequence, and many waves of CTAs each one or two round trips to L2 long, where more
+// resident warps matter more); the first everything else: one-wave grids (fewer CTAs per SM
+// spread them over more SMs) and shapes with a sequence split many ways, whose merge is a
+// chain of batches on the step's critical path.  Measured in the whole step: compute-bound
+// 218.4-219.4 against 220.1-221.8 us, causal (s_q = 2) 220.2-221.4 against 221.8-222.6 us;
+// skewed (one sequence in 42 splits) 88.0-88.1 us with the first against 91.1-91.4 us.
 //
 // The kernel is launched early (programmatic dependent launch) and runs after the decode
 // kernel's last CTA, so its latency is the tail of every decode call.  It therefore reads
@@ -135,7 +138,7 @@ cudaError_t launch_combine(const int32_t *num_splits, int batch, int s_q, int h_
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  if (int64_t(grid.x) * grid.y * grid.z <= int64_t(2) * 4 * sms)
+  if (R < 128 || int64_t(grid.x) * grid.y * grid.z <= int64_t(2) * 4 * sms)
     return launch_early(combine_kernel<8, 4>, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv,
                         R, sq_fold, lse_accum, o_accum, out, lse);
   return launch_early(combine_kernel<5, 6>, grid, dim3(kCombineWarps * 32), 0, stream, num_splits, s_q, h_q, h_kv, R,
