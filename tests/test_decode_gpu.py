@@ -273,6 +273,29 @@ def test_all_sequences_empty(h_q):
     assert (out == 0).all()
 
 
+@pytest.mark.parametrize("h_q", [16, 128], ids=["16-row-kernel", "cta-pair-kernel"])
+def test_no_split_steps_back_to_back(h_q):
+    # One part per sequence (num_parts = batch, equal lengths): no sequence is split, so the
+    # combine finds nothing to merge (one of its CTAs still waits for the decode kernel).
+    # Three decodes of different inputs run back to back on one stream over one plan and
+    # one workspace, each checked element-wise afterwards.
+    b, lens = 8, [640] * 8
+    xs = [W.make_inputs(W.custom(b, 1, h_q, 1, lens, causal=True), seed=s) for s in (31, 32, 33)]
+    ds = [to_dev(x) for x in xs]
+    tile, splits = ops.get_mla_metadata(ds[0]["cache_seqlens"], h_q, 1, num_parts=b)
+    assert splits.cpu().tolist() == list(range(b + 1))
+    ws = ops.new_workspace(ops.workspace_size(b, 1, h_q, 1, tile.shape[0]), "cuda")
+    res = [ops.mla_decode_paged(d["q"], d["k_cache"], d["block_table"], d["cache_seqlens"], 512, tile, splits,
+                                softmax_scale=x["softmax_scale"], causal=True, workspace=ws)
+           for x, d in zip(xs, ds)]
+    torch.cuda.synchronize()
+    assert ops.query_status(ws) == ops.MLA_OK
+    for x, (out, lse) in zip(xs, res):
+        ref_out, ref_lse = oracle.mla_decode(x["q"], x["k_cache"], x["block_table"], x["cache_seqlens"],
+                                             dv=512, softmax_scale=x["softmax_scale"], causal=True)
+        assert_parity(out, lse, ref_out, ref_lse)
+
+
 def test_deterministic():
     x = W.make_inputs(W.custom(4, 1, 128, 1, [4000, 100, 2500, 64], causal=True), seed=10)
     a = run_gpu(x)
