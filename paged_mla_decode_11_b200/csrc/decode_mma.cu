@@ -362,8 +362,9 @@ __global__ void __launch_bounds__(MmaTile<BM, DVS>::kThreads, 1)
 // ---------------------------------------------------------------------------------------
 // Sparse variant (kSparse): the keys of a chunk are 32 listed token rows of one query token,
 // gathered row by row with untiled bulk copies into a row-major chunk (rows of 576 bf16
-// padded to 1,168 bytes, so that 8 consecutive rows of a ldmatrix fall in distinct banks);
-// the producer also records which of the 32 entries are real keys (a validity mask).
+// padded to 1,168 bytes, so that 8 consecutive rows of a ldmatrix fall in distinct banks) by
+// two producer warps taking alternate chunks; a producer also records which of the chunk's 32
+// entries are real keys (a validity mask).
 template <bool kSparse>
 struct Mma16T {
   static constexpr int KC = 32;                           // keys per chunk
