@@ -839,7 +839,7 @@ def measure_absorb(args, dev, group, cpu_seconds):
                      "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": f"{peak_kind} (hbm_gbs)", "kernel": "absorb_gemm_kernel (both products)",
                      "kernel_ms": per_step * 1e3,
-                     "kernel_timing": f"average over a graph of {args.steps} passes (three launches each)",
+                     "kernel_timing": f"average over a graph of {args.steps} passes (two launches each)",
                      "algorithmic_bytes_per_launch": nbytes, "algorithmic_flops_per_launch": flops,
                      "achieved_tflops": flops / per_step / 1e12},
         "clocks": clocks,

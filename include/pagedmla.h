@@ -306,7 +306,12 @@ MLA_API int mla_merge_partials(const void *o_parts, const float *lse_parts, int 
  *   out      device bf16 [tokens][heads][128], contiguous
  * bf16 inputs, fp32 accumulation (warp MMA), bf16 results; strides in elements, multiples of
  * 8; q_nope, q_rope, o_latent, the weights and q_out 16-byte aligned, out 4-byte aligned.
- * Errors: MLA_ERR_ARG, MLA_ERR_CUDA.
+ * Each call launches one kernel on `stream` as a programmatic dependent launch: it starts
+ * reading w_uk / w_uv while the kernel before it in the stream is still finishing, and reads
+ * the activations (q_nope, q_rope, o_latent) only after that kernel has completed.  So the
+ * weights must not be written by that kernel (a kernel that writes them and signals
+ * programmatic dependents must do so after those writes); ordinary launches and copies are
+ * always waited for.  Errors: MLA_ERR_ARG, MLA_ERR_CUDA.
  */
 MLA_API int mla_absorb_query(const void *q_nope, const int64_t nope_strides[2], const void *q_rope,
                              const int64_t rope_strides[2], const void *w_uk, int tokens, int heads, void *q_out,

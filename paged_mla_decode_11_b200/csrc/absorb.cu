@@ -11,8 +11,14 @@
 // they run on warp MMA (mma.sync m16n8k16 bf16, fp32 accumulate): a CTA computes a 64-token x
 // BN-column tile of one head (BN = 128 for q', 64 for the output), its four warps 16 tokens x
 // BN columns each, over K chunks of 64 staged in shared memory by cp.async (three stages: two
-// chunks load while one is multiplied).  Tile rows are padded by 16 bytes, so the 8 rows of
-// an ldmatrix fall in distinct banks.
+// chunks load while one is multiplied; q' has only two chunks, so its launch gives the
+// kernel two stages of shared memory and twice as many CTAs fit on an SM).  Tile rows are
+// padded by 16 bytes, so the 8 rows of an ldmatrix fall in distinct banks.
+//
+// Both kernels are programmatic dependent launches: a CTA issues the copies of its weight
+// tiles (model parameters, written long before) before it waits for the previous kernel in
+// the stream, and the activation tiles after, so the weight reads overlap that kernel's
+// tail.  The q' kernel's first column block also copies the rope columns of its tokens.
 #include "launch.h"
 
 namespace pagedmla {
@@ -42,11 +48,14 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // B given as [K][N] (W^UK: k = d, n = latent column) when kKN, else as [N][K] (W^UV: n = d,
 // k = latent column).  M, N, K: tokens (any), columns (a multiple of BN), contraction (a
 // multiple of 64).
+// rope (q' only): q_rope, element (t, h, c) at t * r_row + h * r_head + c, copied into columns
+// 512..575 of C's rows (blockIdx.x == 0 only); nullptr for the output product.
 template <bool kKN, int BN>
 __global__ void __launch_bounds__(kAbWarps * 32)
     absorb_gemm_kernel(const __nv_bfloat16 *__restrict__ A, int64_t a_row, int64_t a_head,
                        const __nv_bfloat16 *__restrict__ B, __nv_bfloat16 *__restrict__ C, int64_t c_row,
-                       int64_t c_head, int M, int N, int K) {
+                       int64_t c_head, int M, int N, int K, const __nv_bfloat16 *__restrict__ rope, int64_t r_row,
+                       int64_t r_head) {
   using T = AbsorbTile<kKN, BN>;
   extern __shared__ __align__(16) uint8_t absorb_smem[];
   const uint32_t sbase = smem_u32(absorb_smem);
@@ -55,13 +64,17 @@ __global__ void __launch_bounds__(kAbWarps * 32)
   const int n0 = blockIdx.x * BN, h = blockIdx.y, m0 = blockIdx.z * kAbBM;
   const __nv_bfloat16 *Ah = A + int64_t(h) * a_head;
   const __nv_bfloat16 *Bh = B + int64_t(h) * K * N;
+  grid_launch_dependents();  // the next kernel may start its prologue
 
-  auto load_stage = [&](int st, int k0) {
-    const uint32_t sa = sbase + st * T::kStage, sb = sa + T::kABytes;
+  auto load_a = [&](int st, int k0) {
+    const uint32_t sa = sbase + st * T::kStage;
     for (int i = tid; i < kAbBM * (kAbBK / 8); i += kAbWarps * 32) {
       const int r = i / (kAbBK / 8), c = i % (kAbBK / 8), t = m0 + r;
       cp_async16_zfill(sa + r * T::kARow + c * 16, Ah + int64_t(min(t, M - 1)) * a_row + k0 + c * 8, t < M ? 16u : 0u);
     }
+  };
+  auto load_b = [&](int st, int k0) {
+    const uint32_t sb = sbase + st * T::kStage + T::kABytes;
     if constexpr (kKN) {
       for (int i = tid; i < kAbBK * (BN / 8); i += kAbWarps * 32) {
         const int r = i / (BN / 8), c = i % (BN / 8);
@@ -73,26 +86,43 @@ __global__ void __launch_bounds__(kAbWarps * 32)
         cp_async16_zfill(sb + r * T::kBRow + c * 16, Bh + int64_t(n0 + r) * K + k0 + c * 8, 16u);
       }
     }
-    cp_async_commit();
   };
 
   float acc[BN / 8][4];
 #pragma unroll
   for (int j = 0; j < BN / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
   const int nk = K / kAbBK;
-  // one commit group per chunk (empty past the end), so "all but the newest S - 2 groups
-  // landed" means chunk kc has landed
+  // One commit group per chunk (empty past the end), so "all but the newest S - 2 groups
+  // landed" means chunk kc has landed.  The prologue's weight copies are issued before the
+  // dependency wait and fall into the first group, which is older than any of their chunks.
+#pragma unroll
+  for (int st = 0; st < kAbStages - 1; ++st)
+    if (st < nk) load_b(st, st * kAbBK);
+  grid_dependency_wait();  // the activations may come from the kernel just before
 #pragma unroll
   for (int st = 0; st < kAbStages - 1; ++st) {
-    if (st < nk) load_stage(st, st * kAbBK);
-    else cp_async_commit();
+    if (st < nk) load_a(st, st * kAbBK);
+    cp_async_commit();
+  }
+  if constexpr (kKN) {
+    // the rope columns pass through: 64 tokens x 8 chunks of 16 bytes, while the copies fly
+    if (blockIdx.x == 0)
+      for (int i = tid; i < kAbBM * 8; i += kAbWarps * 32) {
+        const int t = m0 + i / 8, c = i % 8;
+        if (t < M)
+          *reinterpret_cast<uint4 *>(C + int64_t(h) * c_head + int64_t(t) * c_row + 512 + 8 * c) =
+              *reinterpret_cast<const uint4 *>(rope + t * r_row + h * r_head + 8 * c);
+      }
   }
   for (int kc = 0; kc < nk; ++kc) {
     cp_async_wait<kAbStages - 2>();
     __syncthreads();  // chunk kc is visible to all warps; chunk kc - 1's stage is free
     const int kn = kc + kAbStages - 1;
-    if (kn < nk) load_stage(kn % kAbStages, kn * kAbBK);
-    else cp_async_commit();
+    if (kn < nk) {
+      load_a(kn % kAbStages, kn * kAbBK);
+      load_b(kn % kAbStages, kn * kAbBK);
+    }
+    cp_async_commit();
     const uint32_t sa = sbase + (kc % kAbStages) * T::kStage, sb = sa + T::kABytes;
 #pragma unroll
     for (int ks = 0; ks < kAbBK / 16; ++ks) {
@@ -123,31 +153,17 @@ __global__ void __launch_bounds__(kAbWarps * 32)
   }
 }
 
-// Copies q_rope into columns 512-575 of q' (8 bf16 per thread).
-__global__ void rope_copy_kernel(const __nv_bfloat16 *__restrict__ q_rope, int64_t r_row, int64_t r_head,
-                                 __nv_bfloat16 *__restrict__ q_out, int T, int H) {
-  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;  // (t, h, 8-column chunk)
-  if (i >= int64_t(T) * H * 8) return;
-  const int c = int(i % 8), h = int((i / 8) % H), t = int(i / (8 * H));
-  const uint4 v = *reinterpret_cast<const uint4 *>(q_rope + t * r_row + h * r_head + 8 * c);
-  *reinterpret_cast<uint4 *>(q_out + (int64_t(t) * H + h) * kD + 512 + 8 * c) = v;
-}
-
 cudaError_t launch_absorb_q(const __nv_bfloat16 *q_nope, int64_t n_row, int64_t n_head, const __nv_bfloat16 *q_rope,
                             int64_t r_row, int64_t r_head, const __nv_bfloat16 *w_uk, __nv_bfloat16 *q_out, int T,
                             int H, cudaStream_t stream) {
   constexpr int kBN = 128;
-  constexpr int kSmem = AbsorbTile<true, kBN>::kSmem;
+  // K = 128: two chunks, stages 0 and 1 only (the third stage of the ring is never reached)
+  constexpr int kSmem = 2 * AbsorbTile<true, kBN>::kStage;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(absorb_gemm_kernel<true, kBN>), kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(512 / kBN, H, (T + kAbBM - 1) / kAbBM);
-  absorb_gemm_kernel<true, kBN><<<grid, kAbWarps * 32, kSmem, stream>>>(q_nope, n_row, n_head, w_uk, q_out,
-                                                                   int64_t(H) * kD, kD, T, 512, 128);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int64_t n = int64_t(T) * H * 8;
-  rope_copy_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(q_rope, r_row, r_head, q_out, T, H);
-  return cudaGetLastError();
+  return launch_early(absorb_gemm_kernel<true, kBN>, grid, dim3(kAbWarps * 32), kSmem, stream, q_nope, n_row, n_head,
+                      w_uk, q_out, int64_t(H) * kD, int64_t(kD), T, 512, 128, q_rope, r_row, r_head);
 }
 
 cudaError_t launch_absorb_out(const __nv_bfloat16 *o_lat, int64_t l_row, int64_t l_head, const __nv_bfloat16 *w_uv,
@@ -157,9 +173,9 @@ cudaError_t launch_absorb_out(const __nv_bfloat16 *o_lat, int64_t l_row, int64_t
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(absorb_gemm_kernel<false, kBN>), kSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(128 / kBN, H, (T + kAbBM - 1) / kAbBM);
-  absorb_gemm_kernel<false, kBN><<<grid, kAbWarps * 32, kSmem, stream>>>(o_lat, l_row, l_head, w_uv, out,
-                                                                    int64_t(H) * 128, 128, T, 128, 512);
-  return cudaGetLastError();
+  return launch_early(absorb_gemm_kernel<false, kBN>, grid, dim3(kAbWarps * 32), kSmem, stream, o_lat, l_row, l_head,
+                      w_uv, out, int64_t(H) * 128, int64_t(128), T, 128, 512,
+                      static_cast<const __nv_bfloat16 *>(nullptr), int64_t(0), int64_t(0));
 }
 
 }  // namespace pagedmla
