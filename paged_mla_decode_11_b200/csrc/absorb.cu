@@ -34,6 +34,7 @@ struct AbsorbTile {
   static constexpr int kBBytes = kKN ? kAbBK * kBRow : BN * kBRow;
   static constexpr int kStage = kABytes + kBBytes;
   static constexpr int kSmem = kAbStages * kStage;
+  static_assert(!kKN || kAbWarps * 16 * (BN * 2 + 16) <= 2 * kStage, "q' output staging fits in two stages");
 };
 
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_bytes) {
@@ -142,14 +143,41 @@ __global__ void __launch_bounds__(kAbWarps * 32)
       }
     }
   }
+  if constexpr (kKN) {
+    // q' (16-byte aligned): the warp's 16 x BN tile goes through shared memory (rows padded by
+    // 16 bytes: the 8 rows of a fragment store fall in distinct banks) and leaves as 16-byte
+    // stores, each warp instruction covering two whole 256-byte row segments
+    constexpr int kORow = BN * 2 + 16, kChunks = BN / 8;
+    __syncthreads();  // every warp has finished reading the ring
+    const uint32_t so = sbase + warp * 16 * kORow;
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int t = m0 + warp * 16 + g4 + 8 * r;
-    if (t >= M) continue;
-    __nv_bfloat16 *crow = C + int64_t(h) * c_head + int64_t(t) * c_row + n0 + 2 * c4;
+    for (int r = 0; r < 2; ++r)
 #pragma unroll
-    for (int j = 0; j < BN / 8; ++j)
-      *reinterpret_cast<uint32_t *>(crow + 8 * j) = pack_bf16x2(acc[j][2 * r], acc[j][2 * r + 1]);
+      for (int j = 0; j < BN / 8; ++j)
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(so + (g4 + 8 * r) * kORow + (j * 8 + 2 * c4) * 2),
+                     "r"(pack_bf16x2(acc[j][2 * r], acc[j][2 * r + 1])));
+    __syncwarp();
+#pragma unroll
+    for (int q = lane; q < 16 * kChunks; q += 32) {
+      const int row = q / kChunks, c = q % kChunks, t = m0 + warp * 16 + row;
+      if (t >= M) continue;
+      uint32_t v0, v1, v2, v3;
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                   : "r"(so + row * kORow + c * 16));
+      *reinterpret_cast<uint4 *>(C + int64_t(h) * c_head + int64_t(t) * c_row + n0 + 8 * c) = make_uint4(v0, v1, v2, v3);
+    }
+  } else {
+    // the output (4-byte aligned): fragment stores straight from the accumulators
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int t = m0 + warp * 16 + g4 + 8 * r;
+      if (t >= M) continue;
+      __nv_bfloat16 *crow = C + int64_t(h) * c_head + int64_t(t) * c_row + n0 + 2 * c4;
+#pragma unroll
+      for (int j = 0; j < BN / 8; ++j)
+        *reinterpret_cast<uint32_t *>(crow + 8 * j) = pack_bf16x2(acc[j][2 * r], acc[j][2 * r + 1]);
+    }
   }
 }
 
