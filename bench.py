@@ -44,6 +44,7 @@ import statistics
 import subprocess
 import sys
 import time
+from typing import Optional
 
 import torch
 
@@ -65,6 +66,7 @@ KERNEL_SOURCES = {
     "decode_wide_kernel": ["common.cuh", "decode_wide.cu"],
     "decode_pair_kernel": ["common.cuh", "decode_pair.cu"],
     "decode_fp8_kernel": ["common.cuh", "decode_fp8.cu"],
+    "absorb_gemm_kernel": ["common.cuh", "absorb.cu"],
 }
 
 
@@ -153,10 +155,11 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str, kernel: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on
-    the current sources of that decode kernel; None otherwise."""
-    path = os.path.join(ROOT, "profiles", f"decode_{workload}_ncu.md")
+def recorded_traffic(workload: str, kernel: str, summary: Optional[str] = None):
+    """DRAM bytes per decode launch (per pass of both products for the absorption) from the
+    committed ncu summary, if it was taken on the current sources of that kernel; None
+    otherwise."""
+    path = os.path.join(ROOT, "profiles", summary or f"decode_{workload}_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -836,7 +839,8 @@ def measure_absorb(args, dev, group, cpu_seconds):
                                f"~N(0,1) bf16, seed {args.seed}"},
         "unit": "GB/s", "value": achieved, "ms_per_step": per_step * 1e3,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": recorded_traffic("absorb", "absorb_gemm_kernel", "absorb_ncu.md"),
                      "peak_source": f"{peak_kind} (hbm_gbs)", "kernel": "absorb_gemm_kernel (both products)",
                      "kernel_ms": per_step * 1e3,
                      "kernel_timing": f"average over a graph of {args.steps} passes (two launches each)",
@@ -938,6 +942,15 @@ def run_ours(args):
     dev = torch.device("cuda", local_rank)
     group = RankGroup("nccl", dev)
 
+    if args.only:
+        # one supporting product alone (one GPU), e.g. as the command a profiler runs
+        if world != 1:
+            raise SystemExit("--only runs on one GPU")
+        fn = measure_absorb if args.only == "absorb" else measure_merge
+        r = fn(args, dev, group, cpu_seconds=0.0 if args.no_cpu_baseline else 2.0)
+        group.close()
+        print(json.dumps({"only": args.only, **r}), flush=True)
+        return
     head = measure(args.workload, args, dev, group, rank, world, with_e2e=True, cpu_seconds=10.0)
     # every workload of the specification on the same line (one GPU only: at N > 1 the
     # per-rank work is the headline workload alone)
@@ -988,6 +1001,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="measure only --workload (by default one GPU also measures every workload)")
+    ap.add_argument("--only", choices=["absorb", "shard_merge"],
+                    help="measure one supporting product alone and print its result (one GPU)")
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "warp_mma"],
                     help="decode kernel choice (auto = the library's choice by shape)")
     args = ap.parse_args()
