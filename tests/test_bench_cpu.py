@@ -67,6 +67,31 @@ def test_traffic_follows_the_kernel_code(bench, monkeypatch, tmp_path, workload,
     assert bench.recorded_traffic(workload, kernel) is None
 
 
+def test_absorb_traffic_follows_the_kernel_code(bench, monkeypatch, tmp_path):
+    root = _copy_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    path = root / "profiles" / "absorb_ncu.md"
+    text = path.read_text()
+    recorded = float(re.search(r"traffic_bytes_per_launch:\s*(\S+)", text).group(1))
+    stamped = re.sub(r"kernel_source_hash: \S+",
+                     "kernel_source_hash: " + bench.kernel_source_hash("absorb_gemm_kernel"), text)
+    path.write_text(stamped)
+    assert bench.recorded_traffic("absorb", "absorb_gemm_kernel", "absorb_ncu.md") == recorded
+    src = root / "paged_mla_decode_11_b200" / "csrc" / "absorb.cu"
+    src.write_text(src.read_text() + "\nstatic int unused_marker_for_the_test;\n")
+    assert bench.recorded_traffic("absorb", "absorb_gemm_kernel", "absorb_ncu.md") is None
+
+
+def test_committed_absorb_traffic_is_the_algorithmic_reads(bench):
+    # the two products read every weight and activation byte once (their 23 MB of results
+    # stay in L2 while they run, so the capture counts reads only)
+    T, H = bench.ABSORB_TOKENS, bench.ABSORB_HEADS
+    text = open(os.path.join(ROOT, "profiles", "absorb_ncu.md")).read()
+    traffic = float(re.search(r"traffic_bytes_per_launch:\s*(\S+)", text).group(1))
+    reads = 2 * (T * H * 128 + T * H * 64 + H * 128 * 512 + T * H * 512 + H * 128 * 512)
+    assert 0.999 <= traffic / reads <= 1.01
+
+
 @pytest.mark.parametrize("workload,lo,hi", [("memory_bound", 0.99, 1.05), ("compute_bound", 0.99, 1.10)])
 def test_committed_traffic_is_close_to_the_algorithmic_bytes(bench, workload, lo, hi):
     # whatever kernel version it was taken on, a committed figure far from the algorithmic
