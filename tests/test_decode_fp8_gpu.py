@@ -55,7 +55,7 @@ def fp8_parity(x, **kw):
 FP8_CASES = [
     # (batch, s_q, h_q, h_kv, seqlens, causal)
     (2, 1, 16, 1, [37, 130], True),                 # the tiny decode shape
-    (5, 1, 16, 1, [1, 31, 32, 33, 300], False),     # ragged ends around 32-token chunks
+    (5, 1, 16, 1, [1, 31, 32, 33, 300], False),     # ragged ends around half pages
     (3, 1, 16, 1, [0, 5, 0], True),                 # empty sequences
     (2, 2, 8, 1, [1, 66], True),                    # causal multi-token, a row with no visible key
     (2, 1, 32, 2, [100, 200], False),               # two latent heads
@@ -129,6 +129,26 @@ def test_fp8_full_size_memory_bound():
     x = W.make_inputs_fp8(W.WORKLOADS["memory_bound"], seed=0)
     err = fp8_parity(x)
     print(f"memory_bound fp8: out_err_over_max_ref {err:.3e}")
+
+
+def test_fp8_tail_scales_are_not_read():
+    # A sequence's last page holds slots past its length.  They are not keys, so whatever
+    # scales they hold (here NaN and inf) enter neither a chunk's power-of-two factor nor a
+    # product with a zero probability: the result equals the oracle's on clean scales.
+    x = W.make_inputs_fp8(W.custom(4, 1, 16, 1, [37, 130, 69, 64], causal=True), seed=17)
+    ref_out, ref_lse = oracle.mla_decode_fp8(x["q"], x["k8"], x["k_scale"], x["block_table"], x["cache_seqlens"],
+                                             dv=512, softmax_scale=x["softmax_scale"], causal=True)
+    ks = x["k_scale"].clone()
+    for b, L in enumerate(x["cache_seqlens"].tolist()):
+        if L % 64:
+            page = int(x["block_table"][b, (L - 1) // 64])
+            ks[:, page, L % 64:] = float("nan") if b % 2 == 0 else float("inf")
+    out, lse, _, _, _ = run_fp8(dict(x, k_scale=ks))
+    o = out.double().cpu().numpy()
+    l = lse.double().cpu().numpy()
+    assert np.isfinite(o).all() and np.isfinite(l).all()
+    assert np.abs(o - ref_out).max() <= OUT_TOL * np.abs(ref_out).max()
+    assert (np.abs(l - ref_lse) / np.maximum(np.abs(ref_lse), 1.0)).max() <= LSE_RTOL
 
 
 def test_fp8_rejects_more_than_16_rows():
