@@ -200,10 +200,14 @@ MLA_API int mla_decode_paged(const void *q, const int64_t q_strides[3], int batc
  *   k_scale   device fp32 [h_kv][num_pages][page_size]: one scale per token and latent head,
  *             contiguous, 16-byte aligned
  * and the latent row a token contributes (to the score and, first dv columns, to the
- * value) is k_scale * e4m3(k8).  Codes are widened to bf16 exactly in the kernel; all other
- * arguments, layouts, results and errors as in mla_decode_paged (flags: 0 or
- * MLA_FLAG_SKIP_COMBINE; the same workspace size and the same mla_combine).  Errors also:
- * MLA_ERR_UNSUPPORTED for more than 16 rows per latent head.
+ * value) is k_scale * e4m3(k8).  Codes are widened exactly in the kernel (every E4M3 value
+ * is an f16 value) and both products run on f16 tensor-core MMAs with fp32 accumulation, the
+ * query and the probabilities carried in f16 after power-of-two scalings.  The slots of a
+ * sequence's last page past its length are not keys: their scales are never read, their
+ * codes are read and must not be NaN (any finite code).  All other arguments, layouts,
+ * results and errors as in mla_decode_paged (flags: 0 or MLA_FLAG_SKIP_COMBINE; the same
+ * workspace size and the same mla_combine).  Errors also: MLA_ERR_UNSUPPORTED for more than
+ * 16 rows per latent head.
  */
 MLA_API int mla_decode_paged_fp8(const void *q, const int64_t q_strides[3], int batch, int s_q, int h_q,
                                  int d, const void *k8, const float *k_scale, int64_t num_pages,
