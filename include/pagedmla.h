@@ -275,8 +275,8 @@ MLA_API int mla_combine(const int32_t *num_splits, int batch, int s_q, int h_q, 
  * mla_merge_partials -- log-sum-exp merge of n_parts partial decodes of the same query rows,
  * each over a disjoint part of the keys (a sequence sharded over GPUs: every GPU decodes its
  * shard of the pages with mla_decode_paged, the (out, lse) of all shards are gathered, then
- * merged here).  The merge is the combine's (north_star: "split-KV partials are merged by a
- * log-sum-exp combine"): lse = ln sum_k exp(lse_k), out = sum_k exp(lse_k - lse) out_k;
+ * merged here).  The merge is mla_combine's log-sum-exp merge, applied across GPUs instead of
+ * across the splits of one GPU: lse = ln sum_k exp(lse_k), out = sum_k exp(lse_k - lse) out_k;
  * partials with lse_k = -inf weigh nothing; rows with no key in any part get out = 0 and
  * lse = -inf.
  *   o_parts    device bf16 [n_parts][batch][s_q][h_q][dv], contiguous, 16-byte aligned
